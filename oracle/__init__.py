@@ -1,0 +1,110 @@
+"""fp64 CPU oracle for residual binarization -- TEST INFRASTRUCTURE ONLY.
+
+Only the tests, the package's smoke check and the bench's CPU-baseline leg may
+import this module. The product (the CUDA library and its Python binding)
+never imports it and shares no code with it.
+
+The arithmetic lives in ``rb_oracle.c`` (plain C, fp64, OpenMP over rows);
+this wrapper only converts numpy arrays and loads the shared object, building
+it with gcc on first use. See ``rb_oracle.c`` for the passages each function
+follows.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "rb_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile rb_oracle.c into liboracle.so (gcc, -O2, OpenMP, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared",
+                               "-fno-fast-math", "-ffp-contract=off", _SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            p = ctypes.c_void_p
+            i64, i32 = ctypes.c_int64, ctypes.c_int32
+            lib.rbo_pack.argtypes = [p, i64, i64, i32, i64, p, p, p]
+            lib.rbo_pack.restype = ctypes.c_int
+            lib.rbo_matvec.argtypes = [p, p, i64, i64, i32, i64, p, i64, p, p]
+            lib.rbo_matvec.restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def pack(W: np.ndarray, n_paths: int, group: int = 0, want_rabs: bool = False):
+    """Derive N residual sign planes and scales from one weight matrix.
+
+    W: (M, K) float16/float32/float64. group: 0 for one scale per row, else the
+    number of columns per scale. Returns (planes uint32 [N, M, K/32],
+    alpha float64 [N, M, K/G], rabs float64 [N, M, K] or None).
+    """
+    W = np.ascontiguousarray(W, dtype=np.float64)
+    M, K = W.shape
+    G = K if group == 0 else group
+    planes = np.zeros((n_paths, M, K // 32), dtype=np.uint32)
+    alpha = np.zeros((n_paths, M, K // G), dtype=np.float64)
+    rabs = np.zeros((n_paths, M, K), dtype=np.float64) if want_rabs else None
+    rc = _load().rbo_pack(_ptr(W), M, K, n_paths, G, _ptr(planes), _ptr(alpha),
+                          _ptr(rabs) if rabs is not None else None)
+    if rc != 0:
+        raise ValueError(f"bad shape M={M} K={K} N={n_paths} G={G}")
+    return planes, alpha, rabs
+
+
+def matvec(planes: np.ndarray, alpha: np.ndarray, x: np.ndarray):
+    """y[t, i] = sum_k sum_j alpha_k[i, g(j)] * (+-1) * x[t, j] and its tolerance scale.
+
+    planes uint32 [N, M, K/32]; alpha [N, M, K/G] (any float dtype, widened to
+    fp64); x [T, K]. Returns (y float64 [T, M], denom float64 [T, M]).
+    """
+    planes = np.ascontiguousarray(planes, dtype=np.uint32)
+    alpha = np.ascontiguousarray(alpha, dtype=np.float64)
+    x = np.ascontiguousarray(np.atleast_2d(x), dtype=np.float64)
+    N, M, W32 = planes.shape
+    K = W32 * 32
+    G = K // alpha.shape[2]
+    T = x.shape[0]
+    if x.shape[1] != K or alpha.shape[:2] != (N, M):
+        raise ValueError("shape mismatch")
+    y = np.zeros((T, M), dtype=np.float64)
+    den = np.zeros((T, M), dtype=np.float64)
+    rc = _load().rbo_matvec(_ptr(planes), _ptr(alpha), M, K, N, G, _ptr(x), T, _ptr(y), _ptr(den))
+    if rc != 0:
+        raise ValueError("bad shape")
+    return y, den
+
+
+def alpha_to_f16(alpha: np.ndarray) -> np.ndarray:
+    """Round fp64 scales to the nearest fp16 (ties to even): the stored fp16 copy."""
+    return np.asarray(alpha, dtype=np.float64).astype(np.float16)
+
+
+from .compare import (  # noqa: E402,F401
+    compare_planes,
+    compare_scales,
+    compare_scales_f16,
+    compare_outputs,
+)

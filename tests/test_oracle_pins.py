@@ -1,0 +1,318 @@
+"""Pins of the fp64 oracle to facts that do not come from the oracle itself.
+
+* brute force over every sign pattern and a scale search on short rows
+  (the scale and sign choice are the least-squares optimum for one path,
+  and every later path is the optimum for the residual the earlier ones left);
+* hand-worked derivations and packed-word fixtures under tests/golden/;
+* invariants the derivation implies (energy identity, orthogonality of the
+  residual to the last sign plane, non-increasing residual norm);
+* the N = 1 special case (plain sign binarisation with a mean-|w| scale);
+* the matvec against a dense BLAS product, closed forms for x = 1 and x = e_j;
+* population values for Gaussian and Student-t rows (quadrature, not sampling);
+* the paper's storage ratios (RaBiT section 4.1 and 5, appendix D).
+"""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _signs(planes):
+    b = np.ascontiguousarray(planes, dtype="<u4").view(np.uint8)
+    bits = np.unpackbits(b, axis=-1, bitorder="little").reshape(planes.shape[0], planes.shape[1], -1)
+    return np.where(bits == 1, 1.0, -1.0)
+
+
+def _residuals(W, planes, alpha, G):
+    """R_k for k = 0..N rebuilt from the oracle's outputs (numpy, not the oracle)."""
+    S = _signs(planes)
+    N = S.shape[0]
+    A = np.repeat(alpha, G, axis=2)
+    R = [W.astype(np.float64)]
+    for k in range(N):
+        R.append(R[-1] - A[k] * S[k])
+    return R
+
+
+def _best_scale_objective(r, s):
+    """min over a >= 0 of ||r - a s||^2 by a grid plus golden-section search."""
+    hi = float(np.max(np.abs(r))) * 1.5 + 1e-12
+    f = lambda a: float(np.sum((r - a * s) ** 2))
+    grid = np.linspace(0.0, hi, 401)
+    vals = np.array([f(a) for a in grid])
+    m = int(np.argmin(vals))
+    lo_, hi_ = grid[max(m - 1, 0)], grid[min(m + 1, len(grid) - 1)]
+    g = (math.sqrt(5) - 1) / 2
+    c, d = hi_ - g * (hi_ - lo_), lo_ + g * (hi_ - lo_)
+    for _ in range(200):
+        if f(c) < f(d):
+            hi_ = d
+        else:
+            lo_ = c
+        c, d = hi_ - g * (hi_ - lo_), lo_ + g * (hi_ - lo_)
+    a = (lo_ + hi_) / 2
+    return f(a), a
+
+
+@pytest.mark.parametrize("seed", [1, 2, 3])
+def test_brute_force_one_path_is_optimal(seed):
+    """(sign(r), mean|r|) attains the global least-squares optimum over all
+    2^n sign patterns and every scale a >= 0 (n = 10 free columns; the other
+    22 columns of the 32-column group are zero and cost a^2 each whatever
+    their sign)."""
+    rng = np.random.default_rng(seed)
+    n = 10
+    r = rng.standard_normal(n)
+    r[3] = 0.0
+    W = np.zeros((1, 32))
+    W[0, :n] = r
+    planes, alpha, _ = oracle.pack(W, 1, 32)
+    s_or, a_or = _signs(planes)[0, 0], alpha[0, 0, 0]
+    best, best_s = math.inf, None
+    for bits in itertools.product((1.0, -1.0), repeat=n):
+        s = np.concatenate([np.array(bits), np.ones(32 - n)])
+        v, _ = _best_scale_objective(W[0], s)
+        if v < best:
+            best, best_s = v, s
+    v_or = float(np.sum((W[0] - a_or * s_or) ** 2))
+    assert v_or <= best * (1 + 1e-10) + 1e-14
+    nz = r != 0
+    assert np.all(best_s[:n][nz] == s_or[:n][nz])
+    # on a dense 32-column row, no single sign flip (with its own best scale) does better
+    base = np.tile(r, 4)[:32]
+    planes, alpha, _ = oracle.pack(base[None, :], 1, 32)
+    s0, a0 = _signs(planes)[0, 0], alpha[0, 0, 0]
+    v0 = float(np.sum((base - a0 * s0) ** 2))
+    for j in range(32):
+        s2 = s0.copy()
+        s2[j] = -s2[j]
+        v2, _ = _best_scale_objective(base, s2)
+        assert v0 <= v2 * (1 + 1e-12) + 1e-15
+
+
+@pytest.mark.parametrize("seed", [4, 5])
+def test_brute_force_each_path_fits_previous_residual(seed):
+    """Path k+1 is the single-path optimum for R_k (sequential derivation)."""
+    rng = np.random.default_rng(seed)
+    n = 9
+    W = np.zeros((1, 32))
+    W[0, :n] = rng.standard_normal(n) * 0.02
+    N = 3
+    planes, alpha, _ = oracle.pack(W, N, 32)
+    R = _residuals(W, planes, alpha, 32)
+    S = _signs(planes)
+    for k in range(N):
+        r = R[k][0]
+        best = math.inf
+        for bits in itertools.product((1.0, -1.0), repeat=n):
+            s = np.concatenate([np.array(bits), np.ones(32 - n)])
+            v, _ = _best_scale_objective(r, s)
+            best = min(best, v)
+        v_or = float(np.sum((r - alpha[k, 0, 0] * S[k, 0]) ** 2))
+        assert v_or <= best * (1 + 1e-9) + 1e-18, (k, v_or, best)
+
+
+def _golden_lines(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                yield [p.strip() for p in line.split("|")]
+
+
+def test_bit_layout_fixtures():
+    rows = list(_golden_lines("bit_layout.txt"))
+    assert len(rows) >= 8
+    for name, vals, word in rows:
+        w = np.array([float(v) for v in vals.split(",")])
+        assert w.size == 32
+        planes, alpha, _ = oracle.pack(w[None, :], 1, 0)
+        assert int(planes[0, 0, 0]) == int(word, 16), name
+
+
+def test_worked_examples():
+    for name, vals, n, alphas, words in _golden_lines("worked_examples.txt"):
+        w = np.array([float(v) for v in vals.split(",")])
+        N = int(n)
+        planes, alpha, _ = oracle.pack(w[None, :], N, 0)
+        exp_a = [float(a) for a in alphas.split(",")]
+        exp_w = [int(x, 16) for x in words.split(",")]
+        assert np.allclose(alpha[:, 0, 0], exp_a, rtol=0, atol=1e-15), name
+        assert [int(planes[k, 0, 0]) for k in range(N)] == exp_w, name
+
+
+@pytest.mark.parametrize("group", [0, 128])
+def test_energy_identity_and_orthogonality(group):
+    wl = synth.WORKLOADS["llama2_7b_decode"]
+    W = synth.host_weight(wl, 0, "q", M=16, K=512).astype(np.float64)
+    N = 4
+    planes, alpha, _ = oracle.pack(W, N, group)
+    G = 512 if group == 0 else group
+    R = _residuals(W, planes, alpha, G)
+    S = _signs(planes)
+    ng = 512 // G
+    for k in range(N):
+        e0 = (R[k].reshape(16, ng, G) ** 2).sum(-1)
+        e1 = (R[k + 1].reshape(16, ng, G) ** 2).sum(-1)
+        # ||R_k||^2 = ||R_{k-1}||^2 - G alpha_k^2 in every row / group
+        assert np.allclose(e1, e0 - G * alpha[k] ** 2, rtol=1e-10, atol=1e-18)
+        assert np.all(e1 <= e0 * (1 + 1e-12))
+        # the residual is orthogonal to the sign plane it was reduced by
+        dot = (R[k + 1] * S[k]).reshape(16, ng, G).sum(-1)
+        assert np.all(np.abs(dot) <= 1e-10 * np.sqrt(e0 * G) + 1e-18)
+
+
+def test_single_path_is_sign_binarisation():
+    rng = np.random.default_rng(7)
+    W = rng.standard_normal((8, 256)).astype(np.float32)
+    W[0, :5] = 0.0
+    W[1, :3] = -0.0
+    planes, alpha, _ = oracle.pack(W, 1, 0)
+    S = _signs(planes)[0]
+    assert np.array_equal(S, np.where(W >= 0, 1.0, -1.0))
+    assert np.allclose(alpha[0, :, 0], np.abs(W.astype(np.float64)).mean(1), rtol=1e-15)
+
+
+def test_zero_rows_and_groups():
+    W = np.zeros((3, 256))
+    W[1, 128:] = np.linspace(-1, 1, 128)
+    planes, alpha, _ = oracle.pack(W, 3, 128)
+    assert np.all(planes[:, 0] == 0xFFFFFFFF)
+    assert np.all(alpha[:, 0] == 0.0)
+    assert np.all(alpha[:, 1, 0] == 0.0) and np.all(planes[:, 1, :4] == 0xFFFFFFFF)
+    assert alpha[0, 1, 1] > 0
+
+
+def test_groups_are_independent():
+    rng = np.random.default_rng(9)
+    W = rng.standard_normal((4, 512))
+    p1, a1, _ = oracle.pack(W, 3, 128)
+    W2 = W.copy()
+    W2[:, 128:256] *= 7.0
+    p2, a2, _ = oracle.pack(W2, 3, 128)
+    keep = np.r_[0:4, 8:16]
+    assert np.array_equal(p1[:, :, keep], p2[:, :, keep])
+    assert np.array_equal(a1[:, :, [0, 2, 3]], a2[:, :, [0, 2, 3]])
+    assert np.allclose(a2[:, :, 1], 7.0 * a1[:, :, 1], rtol=1e-14)
+
+
+@pytest.mark.parametrize("group", [0, 128])
+def test_matvec_against_dense_blas(group):
+    rng = np.random.default_rng(11)
+    M, K, N, T = 24, 384, 3, 5
+    W = rng.standard_normal((M, K))
+    planes, alpha, _ = oracle.pack(W, N, group)
+    G = K if group == 0 else group
+    x = rng.standard_normal((T, K))
+    y, den = oracle.matvec(planes, alpha, x)
+    What = (np.repeat(alpha, G, axis=2) * _signs(planes)).sum(0)      # [M, K]
+    ref = x @ What.T
+    assert np.allclose(y, ref, rtol=0, atol=1e-12 * np.abs(den).max())
+    assert np.allclose(den, np.abs(x) @ np.repeat(alpha, G, axis=2).sum(0).T, rtol=1e-12)
+
+
+def test_matvec_closed_forms():
+    rng = np.random.default_rng(12)
+    M, K, N = 10, 256, 2
+    W = rng.standard_normal((M, K))
+    planes, alpha, _ = oracle.pack(W, N, 128)
+    # x = 1: y_i = sum_k sum_g alpha_k[i,g] (2 popcount(group bits) - 128)
+    y, _ = oracle.matvec(planes, alpha, np.ones((1, K)))
+    for i in range(M):
+        acc = 0.0
+        for k in range(N):
+            for g in range(2):
+                pc = sum(int(w).bit_count() for w in planes[k, i, 4 * g:4 * g + 4])
+                acc += alpha[k, i, g] * (2 * pc - 128)
+        assert abs(y[0, i] - acc) <= 1e-12 * abs(alpha[:, i]).sum() * K
+    # x = e_j: the column j of W^
+    for j in (0, 31, 32, 200, 255):
+        e = np.zeros((1, K))
+        e[0, j] = 1.0
+        y, _ = oracle.matvec(planes, alpha, e)
+        col = sum(alpha[k, :, j // 128] * np.where((planes[k, :, j // 32] >> (j % 32)) & 1, 1.0, -1.0)
+                  for k in range(N))
+        assert np.allclose(y[0], col, rtol=0, atol=1e-15)
+
+
+def _gauss_pop_constants():
+    from scipy import integrate
+    a1 = math.sqrt(2 / math.pi)
+    phi = lambda z: math.exp(-z * z / 2) / math.sqrt(2 * math.pi)
+    # E| |Z| - a1 | for a standard normal Z
+    a2 = integrate.quad(lambda z: abs(z - a1) * 2 * phi(z), 0, a1)[0] + \
+        integrate.quad(lambda z: abs(z - a1) * 2 * phi(z), a1, np.inf)[0]
+    return a1, a2
+
+
+def test_gaussian_population_scales():
+    a1, a2 = _gauss_pop_constants()
+    assert abs(a1 - 0.797885) < 1e-6 and abs(a2 - 0.482624) < 1e-6
+    wl = synth.WORKLOADS["llama3_70b_decode"]
+    W = synth.host_weight(wl, 0, "attn", M=256, K=4096).astype(np.float64)
+    planes, alpha, _ = oracle.pack(W, 2, 0)
+    sigma = synth.configs.W_STD
+    m1 = alpha[0].mean() / sigma
+    m2 = alpha[1].mean() / sigma
+    assert abs(m1 / a1 - 1) < 5e-3, m1
+    assert abs(m2 / a2 - 1) < 5e-3, m2
+    R = _residuals(W, planes, alpha, 4096)
+    e0 = (W ** 2).sum()
+    mse1 = (R[1] ** 2).sum() / e0
+    mse2 = (R[2] ** 2).sum() / e0
+    assert abs(mse1 - (1 - 2 / math.pi)) < 5e-3
+    assert abs(mse2 - (1 - 2 / math.pi - a2 * a2)) < 5e-3
+
+
+def test_student_t_population_scale():
+    from scipy import stats
+    e_abs = stats.t(4).expect(abs)
+    assert abs(e_abs - 1.0) < 1e-9        # E|T_4| = 1
+    wl = synth.WORKLOADS["qbb_g128"]
+    W = synth.host_weight(wl, 0, "up", M=256, K=4096).astype(np.float64)
+    planes, alpha, _ = oracle.pack(W, 4, 128)
+    target = synth.configs.W_STD / math.sqrt(2.0) * e_abs
+    assert abs(alpha[0].mean() / target - 1) < 1e-2
+    assert np.all(np.diff(alpha.mean(axis=(1, 2))) < 0)
+
+
+def test_storage_ratios_from_the_paper():
+    """RaBiT: 8x smaller than FP16 at two paths (section 5), 32x per plane vs
+    fp32 (appendix D), about 2.02 effective bits with per-channel vectors
+    (section 4.1)."""
+    M = K = 4096
+    planes, alpha, _ = oracle.pack(np.ones((2, K)), 2, 0)
+    words_per_row = planes.shape[2]
+    plane_bytes = 2 * M * words_per_row * 4
+    assert (M * K * 2) / plane_bytes == 8.0
+    assert (M * K * 4) / (M * words_per_row * 4) == 32.0
+    # two paths, an fp16 output-channel and input-channel vector per path
+    bits = (plane_bytes * 8 + 2 * 16 * (M + K)) / (M * K)
+    assert round(bits, 2) == 2.02
+
+
+def test_compare_helpers_catch_plausible_mistakes():
+    rng = np.random.default_rng(21)
+    W = rng.standard_normal((8, 256))
+    planes, alpha, rabs = oracle.pack(W, 2, 0, want_rabs=True)
+    assert oracle.compare_planes(planes, planes, rabs, alpha).ok
+    bad = planes.copy()
+    bad[1, 3, 2] ^= 1 << 5
+    assert not oracle.compare_planes(bad, planes, rabs, alpha).ok
+    assert oracle.compare_scales(alpha * (1 + 2e-6), alpha)[0] > 0
+    assert oracle.compare_scales(alpha * (1 + 5e-7), alpha)[0] == 0
+    x = rng.standard_normal((2, 256))
+    y, den = oracle.matvec(planes, alpha, x)
+    # a transposed operand or a dropped path is far outside the tolerance
+    y_drop, _ = oracle.matvec(planes[:1], alpha[:1], x)
+    assert oracle.compare_outputs(y_drop, y, den)[0] > 0
+    y_flip, _ = oracle.matvec(planes[::-1].copy(), alpha, x)
+    assert oracle.compare_outputs(y_flip, y, den)[0] > 0
+    assert oracle.compare_scales_f16(oracle.alpha_to_f16(alpha), alpha) == 0
