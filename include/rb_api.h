@@ -1,0 +1,174 @@
+/*
+ * rb_api.h -- C ABI of the residual-binary-weight linear layer on B200 (sm_100a).
+ *
+ * A linear layer W (M x K) is stored as W ~= sum_k alpha_k (.) B_k with N binary
+ * planes B_k in {-1, +1}^(M x K) and non-negative scales alpha_k, one per row
+ * or one per 128 input columns of each row.
+ *
+ *   RaBiT: Residual-Aware Binarization Training (arXiv 2602.05367),
+ *     section 4.1  -- binary cores with per-channel scale vectors, evaluated
+ *                     with additions and subtractions, k = 2 paths;
+ *     section 4.2  -- every path derived in turn from one shared
+ *                     full-precision weight, the residual updated after each;
+ *     appendix A   -- R1 = W_FP - W^_1, B2 = sign(R1);
+ *     appendix D   -- bit-packed binary GEMV, 32 columns per uint32.
+ *   QBB: Quantization with Binary Bases for LLMs (atlas.scime.ai summary),
+ *     Approach / Key results -- N = 4 binary bases, fp16 scales, one scale
+ *     per 128 input columns (W(4x1)A16g128), cascaded analytical residual
+ *     initialisation.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Pointers marked "device" must be CUDA device memory of the current device;
+ *   the caller owns every buffer. Calls never allocate device memory.
+ * - Every call that takes `stream` (a cudaStream_t, NULL for the legacy
+ *   default stream) only enqueues work and returns; results are ready when the
+ *   stream reaches that point.
+ * - Arguments are validated on the host before anything is enqueued; a call
+ *   that returns an error has enqueued nothing, except where stated.
+ * - Planes: uint32 words [N][M][K/32], row-major. Bit j of word w of a row
+ *   holds column 32*w + j (least significant bit first); a set bit means +1.
+ *   sign(0) = +1, including -0.0. (The paper fixes 32 columns per word but not
+ *   the bit order or polarity; this is the reading the library uses.)
+ * - Scales: [N][M][K/G] with G = K (group = 0) or G = 128 (group = 128).
+ * - K must be a positive multiple of 128, M positive, N in 1..8.
+ * - Non-finite weights or activations are outside the contract.
+ */
+#ifndef RB_API_H
+#define RB_API_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define RB_API __attribute__((visibility("default")))
+#else
+#define RB_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    RB_OK = 0,
+    RB_ERR_INVALID_ARG = 1,   /* null pointer, bad size or leading dimension */
+    RB_ERR_UNSUPPORTED = 2,   /* valid request the kernels do not implement */
+    RB_ERR_ALIGNMENT = 3,     /* pointer or row pitch not 16-byte aligned */
+    RB_ERR_WORKSPACE = 4,     /* workspace missing or smaller than required */
+    RB_ERR_CUDA = 5,          /* a CUDA runtime call or kernel launch failed */
+    RB_ERR_DEVICE = 6         /* a kernel reported a failure through its flag */
+} rb_status;
+
+typedef enum { RB_F32 = 0, RB_F16 = 1 } rb_dtype;
+
+typedef struct {
+    int64_t M;        /* output rows (> 0) */
+    int64_t K;        /* input columns (> 0, multiple of 128) */
+    int32_t n_paths;  /* N, 1..8 */
+    int32_t group;    /* 0: one scale per row; 128: one scale per 128 columns */
+} rb_layout;
+
+/* Number of uint32 plane words, N * M * K / 32 (0 for an invalid layout). */
+RB_API size_t rb_planes_words(rb_layout L);
+
+/* Number of scales, N * M * (K / G) (0 for an invalid layout). */
+RB_API size_t rb_scales_count(rb_layout L);
+
+/* Human-readable name of a status code (static string). */
+RB_API const char* rb_status_string(rb_status s);
+
+/* Detail of the last error returned on the calling host thread ("" if none). */
+RB_API const char* rb_last_error(void);
+
+/*
+ * rb_pack -- derive N residual sign planes and their scales from one shared
+ * full-precision weight (RaBiT section 4.2 and appendix G; QBB cascaded
+ * analytical residual initialisation). For each row, or each 128-column
+ * group of a row:
+ *     R_0 = W;  for k = 1..N:  B_k = sign(R_{k-1})  (sign(0) = +1),
+ *     alpha_k = mean |R_{k-1}| over the row or group,
+ *     R_k = R_{k-1} - alpha_k * B_k.
+ * Arithmetic: residuals in fp32, sums of |R| accumulated in fp64, alpha_k
+ * rounded to fp32 and that fp32 value used in the residual update.
+ *
+ * W         device, M rows of K elements, row pitch `ldw` elements (>= K);
+ *           w_dtype RB_F16 or RB_F32. Base and row pitch 16-byte aligned.
+ * planes    device, out, rb_planes_words(L) words, 16-byte aligned.
+ * alpha     device, out, rb_scales_count(L) fp32 scales.
+ * alpha_f16 device, out, nullable: the same scales rounded to nearest fp16.
+ * Errors: RB_ERR_INVALID_ARG / UNSUPPORTED / ALIGNMENT before launch;
+ *         RB_ERR_CUDA if the launch fails. One scale per row supports
+ *         K <= 65536.
+ */
+RB_API rb_status rb_pack(const void* W, rb_dtype w_dtype, int64_t ldw, rb_layout L,
+                  uint32_t* planes, float* alpha, void* alpha_f16, void* stream);
+
+/*
+ * rb_gemv -- y_t = sum_k alpha_k (.) (B_k x_t) for a small batch of tokens
+ * (RaBiT section 4.1, appendix D: matmul-free evaluation, all paths in one
+ * pass). Runs on CUDA cores: each 8-column block of x is expanded once into a
+ * shared-memory table of its 256 signed sums (built as 2 * masked sum - block
+ * sum), and every plane byte then costs one table lookup and one add.
+ *
+ * planes    device, rb_planes_words(L) words in the layout above.
+ * alpha     device, rb_scales_count(L) scales of type alpha_dtype.
+ * x         device, T rows of K fp16 values, row pitch ldx elements (>= K);
+ *           base and row pitch 16-byte aligned.
+ * y         device, out, T rows of M values of type y_dtype, pitch ldy >= M.
+ * T         tokens, 1..64.
+ * workspace device scratch of at least rb_gemv_workspace_bytes(L, T) bytes,
+ *           16-byte aligned; its first bytes are cleared by the call (a
+ *           memset on `stream`) and it must not be shared by calls that may
+ *           overlap on the GPU. May be NULL when that size is 0.
+ * Errors: as rb_pack; RB_ERR_WORKSPACE if the workspace is too small. A
+ *         kernel-side failure is recorded in the workspace; rb_gemv_check()
+ *         reads it back.
+ */
+RB_API rb_status rb_gemv(const uint32_t* planes, const void* alpha, rb_dtype alpha_dtype,
+                  rb_layout L, const void* x, int64_t ldx, int32_t T,
+                  void* y, rb_dtype y_dtype, int64_t ldy,
+                  void* workspace, size_t ws_bytes, void* stream);
+
+RB_API size_t rb_gemv_workspace_bytes(rb_layout L, int32_t T);
+
+/* One matrix of a grouped matvec; x is [T][K] and y is [T][M], both dense. */
+typedef struct {
+    const uint32_t* planes;  /* device, [N][M][K/32] */
+    const void* alpha;       /* device, [N][M][K/G] */
+    const void* x;           /* device, fp16 [T][K], 16-byte aligned */
+    void* y;                 /* device, [T][M] */
+    int64_t M;
+    int64_t K;
+} rb_gemv_desc;
+
+/*
+ * rb_gemv_grouped -- the same operation over n independent matrices in one
+ * persistent launch (a decode step through a stack of layers). Work is
+ * handed out to CTAs from a counter in the workspace.
+ *
+ * descs_host  host, n descriptors, read for validation and sizing only.
+ * descs_dev   device, the same n descriptors (the caller uploads them once).
+ * n           1..2047.  n_paths, group, alpha_dtype, y_dtype: shared by all.
+ * T           tokens, 1..64.
+ * workspace   device scratch of rb_gemv_grouped_workspace_bytes(...) bytes.
+ */
+RB_API rb_status rb_gemv_grouped(const rb_gemv_desc* descs_host, const rb_gemv_desc* descs_dev,
+                          int32_t n, int32_t n_paths, int32_t group,
+                          rb_dtype alpha_dtype, rb_dtype y_dtype, int32_t T,
+                          void* workspace, size_t ws_bytes, void* stream);
+
+RB_API size_t rb_gemv_grouped_workspace_bytes(const rb_gemv_desc* descs_host, int32_t n,
+                                       int32_t n_paths, int32_t T);
+
+/*
+ * rb_gemv_check -- wait for `stream`, then report RB_ERR_DEVICE if a matvec
+ * kernel that used `workspace` recorded a failure, else RB_OK.
+ */
+RB_API rb_status rb_gemv_check(const void* workspace, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RB_API_H */

@@ -1,0 +1,167 @@
+"""Python entry points: marshal torch tensors into the C ABI of librb.so."""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional, Sequence
+
+import torch
+
+from . import _lib
+from ._lib import GemvDesc, Layout, check
+
+_DT = {torch.float32: _lib.RB_F32, torch.float16: _lib.RB_F16}
+
+
+def _stream(device: torch.device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _p(t: Optional[torch.Tensor]):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def layout(M: int, K: int, n_paths: int, group: int = 0) -> Layout:
+    return Layout(M, K, n_paths, group)
+
+
+def planes_words(M: int, K: int, n_paths: int, group: int = 0) -> int:
+    return _lib.load().rb_planes_words(layout(M, K, n_paths, group))
+
+
+def scales_count(M: int, K: int, n_paths: int, group: int = 0) -> int:
+    return _lib.load().rb_scales_count(layout(M, K, n_paths, group))
+
+
+def _require_cuda(*ts: torch.Tensor) -> torch.device:
+    dev = None
+    for t in ts:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError("tensors must live on a CUDA device")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError("tensors are on different devices")
+    return dev
+
+
+def pack(W: torch.Tensor, n_paths: int = 2, group: int = 0, alpha_f16: bool = False):
+    """Derive N residual sign planes and scales from the shared weight W (M x K).
+
+    Returns (planes int32 [N, M, K/32] holding uint32 words, alpha fp32
+    [N, M, K/G], alpha16 fp16 [N, M, K/G] or None).
+    """
+    lib = _lib.load()
+    dev = _require_cuda(W)
+    if W.dim() != 2 or W.stride(1) != 1 or W.dtype not in _DT:
+        raise ValueError("W must be a 2-D fp16/fp32 tensor with unit column stride")
+    M, K = W.shape
+    G = K if group == 0 else group
+    planes = torch.empty((n_paths, M, K // 32), dtype=torch.int32, device=dev)
+    alpha = torch.empty((n_paths, M, K // G), dtype=torch.float32, device=dev)
+    a16 = torch.empty((n_paths, M, K // G), dtype=torch.float16, device=dev) if alpha_f16 else None
+    with torch.cuda.device(dev):
+        check(lib.rb_pack(_p(W), _DT[W.dtype], W.stride(0), layout(M, K, n_paths, group),
+                          _p(planes), _p(alpha), _p(a16), _stream(dev)))
+    return planes, alpha, a16
+
+
+def gemv_workspace_bytes(M: int, K: int, n_paths: int, group: int, T: int) -> int:
+    return _lib.load().rb_gemv_workspace_bytes(layout(M, K, n_paths, group), T)
+
+
+def _x2d(x: torch.Tensor) -> torch.Tensor:
+    if x.dim() == 1:
+        x = x.unsqueeze(0)
+    if x.dtype != torch.float16 or x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be fp16 [T, K] with unit column stride")
+    return x
+
+
+def gemv(planes: torch.Tensor, alpha: torch.Tensor, x: torch.Tensor, group: int = 0,
+         y: Optional[torch.Tensor] = None, y_dtype: torch.dtype = torch.float16,
+         workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """y[t] = sum_k alpha_k (.) (B_k x[t]) for T <= 64 tokens (CUDA-core table kernel)."""
+    lib = _lib.load()
+    x = _x2d(x)
+    dev = _require_cuda(planes, alpha, x, y, workspace)
+    N, M, W32 = planes.shape
+    K = W32 * 32
+    T = x.shape[0]
+    if y is None:
+        y = torch.empty((T, M), dtype=y_dtype, device=dev)
+    L = layout(M, K, N, group)
+    need = lib.rb_gemv_workspace_bytes(L, T)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        check(lib.rb_gemv(_p(planes), _p(alpha), _DT[alpha.dtype], L, _p(x), x.stride(0), T,
+                          _p(y), _DT[y.dtype], y.stride(0), _p(workspace),
+                          workspace.numel() * workspace.element_size(), _stream(dev)))
+    return y
+
+
+class GroupedGemv:
+    """One persistent launch over many (planes, alpha, x, y) matrices.
+
+    The descriptor table is uploaded once at construction; call ``run()`` for
+    every step (the x tensors are read and the y tensors written in place).
+    """
+
+    def __init__(self, items: Sequence[tuple], n_paths: int, group: int = 0, T: int = 1):
+        lib = _lib.load()
+        self.n_paths, self.group, self.T = n_paths, group, T
+        self.items = list(items)   # keep tensors alive
+        n = len(self.items)
+        self.host = (GemvDesc * n)()
+        adt = ydt = None
+        dev = None
+        for i, (planes, alpha, x, y) in enumerate(self.items):
+            dev = _require_cuda(planes, alpha, x, y)
+            N, M, W32 = planes.shape
+            if N != n_paths or x.shape[-1] != W32 * 32 or y.shape[-1] != M:
+                raise ValueError(f"item {i}: inconsistent shapes")
+            if not (x.is_contiguous() and y.is_contiguous()):
+                raise ValueError(f"item {i}: x and y must be contiguous [T, K] / [T, M]")
+            adt = alpha.dtype if adt is None else adt
+            ydt = y.dtype if ydt is None else ydt
+            if alpha.dtype != adt or y.dtype != ydt:
+                raise ValueError("all items must share the scale and output dtypes")
+            self.host[i] = GemvDesc(planes.data_ptr(), alpha.data_ptr(), x.data_ptr(), y.data_ptr(), M, W32 * 32)
+        self.device = dev
+        raw = bytes(self.host)
+        self.dev_descs = torch.frombuffer(bytearray(raw), dtype=torch.uint8).to(dev)
+        self.alpha_dtype, self.y_dtype = _DT[adt], _DT[ydt]
+        need = lib.rb_gemv_grouped_workspace_bytes(self.host, n, n_paths, T)
+        self.workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+        self.n = n
+
+    def run(self) -> None:
+        lib = _lib.load()
+        with torch.cuda.device(self.device):
+            check(lib.rb_gemv_grouped(ctypes.cast(self.host, ctypes.c_void_p), _p(self.dev_descs), self.n,
+                                      self.n_paths, self.group, self.alpha_dtype, self.y_dtype, self.T,
+                                      _p(self.workspace), self.workspace.numel(), _stream(self.device)))
+
+    def check_device_flag(self) -> None:
+        check(_lib.load().rb_gemv_check(_p(self.workspace), _stream(self.device)))
+
+
+def gemm(planes: torch.Tensor, alpha: torch.Tensor, X: torch.Tensor, group: int = 0,
+         Y: Optional[torch.Tensor] = None, y_dtype: torch.dtype = torch.float16) -> torch.Tensor:
+    """Y[t] = sum_k alpha_k (.) (B_k X[t]) for a prefill block (tcgen05 tensor-core kernel)."""
+    lib = _lib.load()
+    if not hasattr(lib, "rb_gemm"):
+        raise _lib.RbError(2, "this build has no rb_gemm")
+    X = _x2d(X)
+    dev = _require_cuda(planes, alpha, X, Y)
+    N, M, W32 = planes.shape
+    K = W32 * 32
+    T = X.shape[0]
+    if Y is None:
+        Y = torch.empty((T, M), dtype=y_dtype, device=dev)
+    with torch.cuda.device(dev):
+        check(lib.rb_gemm(_p(planes), _p(alpha), _DT[alpha.dtype], layout(M, K, N, group), _p(X), X.stride(0), T,
+                          _p(Y), _DT[Y.dtype], Y.stride(0), _stream(dev)))
+    return Y

@@ -1,0 +1,260 @@
+// Host side of the C ABI declared in include/rb_api.h: argument validation,
+// launch planning and error reporting. Every check runs before anything is
+// enqueued; the kernels live in rb_pack.cu, rb_gemv.cu and rb_gemm.cu.
+#include "../../include/rb_api.h"
+#include "rb_internal.cuh"
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+namespace rb {
+
+static thread_local std::string g_last_error;
+
+static rb_status fail(rb_status s, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return s;
+}
+
+static rb_status cuda_fail(cudaError_t e, const char* where) {
+    return fail(RB_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+int device_sm_count() {
+    static std::mutex mu;
+    static std::vector<int> cache;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    std::lock_guard<std::mutex> lk(mu);
+    if (static_cast<int>(cache.size()) <= dev) cache.resize(dev + 1, 0);
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static rb_status check_layout(const rb_layout& L) {
+    if (L.M <= 0 || L.K <= 0) return fail(RB_ERR_INVALID_ARG, "M and K must be positive (M=%lld K=%lld)",
+                                          (long long)L.M, (long long)L.K);
+    if (L.K % 128 != 0) return fail(RB_ERR_UNSUPPORTED, "K=%lld is not a multiple of 128", (long long)L.K);
+    if (L.n_paths < 1 || L.n_paths > 8) return fail(RB_ERR_UNSUPPORTED, "n_paths=%d outside 1..8", L.n_paths);
+    if (L.group != 0 && L.group != 128) return fail(RB_ERR_UNSUPPORTED, "group=%d (0 or 128)", L.group);
+    // plane word offsets and row indices are kept in 32 bits on the device
+    if (static_cast<double>(L.n_paths) * L.M * (L.K / 32) >= 4294967296.0 || L.M >= (1ll << 31) ||
+        static_cast<double>(L.n_paths) * L.M * (L.K / 128) >= 4294967296.0)
+        return fail(RB_ERR_UNSUPPORTED, "layout too large (N*M*K/32 must stay below 2^32)");
+    return RB_OK;
+}
+
+static size_t dtype_size(rb_dtype d) { return d == RB_F16 ? 2 : 4; }
+
+static bool valid_dtype(rb_dtype d) { return d == RB_F16 || d == RB_F32; }
+
+static size_t gv_ws_bytes(const GvPlan& pl) {
+    if (pl.counters == 0 && pl.partials == 0) return GV_HEADER_BYTES;
+    return GV_HEADER_BYTES + ((pl.counters + 3) & ~size_t(3)) * 4 + pl.partials * 4;
+}
+
+}  // namespace rb
+
+using namespace rb;
+
+extern "C" {
+
+size_t rb_planes_words(rb_layout L) {
+    if (check_layout(L) != RB_OK) return 0;
+    return static_cast<size_t>(L.n_paths) * L.M * (L.K / 32);
+}
+
+size_t rb_scales_count(rb_layout L) {
+    if (check_layout(L) != RB_OK) return 0;
+    const int64_t G = L.group ? L.group : L.K;
+    return static_cast<size_t>(L.n_paths) * L.M * (L.K / G);
+}
+
+const char* rb_status_string(rb_status s) {
+    switch (s) {
+        case RB_OK: return "RB_OK";
+        case RB_ERR_INVALID_ARG: return "RB_ERR_INVALID_ARG";
+        case RB_ERR_UNSUPPORTED: return "RB_ERR_UNSUPPORTED";
+        case RB_ERR_ALIGNMENT: return "RB_ERR_ALIGNMENT";
+        case RB_ERR_WORKSPACE: return "RB_ERR_WORKSPACE";
+        case RB_ERR_CUDA: return "RB_ERR_CUDA";
+        case RB_ERR_DEVICE: return "RB_ERR_DEVICE";
+    }
+    return "RB_ERR_UNKNOWN";
+}
+
+const char* rb_last_error(void) { return g_last_error.c_str(); }
+
+rb_status rb_pack(const void* W, rb_dtype w_dtype, int64_t ldw, rb_layout L,
+                  uint32_t* planes, float* alpha, void* alpha_f16, void* stream) {
+    g_last_error.clear();
+    rb_status st = check_layout(L);
+    if (st != RB_OK) return st;
+    if (!W || !planes || !alpha) return fail(RB_ERR_INVALID_ARG, "null W, planes or alpha");
+    if (!valid_dtype(w_dtype)) return fail(RB_ERR_INVALID_ARG, "bad w_dtype %d", (int)w_dtype);
+    if (ldw < L.K) return fail(RB_ERR_INVALID_ARG, "ldw=%lld < K=%lld", (long long)ldw, (long long)L.K);
+    if (!aligned16(W) || (ldw * dtype_size(w_dtype)) % 16 != 0)
+        return fail(RB_ERR_ALIGNMENT, "W and its row pitch must be 16-byte aligned");
+    if (!aligned16(planes)) return fail(RB_ERR_ALIGNMENT, "planes must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(alpha) & 3u) || (reinterpret_cast<uintptr_t>(alpha_f16) & 1u))
+        return fail(RB_ERR_ALIGNMENT, "alpha must be 4-byte aligned, alpha_f16 2-byte aligned");
+    if (L.group == 0 && L.K > 65536) return fail(RB_ERR_UNSUPPORTED, "one scale per row supports K <= 65536");
+    PackArgs a{W, ldw, L.M, L.K, L.n_paths, L.group, w_dtype == RB_F16, planes, alpha,
+               static_cast<__half*>(alpha_f16)};
+    cudaError_t e = launch_pack(a, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "rb_pack launch");
+    return RB_OK;
+}
+
+size_t rb_gemv_workspace_bytes(rb_layout L, int32_t T) {
+    if (check_layout(L) != RB_OK || T < 1) return 0;
+    GvPlan pl = gemv_plan_single(L.M, L.K, L.n_paths, L.group, T, device_sm_count());
+    return gv_ws_bytes(pl);
+}
+
+static rb_status check_gemv_common(const void* alpha, rb_dtype alpha_dtype, rb_dtype y_dtype, int32_t T) {
+    if (!valid_dtype(alpha_dtype) || !valid_dtype(y_dtype)) return fail(RB_ERR_INVALID_ARG, "bad dtype");
+    if (T < 1 || T > 64) return fail(RB_ERR_UNSUPPORTED, "T=%d outside 1..64", T);
+    if (reinterpret_cast<uintptr_t>(alpha) & (dtype_size(alpha_dtype) - 1))
+        return fail(RB_ERR_ALIGNMENT, "alpha misaligned for its dtype");
+    return RB_OK;
+}
+
+rb_status rb_gemv(const uint32_t* planes, const void* alpha, rb_dtype alpha_dtype,
+                  rb_layout L, const void* x, int64_t ldx, int32_t T,
+                  void* y, rb_dtype y_dtype, int64_t ldy,
+                  void* workspace, size_t ws_bytes, void* stream) {
+    g_last_error.clear();
+    rb_status st = check_layout(L);
+    if (st != RB_OK) return st;
+    if (!planes || !alpha || !x || !y) return fail(RB_ERR_INVALID_ARG, "null planes, alpha, x or y");
+    if ((st = check_gemv_common(alpha, alpha_dtype, y_dtype, T)) != RB_OK) return st;
+    if (ldx < L.K || ldy < L.M) return fail(RB_ERR_INVALID_ARG, "ldx < K or ldy < M");
+    if (!aligned16(planes) || !aligned16(x) || (ldx * 2) % 16 != 0)
+        return fail(RB_ERR_ALIGNMENT, "planes, x and the row pitch of x must be 16-byte aligned");
+    if (reinterpret_cast<uintptr_t>(y) & (dtype_size(y_dtype) - 1)) return fail(RB_ERR_ALIGNMENT, "y misaligned");
+    const int sms = device_sm_count();
+    GvPlan pl = gemv_plan_single(L.M, L.K, L.n_paths, L.group, T, sms);
+    const size_t need = gv_ws_bytes(pl);
+    if (!workspace || ws_bytes < need || !aligned16(workspace))
+        return fail(RB_ERR_WORKSPACE, "workspace needs %zu bytes (16-byte aligned), got %zu", need, ws_bytes);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t clear = GV_HEADER_BYTES + ((pl.counters + 3) & ~size_t(3)) * 4;
+    cudaError_t e = cudaMemsetAsync(workspace, 0, clear, s);
+    if (e != cudaSuccess) return cuda_fail(e, "rb_gemv workspace clear");
+    GvArgs a{};
+    a.one = GvJob{planes, alpha, x, y, L.M, L.K};
+    a.jobs = nullptr;
+    a.n_jobs = 1;
+    a.n_paths = L.n_paths;
+    a.group = L.group;
+    a.alpha_f16 = alpha_dtype == RB_F16;
+    a.y_f16 = y_dtype == RB_F16;
+    a.T = T;
+    a.ldx = ldx;
+    a.ldy = ldy;
+    a.chunk_slices = pl.chunk_slices;
+    a.dynamic = false;
+    a.workspace = workspace;
+    a.ws_bytes = ws_bytes;
+    e = launch_gemv(a, pl, s);
+    if (e != cudaSuccess) return cuda_fail(e, "rb_gemv launch");
+    return RB_OK;
+}
+
+static rb_status check_descs(const rb_gemv_desc* d, int32_t n, int32_t n_paths, int32_t group) {
+    if (!d) return fail(RB_ERR_INVALID_ARG, "null descriptors");
+    if (n < 1 || n > gemv_max_jobs()) return fail(RB_ERR_UNSUPPORTED, "n=%d outside 1..%d", n, gemv_max_jobs());
+    for (int32_t i = 0; i < n; ++i) {
+        rb_layout L{d[i].M, d[i].K, n_paths, group};
+        rb_status st = check_layout(L);
+        if (st != RB_OK) return fail(st, "descriptor %d: %s", i, g_last_error.c_str());
+        if (!d[i].planes || !d[i].alpha || !d[i].x || !d[i].y)
+            return fail(RB_ERR_INVALID_ARG, "descriptor %d has a null pointer", i);
+        if (!aligned16(d[i].planes) || !aligned16(d[i].x))
+            return fail(RB_ERR_ALIGNMENT, "descriptor %d: planes and x must be 16-byte aligned", i);
+    }
+    return RB_OK;
+}
+
+size_t rb_gemv_grouped_workspace_bytes(const rb_gemv_desc* descs_host, int32_t n, int32_t n_paths, int32_t T) {
+    if (!descs_host || n < 1 || n_paths < 1 || n_paths > 8 || T < 1) return 0;
+    // the scale granularity does not change the plan's size bound: use the
+    // larger of the two row-block sizes' counts
+    size_t best = 0;
+    for (int group : {0, 128}) {
+        GvPlan pl = gemv_plan_grouped(reinterpret_cast<const GvJob*>(descs_host), n, n_paths, group, T);
+        const size_t b = gv_ws_bytes(pl);
+        if (b > best) best = b;
+    }
+    return best;
+}
+
+rb_status rb_gemv_grouped(const rb_gemv_desc* descs_host, const rb_gemv_desc* descs_dev,
+                          int32_t n, int32_t n_paths, int32_t group,
+                          rb_dtype alpha_dtype, rb_dtype y_dtype, int32_t T,
+                          void* workspace, size_t ws_bytes, void* stream) {
+    g_last_error.clear();
+    static_assert(sizeof(rb_gemv_desc) == sizeof(GvJob), "descriptor layout");
+    rb_status st = check_descs(descs_host, n, n_paths, group);
+    if (st != RB_OK) return st;
+    if (!descs_dev || (reinterpret_cast<uintptr_t>(descs_dev) & 7u))
+        return fail(RB_ERR_INVALID_ARG, "descs_dev must be a non-null, 8-byte aligned device pointer");
+    if ((st = check_gemv_common(descs_host[0].alpha, alpha_dtype, y_dtype, T)) != RB_OK) return st;
+    GvPlan pl = gemv_plan_grouped(reinterpret_cast<const GvJob*>(descs_host), n, n_paths, group, T);
+    const size_t need = gv_ws_bytes(pl);
+    if (!workspace || ws_bytes < need || !aligned16(workspace))
+        return fail(RB_ERR_WORKSPACE, "workspace needs %zu bytes (16-byte aligned), got %zu", need, ws_bytes);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t clear = GV_HEADER_BYTES + ((pl.counters + 3) & ~size_t(3)) * 4;
+    cudaError_t e = cudaMemsetAsync(workspace, 0, clear, s);
+    if (e != cudaSuccess) return cuda_fail(e, "rb_gemv_grouped workspace clear");
+    GvArgs a{};
+    a.one = GvJob{};
+    a.jobs = reinterpret_cast<const GvJob*>(descs_dev);
+    a.n_jobs = n;
+    a.n_paths = n_paths;
+    a.group = group;
+    a.alpha_f16 = alpha_dtype == RB_F16;
+    a.y_f16 = y_dtype == RB_F16;
+    a.T = T;
+    a.ldx = 0;
+    a.ldy = 0;
+    a.chunk_slices = pl.chunk_slices;
+    a.dynamic = true;
+    a.workspace = workspace;
+    a.ws_bytes = ws_bytes;
+    e = launch_gemv(a, pl, s);
+    if (e != cudaSuccess) return cuda_fail(e, "rb_gemv_grouped launch");
+    return RB_OK;
+}
+
+rb_status rb_gemv_check(const void* workspace, void* stream) {
+    g_last_error.clear();
+    if (!workspace) return fail(RB_ERR_INVALID_ARG, "null workspace");
+    uint32_t flag = 0;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(&flag, static_cast<const uint32_t*>(workspace) + 1, sizeof(flag),
+                                    cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "rb_gemv_check");
+    if (flag) return fail(RB_ERR_DEVICE, "matvec kernel flag 0x%x", flag);
+    return RB_OK;
+}
+
+}  // extern "C"

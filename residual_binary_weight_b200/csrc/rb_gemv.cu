@@ -1,0 +1,492 @@
+// rb_gemv: y_t = sum_k alpha_k (.) (B_k x_t) on CUDA cores, all paths in one pass.
+//
+// RaBiT (arXiv 2602.05367) section 4.1 and appendix D evaluate the layer
+// without multiplications, with additions and subtractions over bit-packed
+// planes. Here every 8-column block c of x is expanded once per CTA into a
+// shared-memory table of its 256 signed sums
+//     T[b][c] = sum_e (bit e of b ? +x[8c+e] : -x[8c+e])
+// (built as 2 * masked sum - block sum, from two 16-entry nibble tables), so
+// a plane byte b costs one PRMT (which forms the table address from the byte
+// and a per-lane base), one LDS and one FADD: 3 instructions per 8 weight
+// bits instead of >= 1 per bit for a select-and-add.
+//
+// Layout of one table: 256 rows of 64 fp32 entries (a 512-column slice of
+// x), 64 KB, placed at shared-window address 0x10000 (a second one, for
+// double buffering, at 0x20000). With the table 64 KB aligned the address of
+// entry (b, c) is 0x10000 | b << 8 | 4c, which PRMT assembles in one
+// instruction: byte 0 (4c) and bytes 2-3 come from the lane's base register,
+// byte 1 is the plane byte.
+//
+// Work split. A CTA (32 warps) owns R rows of one matrix for a K chunk. A
+// warp holds 2J (row, path) items; each item-slice is 16 consecutive plane
+// words, one per lane of a half-warp, so a warp-wide 32-bit load covers two
+// items. Lane l reads byte (q + (l >> 3)) & 3 of its word at step q, which
+// puts the 32 lanes of every LDS on 32 distinct banks. Partial sums stay in
+// registers across the slices of the chunk and are reduced over the 16
+// lanes of each item at the end (transposed butterfly).
+//
+// Per-row scales are applied once per row at the end; per-128-column scales
+// (the QBB layout) multiply each word's partial sum as it is accumulated.
+// A K chunk that is only part of the row writes fp32 partial sums to the
+// workspace; the last CTA to finish a row block adds them in chunk order.
+#include "rb_internal.cuh"
+
+namespace rb {
+namespace {
+
+constexpr int THREADS = 1024;
+constexpr int WARPS = THREADS / 32;
+constexpr int SLICE_COLS = 512;
+constexpr uint32_t TBL0 = 0x10000u;
+constexpr uint32_t TBL_TOGGLE = 0x30000u;   // 0x10000 <-> 0x20000
+constexpr int SMEM_BYTES = 0x30000;          // covers both tables whatever the window base
+constexpr int MAX_JOBS = 2 * THREADS - 1;   // each thread scans two descriptors
+
+// Low shared region (below 0x10000): totals, job prefix sums, scalars.
+struct __align__(16) LowSmem {
+    float tot[WARPS][32];
+    uint32_t unit_prefix[MAX_JOBS + 1];
+    uint32_t ctr_prefix[MAX_JOBS + 1];
+    uint32_t part_prefix[MAX_JOBS + 1];
+    uint32_t wsum[3][WARPS];
+    uint32_t bcast;
+    uint32_t last;
+};
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+__device__ __forceinline__ float lds(uint32_t addr) {
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ void sts(uint32_t addr, float v) {
+    asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v));
+}
+
+// CTA barrier that also orders the inline-asm shared accesses around it.
+__device__ __forceinline__ void cta_sync() { asm volatile("bar.sync 0;" ::: "memory"); }
+
+__device__ __forceinline__ uint32_t ldg_word(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+
+template <int NP, bool G128>
+struct Cfg {
+    static constexpr int J = G128 ? 8 : 16;           // item pairs per warp
+    static constexpr int IPW = 2 * J;                 // items per warp
+    static constexpr int RW = IPW / NP;               // rows per warp
+    static constexpr int ITEMS = RW * NP;             // used items per warp
+    static constexpr int R = WARPS * RW;              // rows per CTA
+};
+
+__device__ __forceinline__ int slices_of(int64_t K) { return static_cast<int>((K + SLICE_COLS - 1) / SLICE_COLS); }
+
+// Build the signed-sum table of slice `s` of x_t into the table at `tbl`.
+__device__ __forceinline__ void build_table(const __half* __restrict__ xt, int64_t K, int s, uint32_t tbl) {
+    const int c = threadIdx.x & 63;
+    const int hi = threadIdx.x >> 6;
+    const int64_t col = static_cast<int64_t>(s) * SLICE_COLS + 8 * c;
+    if (col >= K) return;
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(xt + col));
+    const __half2* h2 = reinterpret_cast<const __half2*>(&u);
+    float x[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __half22float2(h2[i]);
+        x[2 * i] = f.x;
+        x[2 * i + 1] = f.y;
+    }
+    // nibble tables of signed sums: bit e set -> +x_e, clear -> -x_e
+    float p01[4], p23[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        p01[i] = ((i & 1) ? x[0] : -x[0]) + ((i & 2) ? x[1] : -x[1]);
+        p23[i] = ((i & 1) ? x[2] : -x[2]) + ((i & 2) ? x[3] : -x[3]);
+    }
+    const float hsum = (((hi & 1) ? x[4] : -x[4]) + ((hi & 2) ? x[5] : -x[5])) +
+                       (((hi & 4) ? x[6] : -x[6]) + ((hi & 8) ? x[7] : -x[7]));
+    const uint32_t a0 = tbl + (static_cast<uint32_t>(hi) << 12) + 4u * c;
+#pragma unroll
+    for (int lo = 0; lo < 16; ++lo) sts(a0 + (lo << 8), (p01[lo & 3] + p23[lo >> 2]) + hsum);
+}
+
+// Reduce acc[0..J) over the 16 lanes of a half-warp; afterwards lane wd holds
+// the sum of item pair j = wd >> (4 - log2 J) in acc[0].
+template <int J>
+__device__ __forceinline__ void halfwarp_transpose_reduce(float (&acc)[J], int wd) {
+    int cnt = J;
+#pragma unroll
+    for (int off = 8; off >= 1; off >>= 1) {
+        if (cnt > 1) {
+            const int half = cnt >> 1;
+            const bool up = (wd & off) != 0;
+#pragma unroll
+            for (int i = 0; i < J / 2; ++i) {
+                if (i < half) {
+                    const float send = up ? acc[i] : acc[i + half];
+                    const float keep = up ? acc[i + half] : acc[i];
+                    acc[i] = keep + __shfl_xor_sync(FULL_MASK, send, off);
+                }
+            }
+            cnt = half;
+        } else {
+            acc[0] += __shfl_xor_sync(FULL_MASK, acc[0], off);
+        }
+    }
+}
+
+template <int J>
+struct Log2 { static constexpr int v = J == 16 ? 4 : J == 8 ? 3 : J == 4 ? 2 : J == 2 ? 1 : 0; };
+
+template <int NP, bool G128, bool A16>
+__global__ void __launch_bounds__(THREADS, 1) gemv_lut_kernel(GvArgs p, uint32_t* __restrict__ hdr,
+                                                              uint32_t* __restrict__ ctrs,
+                                                              float* __restrict__ parts) {
+    using C = Cfg<NP, G128>;
+    constexpr int J = C::J;
+    extern __shared__ __align__(16) unsigned char dsm[];
+    LowSmem& lo = *reinterpret_cast<LowSmem*>(dsm);
+
+    const uint32_t s0 = smem_addr(dsm);
+    if (s0 + sizeof(LowSmem) > TBL0 || s0 + SMEM_BYTES < TBL0 + 2 * 0x10000u) {
+        if (threadIdx.x == 0) atomicOr(hdr + 1, GV_ERR_SMEM_LAYOUT);
+        return;
+    }
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int h = lane >> 4, wd = lane & 15;
+    const int T = p.T;
+
+    // ---- unit table (prefix sums over jobs), identical in every CTA
+    const int n_jobs = p.jobs ? p.n_jobs : 1;
+    if (n_jobs > MAX_JOBS) {
+        if (tid == 0) atomicOr(hdr + 1, GV_ERR_TOO_MANY_JOBS);
+        return;
+    }
+    {
+        // each thread counts jobs 2*tid and 2*tid + 1, then one block-wide scan
+        uint32_t cu[2] = {0, 0}, cc[2] = {0, 0}, cq[2] = {0, 0};
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int j = 2 * tid + e;
+            if (j < n_jobs) {
+                const int64_t jM = p.jobs ? p.jobs[j].M : p.one.M;
+                const int64_t jK = p.jobs ? p.jobs[j].K : p.one.K;
+                const int nrb = static_cast<int>((jM + C::R - 1) / C::R);
+                const int nch = (slices_of(jK) + p.chunk_slices - 1) / p.chunk_slices;
+                cu[e] = static_cast<uint32_t>(nrb * nch * T);
+                if (nch > 1) {
+                    cc[e] = static_cast<uint32_t>(nrb * T);
+                    cq[e] = static_cast<uint32_t>(nch * T) * static_cast<uint32_t>(jM);
+                }
+            }
+        }
+        uint32_t su = cu[0] + cu[1], sc = cc[0] + cc[1], sq = cq[0] + cq[1];
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const uint32_t a1 = __shfl_up_sync(FULL_MASK, su, off);
+            const uint32_t a2 = __shfl_up_sync(FULL_MASK, sc, off);
+            const uint32_t a3 = __shfl_up_sync(FULL_MASK, sq, off);
+            if (lane >= off) { su += a1; sc += a2; sq += a3; }
+        }
+        if (lane == 31) { lo.wsum[0][warp] = su; lo.wsum[1][warp] = sc; lo.wsum[2][warp] = sq; }
+        cta_sync();
+        if (warp == 0) {
+            uint32_t v0 = lo.wsum[0][lane], v1 = lo.wsum[1][lane], v2 = lo.wsum[2][lane];
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const uint32_t a1 = __shfl_up_sync(FULL_MASK, v0, off);
+                const uint32_t a2 = __shfl_up_sync(FULL_MASK, v1, off);
+                const uint32_t a3 = __shfl_up_sync(FULL_MASK, v2, off);
+                if (lane >= off) { v0 += a1; v1 += a2; v2 += a3; }
+            }
+            lo.wsum[0][lane] = v0; lo.wsum[1][lane] = v1; lo.wsum[2][lane] = v2;   // inclusive
+        }
+        cta_sync();
+        const uint32_t bu = warp ? lo.wsum[0][warp - 1] : 0u;
+        const uint32_t bc = warp ? lo.wsum[1][warp - 1] : 0u;
+        const uint32_t bq = warp ? lo.wsum[2][warp - 1] : 0u;
+        const uint32_t eu = bu + su - (cu[0] + cu[1]);
+        const uint32_t ec = bc + sc - (cc[0] + cc[1]);
+        const uint32_t eq = bq + sq - (cq[0] + cq[1]);
+        const int j0 = 2 * tid;
+        if (j0 <= n_jobs) { lo.unit_prefix[j0] = eu; lo.ctr_prefix[j0] = ec; lo.part_prefix[j0] = eq; }
+        if (j0 + 1 <= n_jobs) {
+            lo.unit_prefix[j0 + 1] = eu + cu[0]; lo.ctr_prefix[j0 + 1] = ec + cc[0]; lo.part_prefix[j0 + 1] = eq + cq[0];
+        }
+    }
+    cta_sync();
+    const uint32_t total_units = lo.unit_prefix[n_jobs];
+
+    // ---- per-lane constants of the lookup
+    const int rot = (lane >> 3) & 3;
+    uint32_t sel[4], base[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const uint32_t qq = static_cast<uint32_t>((q + rot) & 3);
+        sel[q] = 0x7604u | (qq << 4);
+        base[q] = TBL0 + 4u * (4u * wd + qq);
+    }
+
+    uint32_t iter = 0;
+    while (true) {
+        uint32_t u;
+        if (p.dynamic) {
+            if (tid == 0) lo.bcast = atomicAdd(hdr, 1u);
+            cta_sync();
+            u = lo.bcast;
+            cta_sync();
+        } else {
+            u = blockIdx.x + iter * gridDim.x;
+        }
+        ++iter;
+        if (u >= total_units) break;
+
+        // ---- decode the unit: job, then (row block, chunk, token), token fastest
+        int jlo = 0, jhi = n_jobs - 1;
+        while (jlo < jhi) {
+            const int mid = (jlo + jhi + 1) >> 1;
+            if (lo.unit_prefix[mid] <= u) jlo = mid; else jhi = mid - 1;
+        }
+        const GvJob jb = p.jobs ? p.jobs[jlo] : p.one;
+        const int64_t M = jb.M, K = jb.K;
+        const int64_t ldx = p.jobs ? K : p.ldx;
+        const int64_t ldy = p.jobs ? M : p.ldy;
+        const int S = slices_of(K);
+        const int nch = (S + p.chunk_slices - 1) / p.chunk_slices;
+        uint32_t r = u - lo.unit_prefix[jlo];
+        const int t = static_cast<int>(r % T); r /= T;
+        const int ch = static_cast<int>(r % nch);
+        const int rb = static_cast<int>(r / nch);
+        const int s_begin = ch * p.chunk_slices;
+        const int s_end = min(S, s_begin + p.chunk_slices);
+        const int64_t row0 = static_cast<int64_t>(rb) * C::R + warp * C::RW;
+        const int W32 = static_cast<int>(K >> 5);
+        const int gpr = static_cast<int>(K >> 7);
+        const __half* xt = static_cast<const __half*>(jb.x) + t * ldx;
+
+        // item m = 2j + h -> (row row0 + m / NP, path m % NP); word offsets are
+        // kept relative to the plane base (they fit in 32 bits)
+        uint32_t okmask = 0;
+#pragma unroll
+        for (int j = 0; j < J; ++j) {
+            const int m = 2 * j + h;
+            if (m < C::ITEMS && row0 + m / NP < M) okmask |= 1u << j;
+        }
+        // (path * M + row) of item j; fits in 32 bits for every supported shape
+        auto item_prow = [&](int j) -> uint32_t {
+            int rl, path;
+            if (NP % 2 == 0) { rl = (2 * j) / NP; path = (2 * j) % NP + h; }
+            else { rl = h ? (2 * j + 1) / NP : (2 * j) / NP; path = h ? (2 * j + 1) % NP : (2 * j) % NP; }
+            return static_cast<uint32_t>(path) * static_cast<uint32_t>(M) + static_cast<uint32_t>(row0 + rl);
+        };
+        auto item_off = [&](int j) -> uint32_t { return item_prow(j) * static_cast<uint32_t>(W32) + wd; };
+        auto alpha_at = [&](size_t ai) -> float {
+            return A16 ? __half2float(static_cast<const __half*>(jb.alpha)[ai]) : static_cast<const float*>(jb.alpha)[ai];
+        };
+
+        float acc[J];
+        uint32_t wv[J];
+        float av[J];
+#pragma unroll
+        for (int j = 0; j < J; ++j) {
+            acc[j] = 0.0f;
+            av[j] = 0.0f;
+            wv[j] = 0u;
+        }
+        auto words_in = [&](int s) { return min(16, static_cast<int>((K - static_cast<int64_t>(s) * SLICE_COLS) >> 5)); };
+        // G128: the scale of word wd of slice s sits at [(path*M + row) * gpr + 4s + wd/4]
+        auto alpha_idx = [&](int j, int s) -> size_t {
+            return static_cast<size_t>(item_prow(j)) * gpr + 4 * s + (wd >> 2);
+        };
+        auto load_slice = [&](int s) {
+            const bool wok = wd < words_in(s);
+            const uint32_t* ps = jb.planes + 16 * s;
+#pragma unroll
+            for (int j = 0; j < J; ++j) {
+                if (((okmask >> j) & 1u) && wok) {
+                    wv[j] = ldg_word(ps + item_off(j));
+                    if (G128) av[j] = alpha_at(alpha_idx(j, s));
+                }
+            }
+        };
+
+        // ---- slice pipeline: table of slice s in buffer (s - s_begin) & 1
+        uint32_t cur_base[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) cur_base[q] = base[q];
+        load_slice(s_begin);
+        build_table(xt, K, s_begin, TBL0);
+        cta_sync();
+        for (int s = s_begin; s < s_end; ++s) {
+            const int par = (s - s_begin) & 1;
+            const bool has_next = s + 1 < s_end;
+            if (has_next) build_table(xt, K, s + 1, par ? TBL0 : TBL0 + 0x10000u);
+            const bool wok = wd < words_in(s);
+            const bool nok = has_next && wd < words_in(s + 1);
+            const uint32_t* psn = jb.planes + 16 * (s + 1);
+#pragma unroll
+            for (int j = 0; j < J; ++j) {
+                const bool iok = (okmask >> j) & 1u;
+                if (iok && wok) {
+                    const uint32_t w = wv[j];
+                    const float v0 = lds(prmt(w, cur_base[0], sel[0]));
+                    const float v1 = lds(prmt(w, cur_base[1], sel[1]));
+                    const float v2 = lds(prmt(w, cur_base[2], sel[2]));
+                    const float v3 = lds(prmt(w, cur_base[3], sel[3]));
+                    const float ps = (v0 + v1) + (v2 + v3);
+                    if (G128) acc[j] = fmaf(av[j], ps, acc[j]);
+                    else acc[j] += ps;
+                }
+                if (iok && nok) {
+                    wv[j] = ldg_word(psn + item_off(j));
+                    if (G128) av[j] = alpha_at(alpha_idx(j, s + 1));
+                }
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) cur_base[q] ^= TBL_TOGGLE;
+            cta_sync();
+        }
+
+        // ---- reduce over the half-warp; lane wd owns item pair j = wd >> shift
+        halfwarp_transpose_reduce<J>(acc, wd);
+        constexpr int shift = 4 - Log2<J>::v;
+        if ((wd & ((1 << shift) - 1)) == 0) lo.tot[warp][2 * (wd >> shift) + h] = acc[0];
+        __syncwarp();
+
+        // ---- per-row output of this chunk
+        float yv = 0.0f;
+        const int64_t my_row = row0 + lane;
+        const bool row_ok = lane < C::RW && my_row < M;
+        if (row_ok) {
+#pragma unroll
+            for (int k = 0; k < NP; ++k) {
+                const float tk = lo.tot[warp][lane * NP + k];
+                if (G128) {
+                    yv += tk;
+                } else {
+                    const size_t ai = static_cast<size_t>(k) * M + my_row;
+                    const float a = p.alpha_f16 ? __half2float(static_cast<const __half*>(jb.alpha)[ai])
+                                                : static_cast<const float*>(jb.alpha)[ai];
+                    yv = fmaf(a, tk, yv);
+                }
+            }
+        }
+        if (nch == 1) {
+            if (row_ok) {
+                if (p.y_f16) static_cast<__half*>(jb.y)[t * ldy + my_row] = __float2half_rn(yv);
+                else static_cast<float*>(jb.y)[t * ldy + my_row] = yv;
+            }
+        } else {
+            float* part = parts + lo.part_prefix[jlo] + (static_cast<size_t>(t) * nch) * M;
+            if (row_ok) part[static_cast<size_t>(ch) * M + my_row] = yv;
+            __threadfence();
+            cta_sync();
+            if (tid == 0) {
+                const uint32_t prev = atomicAdd(ctrs + lo.ctr_prefix[jlo] + rb * T + t, 1u);
+                lo.last = (prev == static_cast<uint32_t>(nch - 1)) ? 1u : 0u;
+            }
+            cta_sync();
+            if (lo.last) {
+                __threadfence();
+                const int64_t rbase = static_cast<int64_t>(rb) * C::R;
+                for (int i = tid; i < C::R; i += THREADS) {
+                    const int64_t row = rbase + i;
+                    if (row < M) {
+                        float sum = 0.0f;
+                        for (int c = 0; c < nch; ++c) sum += __ldcg(part + static_cast<size_t>(c) * M + row);
+                        if (p.y_f16) static_cast<__half*>(jb.y)[t * ldy + row] = __float2half_rn(sum);
+                        else static_cast<float*>(jb.y)[t * ldy + row] = sum;
+                    }
+                }
+            }
+        }
+        cta_sync();
+    }
+}
+
+template <int NP, bool G128, bool A16>
+cudaError_t launch_one(const GvArgs& a, const GvPlan& plan, cudaStream_t s) {
+    auto kern = gemv_lut_kernel<NP, G128, A16>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    uint32_t* hdr = static_cast<uint32_t*>(a.workspace);
+    uint32_t* ctrs = reinterpret_cast<uint32_t*>(static_cast<char*>(a.workspace) + GV_HEADER_BYTES);
+    float* parts = reinterpret_cast<float*>(ctrs + ((plan.counters + 3) & ~size_t(3)));
+    const int sms = device_sm_count();
+    size_t grid = a.dynamic ? static_cast<size_t>(sms) : plan.units;
+    if (grid > static_cast<size_t>(sms)) grid = sms;
+    if (grid < 1) grid = 1;
+    kern<<<static_cast<unsigned>(grid), THREADS, SMEM_BYTES, s>>>(a, hdr, ctrs, parts);
+    return cudaGetLastError();
+}
+
+template <int NP>
+cudaError_t launch_np(const GvArgs& a, const GvPlan& plan, cudaStream_t s) {
+    if (a.group == 0) return launch_one<NP, false, false>(a, plan, s);   // scale dtype read at run time
+    return a.alpha_f16 ? launch_one<NP, true, true>(a, plan, s) : launch_one<NP, true, false>(a, plan, s);
+}
+
+}  // namespace
+
+int gemv_max_jobs() { return MAX_JOBS; }
+
+int gemv_rows_per_cta(int n_paths, int group) {
+    const int ipw = group ? 16 : 32;
+    return WARPS * (ipw / n_paths);
+}
+
+static void count_job(int64_t M, int64_t K, int R, int chunk, int T, GvPlan& pl) {
+    const int64_t nrb = (M + R - 1) / R;
+    const int64_t S = (K + SLICE_COLS - 1) / SLICE_COLS;
+    const int64_t nch = (S + chunk - 1) / chunk;
+    pl.units += static_cast<size_t>(nrb * nch * T);
+    if (nch > 1) {
+        pl.counters += static_cast<size_t>(nrb * T);
+        pl.partials += static_cast<size_t>(nch * T * M);
+    }
+}
+
+GvPlan gemv_plan_single(int64_t M, int64_t K, int n_paths, int group, int T, int num_sms) {
+    const int R = gemv_rows_per_cta(n_paths, group);
+    const int64_t S = (K + SLICE_COLS - 1) / SLICE_COLS;
+    const int64_t nrb = (M + R - 1) / R;
+    // split K until there are at least two units per SM (or one slice per unit)
+    int64_t nch = 1;
+    while (nch < S && nrb * nch * T < 2 * num_sms) ++nch;
+    const int chunk = static_cast<int>((S + nch - 1) / nch);
+    GvPlan pl{R, chunk, 0, 0, 0};
+    count_job(M, K, R, chunk, T, pl);
+    return pl;
+}
+
+GvPlan gemv_plan_grouped(const GvJob* jobs, int n, int n_paths, int group, int T) {
+    const int R = gemv_rows_per_cta(n_paths, group);
+    const int chunk = 8;   // 4096 columns: wider matrices are split so units stay small
+    GvPlan pl{R, chunk, 0, 0, 0};
+    for (int i = 0; i < n; ++i) count_job(jobs[i].M, jobs[i].K, R, chunk, T, pl);
+    return pl;
+}
+
+cudaError_t launch_gemv(const GvArgs& a, const GvPlan& plan, cudaStream_t s) {
+    switch (a.n_paths) {
+        case 1: return launch_np<1>(a, plan, s);
+        case 2: return launch_np<2>(a, plan, s);
+        case 3: return launch_np<3>(a, plan, s);
+        case 4: return launch_np<4>(a, plan, s);
+        case 5: return launch_np<5>(a, plan, s);
+        case 6: return launch_np<6>(a, plan, s);
+        case 7: return launch_np<7>(a, plan, s);
+        case 8: return launch_np<8>(a, plan, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace rb

@@ -1,0 +1,231 @@
+// rb_pack kernels: residual sign planes and scales from one shared weight.
+//
+// RaBiT (arXiv 2602.05367) section 4.2 and appendix G: the paths are derived
+// in turn from one shared full-precision weight, the residual updated after
+// each path. The scale of a path is mean |R| over its row or 128-column group
+// (QBB summary, cascaded analytical residual initialisation); sign(0) = +1.
+//
+// Two kernels, both HBM-bound streams that read W once and keep the residual
+// of a row (or group) in registers across the N paths:
+//  * one scale per row: one CTA per row, each thread holding CPT chunks of 8
+//    consecutive columns; the fp64 sum of |R| is reduced over the CTA.
+//  * one scale per 128 columns: four lanes per group, each lane holding the 32
+//    columns of one output word; the sum is reduced over the four lanes.
+// |R| is summed in fp32 over at most 8 (row) or 32 (group) values in a
+// balanced tree, then in fp64, so alpha keeps ~2e-7 relative accuracy; the
+// residual stays in fp32 and is updated with the fp32-rounded alpha.
+#include "rb_internal.cuh"
+
+namespace rb {
+namespace {
+
+__device__ __forceinline__ void load8(const __half* p, float (&v)[8]) {
+    const uint4 u = __ldcs(reinterpret_cast<const uint4*>(p));
+    const __half2* h = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __half22float2(h[i]);
+        v[2 * i] = f.x;
+        v[2 * i + 1] = f.y;
+    }
+}
+
+__device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
+    const float4 a = __ldcs(reinterpret_cast<const float4*>(p));
+    const float4 b = __ldcs(reinterpret_cast<const float4*>(p) + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+// Balanced fp32 sum of |v[0..8)|.
+__device__ __forceinline__ float abs_sum8(const float* v) {
+    return ((fabsf(v[0]) + fabsf(v[1])) + (fabsf(v[2]) + fabsf(v[3]))) +
+           ((fabsf(v[4]) + fabsf(v[5])) + (fabsf(v[6]) + fabsf(v[7])));
+}
+
+__device__ __forceinline__ double warp_sum(double v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(FULL_MASK, v, o);
+    return v;
+}
+
+// Sum over the CTA; every thread gets the same value (same order everywhere).
+__device__ __forceinline__ double block_sum(double v, double* red) {
+    v = warp_sum(v);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    double t = lane < nw ? red[lane] : 0.0;
+    t = warp_sum(t);
+    __syncthreads();
+    return t;
+}
+
+// B = +1 when R >= 0 (so -0.0 and +0.0 give +1); returns the packed bits of
+// 8 columns and, unless it is the last path, moves R to R - alpha * B.
+__device__ __forceinline__ uint32_t sign_and_update8(float* r, float a, bool update) {
+    uint32_t bits = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        const bool pos = !(r[e] < 0.0f);
+        bits |= static_cast<uint32_t>(pos) << e;
+        if (update) r[e] -= pos ? a : -a;
+    }
+    return bits;
+}
+
+template <typename WT, int CPT, int MAXT>
+__global__ void __launch_bounds__(MAXT)
+pack_row_kernel(const WT* __restrict__ W, int64_t ldw, int M, int K, int N,
+                uint32_t* __restrict__ planes, float* __restrict__ alpha,
+                __half* __restrict__ alpha16) {
+    __shared__ double red[32];
+    const int row = blockIdx.x;
+    const int chunks = K >> 3;
+    const WT* wrow = W + static_cast<int64_t>(row) * ldw;
+    uint8_t* pbytes = reinterpret_cast<uint8_t*>(planes) + static_cast<size_t>(row) * chunks;
+    const size_t plane_stride = static_cast<size_t>(M) * chunks;
+
+    float r[CPT][8];
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) {
+        const int idx = threadIdx.x + c * blockDim.x;
+        if (idx < chunks) {
+            load8(wrow + 8 * idx, r[c]);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) r[c][e] = 0.0f;
+        }
+    }
+    for (int k = 0; k < N; ++k) {
+        double s = 0.0;
+#pragma unroll
+        for (int c = 0; c < CPT; ++c)
+            if (threadIdx.x + c * blockDim.x < chunks) s += static_cast<double>(abs_sum8(r[c]));
+        s = block_sum(s, red);
+        const float a = static_cast<float>(s / static_cast<double>(K));
+        if (threadIdx.x == 0) {
+            alpha[static_cast<size_t>(k) * M + row] = a;
+            if (alpha16) alpha16[static_cast<size_t>(k) * M + row] = __float2half_rn(a);
+        }
+        const bool update = k + 1 < N;
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) {
+            const int idx = threadIdx.x + c * blockDim.x;
+            if (idx < chunks) {
+                const uint32_t bits = sign_and_update8(r[c], a, update);
+                pbytes[k * plane_stride + idx] = static_cast<uint8_t>(bits);
+            }
+        }
+    }
+}
+
+template <typename WT>
+__device__ __forceinline__ void load32(const WT* p, float (&v)[32]) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float t[8];
+        load8(p + 8 * i, t);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[8 * i + e] = t[e];
+    }
+}
+
+// One scale per (path, row, 128 columns): lanes 4g..4g+3 of a warp own group g
+// (eight groups per warp per step); lane (4g + q) holds columns 32q..32q+31.
+template <typename WT>
+__global__ void __launch_bounds__(256)
+pack_g128_kernel(const WT* __restrict__ W, int64_t ldw, int M, int K, int N,
+                 uint32_t* __restrict__ planes, float* __restrict__ alpha,
+                 __half* __restrict__ alpha16) {
+    const int gpr = K >> 7;
+    const int words = K >> 5;
+    const int64_t total = static_cast<int64_t>(M) * gpr;
+    const int lane = threadIdx.x & 31;
+    const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    for (int64_t g0 = warp * 8; g0 < total; g0 += nwarps * 8) {
+        const int64_t grp = g0 + (lane >> 2);
+        const bool valid = grp < total;
+        const int64_t row = valid ? grp / gpr : 0;
+        const int gi = valid ? static_cast<int>(grp - row * gpr) : 0;
+        const int wi = gi * 4 + (lane & 3);
+        float r[32];
+        if (valid) {
+            load32(W + row * ldw + 32 * wi, r);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) r[e] = 0.0f;
+        }
+        for (int k = 0; k < N; ++k) {
+            float p8[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) p8[i] = abs_sum8(r + 8 * i);
+            double s = static_cast<double>((p8[0] + p8[1]) + (p8[2] + p8[3]));
+            s += __shfl_xor_sync(FULL_MASK, s, 1);
+            s += __shfl_xor_sync(FULL_MASK, s, 2);
+            const float a = static_cast<float>(s * (1.0 / 128.0));
+            const bool update = k + 1 < N;
+            uint32_t word = 0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) word |= sign_and_update8(r + 8 * i, a, update) << (8 * i);
+            if (valid) {
+                planes[(static_cast<int64_t>(k) * M + row) * words + wi] = word;
+                if ((lane & 3) == 0) {
+                    const int64_t ai = (static_cast<int64_t>(k) * M + row) * gpr + gi;
+                    alpha[ai] = a;
+                    if (alpha16) alpha16[ai] = __float2half_rn(a);
+                }
+            }
+        }
+    }
+}
+
+template <typename WT, int CPT, int MAXT = 1024>
+cudaError_t launch_row(const PackArgs& a, int threads, cudaStream_t s) {
+    pack_row_kernel<WT, CPT, MAXT><<<static_cast<unsigned>(a.M), threads, 0, s>>>(
+        static_cast<const WT*>(a.W), a.ldw, static_cast<int>(a.M), static_cast<int>(a.K),
+        a.n_paths, a.planes, a.alpha, a.alpha16);
+    return cudaGetLastError();
+}
+
+template <typename WT>
+cudaError_t launch_row_any(const PackArgs& a, cudaStream_t s) {
+    const int chunks = static_cast<int>(a.K >> 3);
+    int cpt = 1;
+    while (cpt < 8 && (chunks + cpt - 1) / cpt > 512) cpt *= 2;
+    int threads = (chunks + cpt - 1) / cpt;
+    threads = (threads + 31) & ~31;
+    if (threads > 1024) return cudaErrorInvalidConfiguration;
+    switch (cpt) {
+        case 1: return launch_row<WT, 1>(a, threads, s);
+        case 2: return launch_row<WT, 2>(a, threads, s);
+        case 4: return launch_row<WT, 4>(a, threads, s);
+        default:   // 8 chunks (64 values) per thread: give it 128 registers when it fits in 512 threads
+            return threads <= 512 ? launch_row<WT, 8, 512>(a, threads, s) : launch_row<WT, 8, 1024>(a, threads, s);
+    }
+}
+
+template <typename WT>
+cudaError_t launch_g128(const PackArgs& a, cudaStream_t s) {
+    const int64_t groups = a.M * (a.K >> 7);
+    const int64_t warps_needed = (groups + 7) / 8;
+    int64_t blocks = (warps_needed + 7) / 8;
+    const int64_t cap = static_cast<int64_t>(device_sm_count()) * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    pack_g128_kernel<WT><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+        static_cast<const WT*>(a.W), a.ldw, static_cast<int>(a.M), static_cast<int>(a.K),
+        a.n_paths, a.planes, a.alpha, a.alpha16);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_pack(const PackArgs& a, cudaStream_t s) {
+    if (a.group == 0)
+        return a.w_f16 ? launch_row_any<__half>(a, s) : launch_row_any<float>(a, s);
+    return a.w_f16 ? launch_g128<__half>(a, s) : launch_g128<float>(a, s);
+}
+
+}  // namespace rb

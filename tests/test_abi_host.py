@@ -1,0 +1,139 @@
+"""Host-only checks of the C ABI: the library loads, exports every declared
+symbol, sizes its buffers as documented and rejects bad arguments before it
+touches a device. No compute call runs here."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from residual_binary_weight_b200 import _lib
+from residual_binary_weight_b200._lib import GemvDesc, Layout
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "rb_api.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*RB_API\s+(?:const\s+)?[a-z_0-9]+\s*\*?\s*(rb_[a-z_0-9]+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = _lib.load()
+    names = _declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in _lib.EXPORTED, n
+
+
+def test_library_hides_internal_symbols():
+    out = os.popen(f"nm -D --defined-only {_lib.LIB_PATH}").read()
+    exported = {l.split()[-1] for l in out.splitlines() if " T " in l}
+    ours = {n for n in exported if n.startswith("rb_")}
+    assert ours == set(_declared_functions())
+
+
+def test_sizes():
+    lib = _lib.load()
+    assert lib.rb_planes_words(Layout(4096, 4096, 2, 0)) == 2 * 4096 * 128
+    assert lib.rb_scales_count(Layout(4096, 4096, 2, 0)) == 2 * 4096
+    assert lib.rb_scales_count(Layout(11008, 4096, 4, 128)) == 4 * 11008 * 32
+    # invalid layouts size to zero
+    assert lib.rb_planes_words(Layout(4096, 4000, 2, 0)) == 0
+    assert lib.rb_planes_words(Layout(0, 4096, 2, 0)) == 0
+    assert lib.rb_planes_words(Layout(16, 128, 9, 0)) == 0
+    assert lib.rb_scales_count(Layout(16, 128, 2, 64)) == 0
+
+
+def test_status_strings():
+    lib = _lib.load()
+    for code, name in _lib.STATUS_NAMES.items():
+        assert lib.rb_status_string(code).decode() == name
+
+
+FAKE = 1 << 40          # a 16-byte aligned address that is never dereferenced
+
+
+def _status(rc):
+    return _lib.STATUS_NAMES[rc]
+
+
+def test_pack_rejects_bad_arguments_before_launch():
+    lib = _lib.load()
+    L = Layout(64, 256, 2, 0)
+    p = ctypes.c_void_p
+    assert _status(lib.rb_pack(None, 0, 256, L, p(FAKE), p(FAKE), None, None)) == "RB_ERR_INVALID_ARG"
+    assert _status(lib.rb_pack(p(FAKE), 0, 255, L, p(FAKE), p(FAKE), None, None)) == "RB_ERR_INVALID_ARG"
+    assert _status(lib.rb_pack(p(FAKE), 7, 256, L, p(FAKE), p(FAKE), None, None)) == "RB_ERR_INVALID_ARG"
+    assert _status(lib.rb_pack(p(FAKE + 4), 0, 256, L, p(FAKE), p(FAKE), None, None)) == "RB_ERR_ALIGNMENT"
+    assert _status(lib.rb_pack(p(FAKE), 1, 260, L, p(FAKE), p(FAKE), None, None)) == "RB_ERR_ALIGNMENT"
+    assert _status(lib.rb_pack(p(FAKE), 0, 256, L, p(FAKE + 8), p(FAKE), None, None)) == "RB_ERR_ALIGNMENT"
+    assert _status(lib.rb_pack(p(FAKE), 0, 256, Layout(64, 200, 2, 0), p(FAKE), p(FAKE), None, None)) == \
+        "RB_ERR_UNSUPPORTED"
+    assert _status(lib.rb_pack(p(FAKE), 0, 256, Layout(64, 256, 0, 0), p(FAKE), p(FAKE), None, None)) == \
+        "RB_ERR_UNSUPPORTED"
+    assert _status(lib.rb_pack(p(FAKE), 0, 256, Layout(64, 256, 2, 32), p(FAKE), p(FAKE), None, None)) == \
+        "RB_ERR_UNSUPPORTED"
+    assert _status(lib.rb_pack(p(FAKE), 0, 1 << 17, Layout(4, 1 << 17, 2, 0), p(FAKE), p(FAKE), None, None)) == \
+        "RB_ERR_UNSUPPORTED"
+    lib.rb_pack(p(FAKE), 0, 256, Layout(64, 200, 2, 0), p(FAKE), p(FAKE), None, None)
+    assert b"multiple of 128" in lib.rb_last_error()
+
+
+def test_gemv_rejects_bad_arguments_before_launch():
+    lib = _lib.load()
+    L = Layout(64, 256, 2, 0)
+    p = ctypes.c_void_p
+    ok = (p(FAKE), p(FAKE), 0, L, p(FAKE), 256, 1, p(FAKE), 1, 64, p(FAKE), 1 << 20, None)
+
+    def call(**kw):
+        args = list(ok)
+        names = ["planes", "alpha", "adt", "L", "x", "ldx", "T", "y", "ydt", "ldy", "ws", "wsb", "s"]
+        for k, v in kw.items():
+            args[names.index(k)] = v
+        return _status(lib.rb_gemv(*args))
+
+    assert call(planes=None) == "RB_ERR_INVALID_ARG"
+    assert call(T=0) == "RB_ERR_UNSUPPORTED"
+    assert call(T=65) == "RB_ERR_UNSUPPORTED"
+    assert call(ldx=100) == "RB_ERR_INVALID_ARG"
+    assert call(ldy=10) == "RB_ERR_INVALID_ARG"
+    assert call(x=p(FAKE + 2)) == "RB_ERR_ALIGNMENT"
+    assert call(ldx=260) == "RB_ERR_ALIGNMENT"
+    assert call(ws=None) == "RB_ERR_WORKSPACE"
+    assert call(wsb=8) == "RB_ERR_WORKSPACE"
+    assert call(adt=5) == "RB_ERR_INVALID_ARG"
+    assert call(L=Layout(64, 256, 9, 0)) == "RB_ERR_UNSUPPORTED"
+
+
+def test_grouped_rejects_bad_descriptors():
+    lib = _lib.load()
+    p = ctypes.c_void_p
+    d = (GemvDesc * 2)()
+    d[0] = GemvDesc(FAKE, FAKE, FAKE, FAKE, 128, 256)
+    d[1] = GemvDesc(FAKE, FAKE, FAKE, FAKE, 128, 200)
+    host = ctypes.cast(d, p)
+    rc = lib.rb_gemv_grouped(host, p(FAKE), 2, 2, 0, 0, 1, 1, p(FAKE), 1 << 20, None)
+    assert _status(rc) == "RB_ERR_UNSUPPORTED"
+    assert b"descriptor 1" in lib.rb_last_error()
+    d[1] = GemvDesc(FAKE, None, FAKE, FAKE, 128, 256)
+    assert _status(lib.rb_gemv_grouped(host, p(FAKE), 2, 2, 0, 0, 1, 1, p(FAKE), 1 << 20, None)) == \
+        "RB_ERR_INVALID_ARG"
+    d[1] = GemvDesc(FAKE, FAKE, FAKE, FAKE, 128, 256)
+    assert _status(lib.rb_gemv_grouped(host, None, 2, 2, 0, 0, 1, 1, p(FAKE), 1 << 20, None)) == \
+        "RB_ERR_INVALID_ARG"
+    assert _status(lib.rb_gemv_grouped(host, p(FAKE), 0, 2, 0, 0, 1, 1, p(FAKE), 1 << 20, None)) == \
+        "RB_ERR_UNSUPPORTED"
+    assert lib.rb_gemv_grouped_workspace_bytes(host, 2, 2, 1) >= 256
+
+
+def test_workspace_sizes_follow_the_split():
+    lib = _lib.load()
+    # one matrix with few rows is split along K, which needs counters and partial sums
+    small = lib.rb_gemv_workspace_bytes(Layout(512, 8192, 2, 0), 1)
+    assert small > 256 + 4 * 512
+    # a layout that is rejected needs nothing
+    assert lib.rb_gemv_workspace_bytes(Layout(512, 8000, 2, 0), 1) == 0

@@ -1,0 +1,188 @@
+"""rb_gemv / rb_gemv_grouped on the GPU against the fp64 oracle.
+
+Kernel parity: the oracle packs the weight, and the GPU and the oracle both
+evaluate those planes and stored scales on the same x, so no oracle input
+comes from the GPU. Outputs must be within 1e-3 * sum_k sum_j |alpha_k x_j|.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import residual_binary_weight_b200 as rb
+import synth
+from gpu_util import check_gemv_on_oracle_planes, planes_np, to_dev_planes
+
+pytestmark = pytest.mark.gpu
+
+
+def _ok(res, what):
+    nbad, worst = res
+    assert nbad == 0, (what, worst)
+    assert worst < 1e-3
+
+
+def test_layer256_full():
+    wl = synth.WORKLOADS["layer256"]
+    W = synth.host_weight(wl, 0, "w")
+    x = synth.host_activations(wl, 0, "w", 1)
+    _ok(check_gemv_on_oracle_planes(W, x, 2, 0, alpha_f16=False), "layer256")
+
+
+@pytest.mark.parametrize("matrix,rows,T", [("q", 1000, 1), ("gate", 700, 2), ("down", 300, 3)])
+def test_llama2_shapes(matrix, rows, T):
+    wl = synth.WORKLOADS["llama2_7b_decode"]
+    W = synth.host_rows(wl, 1, matrix, range(rows))
+    x = synth.host_activations(wl, 1, matrix, T)
+    _ok(check_gemv_on_oracle_planes(W, x, 2, 0, alpha_f16=False), matrix)
+
+
+@pytest.mark.parametrize("T", [1, 4, 16])
+@pytest.mark.parametrize("matrix,rows", [("up", 200), ("down", 150)])
+def test_qbb_g128(matrix, rows, T):
+    wl = synth.WORKLOADS["qbb_g128"]
+    W = synth.host_rows(wl, 0, matrix, range(rows))
+    x = synth.host_activations(wl, 0, matrix, T)
+    _ok(check_gemv_on_oracle_planes(W, x, 4, 128, alpha_f16=True), (matrix, T))
+
+
+@pytest.mark.parametrize("n_paths", [1, 3, 5, 8])
+@pytest.mark.parametrize("group", [0, 128])
+def test_path_counts(n_paths, group):
+    rng = np.random.default_rng(7 * n_paths + group)
+    W = (rng.standard_normal((333, 1152)) * 0.02).astype(np.float16)
+    x = rng.standard_normal((2, 1152)).astype(np.float16)
+    _ok(check_gemv_on_oracle_planes(W, x, n_paths, group, alpha_f16=(group == 128)), (n_paths, group))
+
+
+@pytest.mark.parametrize("alpha_f16,y_dtype", [(True, torch.float32), (False, torch.float32), (True, torch.float16)])
+def test_dtypes_and_pitches(alpha_f16, y_dtype):
+    rng = np.random.default_rng(3)
+    W = (rng.standard_normal((96, 640)) * 0.02).astype(np.float16)
+    x = rng.standard_normal((3, 640)).astype(np.float16)
+    _ok(check_gemv_on_oracle_planes(W, x, 2, 0, alpha_f16, y_dtype, ldx_pad=8, ldy_pad=5), "pitch")
+    _ok(check_gemv_on_oracle_planes(W, x, 2, 128, alpha_f16, y_dtype, ldx_pad=8, ldy_pad=3), "pitch g128")
+
+
+@pytest.mark.parametrize("K", [128, 384, 640])
+def test_small_and_ragged(K):
+    rng = np.random.default_rng(K)
+    for M in (1, 33):
+        W = (rng.standard_normal((M, K)) * 0.02).astype(np.float32)
+        x = rng.standard_normal((1, K)).astype(np.float16)
+        _ok(check_gemv_on_oracle_planes(W, x, 2, 0, False), (M, K))
+        _ok(check_gemv_on_oracle_planes(W, x, 2, 128, False), (M, K, 128))
+
+
+def test_split_k_single_matrix():
+    """Few rows and long rows: the single-matrix plan splits K into chunks and
+    the last CTA of a row block adds the partial sums."""
+    rng = np.random.default_rng(11)
+    W = (rng.standard_normal((64, 28672)) * 0.02).astype(np.float16)
+    x = rng.standard_normal((1, 28672)).astype(np.float16)
+    _ok(check_gemv_on_oracle_planes(W, x, 2, 0, False), "split")
+    _ok(check_gemv_on_oracle_planes(W, x, 4, 128, True), "split g128")
+
+
+def test_x_equal_one_and_unit_vectors():
+    """Closed forms through the GPU path: x = 1 gives alpha-weighted popcounts,
+    x = e_j extracts column j of the reconstructed weight."""
+    rng = np.random.default_rng(17)
+    M, K = 40, 512
+    W = (rng.standard_normal((M, K)) * 0.02).astype(np.float32)
+    ref_p, ref_a, _ = oracle.pack(W, 2, 0)
+    a32 = ref_a.astype(np.float32)
+    ones = np.ones((1, K), dtype=np.float16)
+    y = rb.gemv(to_dev_planes(ref_p), torch.from_numpy(a32).cuda(), torch.from_numpy(ones).cuda(),
+                y_dtype=torch.float32).cpu().numpy()[0]
+    pc = np.array([[sum(int(w).bit_count() for w in ref_p[k, i]) for i in range(M)] for k in range(2)])
+    exp = (a32.astype(np.float64)[:, :, 0] * (2 * pc - K)).sum(0)
+    assert np.allclose(y, exp, rtol=0, atol=1e-5 * np.abs(a32).sum(0).max() * K)
+    for j in (0, 37, 511):
+        e = np.zeros((1, K), dtype=np.float16)
+        e[0, j] = 1.0
+        y = rb.gemv(to_dev_planes(ref_p), torch.from_numpy(a32).cuda(), torch.from_numpy(e).cuda(),
+                    y_dtype=torch.float32).cpu().numpy()[0]
+        col = sum(a32[k, :, 0].astype(np.float64) * np.where((ref_p[k, :, j // 32] >> (j % 32)) & 1, 1.0, -1.0)
+                  for k in range(2))
+        assert np.allclose(y, col, rtol=1e-6, atol=1e-9)
+
+
+def _grouped_case(wl_name, layer, scale_rows, T, n_paths, group, alpha_f16):
+    wl = synth.WORKLOADS[wl_name]
+    items, refs = [], []
+    for spec in wl.matrices:
+        M = max(1, spec.M // scale_rows)
+        W = synth.host_rows(wl, layer, spec.name, range(M))
+        x = synth.host_activations(wl, layer, spec.name, T)
+        ref_p, ref_a, _ = oracle.pack(W, n_paths, group)
+        stored = oracle.alpha_to_f16(ref_a) if alpha_f16 else ref_a.astype(np.float32)
+        y_ref, den = oracle.matvec(ref_p, stored.astype(np.float64), x.astype(np.float64))
+        y = torch.full((T, M), float("nan"), dtype=torch.float16, device="cuda")
+        items.append((to_dev_planes(ref_p), torch.from_numpy(stored).cuda(), torch.from_numpy(x).cuda(), y))
+        refs.append((y_ref, den))
+    return items, refs
+
+
+@pytest.mark.parametrize("T", [1, 2])
+def test_grouped_llama2_layer(T):
+    items, refs = _grouped_case("llama2_7b_decode", 2, 8, T, 2, 0, False)
+    g = rb.GroupedGemv(items, n_paths=2, group=0, T=T)
+    for _ in range(2):              # the work counter is cleared on every call
+        for it in items:
+            it[3].fill_(float("nan"))
+        g.run()
+        torch.cuda.synchronize()
+        g.check_device_flag()
+        for (_, _, _, y), (y_ref, den) in zip(items, refs):
+            nbad, worst = oracle.compare_outputs(y.float().cpu().numpy(), y_ref, den)
+            assert nbad == 0, worst
+
+
+def test_grouped_qbb_g128():
+    items, refs = _grouped_case("qbb_g128", 0, 16, 1, 4, 128, True)
+    g = rb.GroupedGemv(items, n_paths=4, group=128, T=1)
+    g.run()
+    torch.cuda.synchronize()
+    g.check_device_flag()
+    for (_, _, _, y), (y_ref, den) in zip(items, refs):
+        nbad, worst = oracle.compare_outputs(y.float().cpu().numpy(), y_ref, den)
+        assert nbad == 0, worst
+
+
+def test_full_size_layer_sampled_rows():
+    """One full Llama-2-7B-shaped layer (7 matrices) drawn on the device,
+    packed and evaluated by one grouped launch. For 48 sampled rows per
+    matrix the oracle packs the host copy of the weight row; the GPU planes of
+    those rows must match, and after the rows are replaced by the oracle's
+    planes and scales, the GPU outputs must match the oracle's."""
+    wl = synth.WORKLOADS["llama2_7b_decode"]
+    rng = np.random.default_rng(2)
+    items, checks = [], []
+    for spec in wl.matrices:
+        W = synth.device_weight(wl, 0, spec.name, "cuda")
+        x = synth.device_activations(wl, 0, spec.name, 1, "cuda")
+        planes, alpha, _ = rb.pack(W, 2, 0)
+        rows = np.sort(rng.choice(spec.M, 48, replace=False))
+        idx = torch.from_numpy(rows).cuda()
+        Wr = W.index_select(0, idx).cpu().numpy()
+        ref_p, ref_a, rabs = oracle.pack(Wr, 2, 0, want_rabs=True)
+        rep = oracle.compare_planes(planes_np(planes[:, idx]), ref_p, rabs, ref_a)
+        assert rep.bad == 0, (spec.name, rep)
+        assert oracle.compare_scales(alpha[:, idx].cpu().numpy(), ref_a)[0] == 0
+        planes[:, idx] = to_dev_planes(ref_p)
+        a32 = ref_a.astype(np.float32)
+        alpha[:, idx] = torch.from_numpy(a32).cuda()
+        del W
+        y = torch.empty((1, spec.M), dtype=torch.float16, device="cuda")
+        items.append((planes, alpha, x, y))
+        y_ref, den = oracle.matvec(ref_p, a32.astype(np.float64), x.cpu().numpy().astype(np.float64))
+        checks.append((idx, y_ref, den))
+    g = rb.GroupedGemv(items, n_paths=2, group=0, T=1)
+    g.run()
+    torch.cuda.synchronize()
+    g.check_device_flag()
+    for (_, _, _, y), (idx, y_ref, den) in zip(items, checks):
+        got = y[:, idx].float().cpu().numpy()
+        nbad, worst = oracle.compare_outputs(got, y_ref, den)
+        assert nbad == 0, worst
