@@ -26,10 +26,16 @@
  *   stream reaches that point.
  * - Arguments are validated on the host before anything is enqueued; a call
  *   that returns an error has enqueued nothing, except where stated.
- * - Planes: uint32 words [N][M][K/32], row-major. Bit j of word w of a row
- *   holds column 32*w + j (least significant bit first); a set bit means +1.
- *   sign(0) = +1, including -0.0. (The paper fixes 32 columns per word but not
- *   the bit order or polarity; this is the reading the library uses.)
+ * - Plane words: bit j of word w of a row holds column 32*w + j (least
+ *   significant bit first); a set bit means +1; sign(0) = +1, including -0.0.
+ *   (The paper fixes 32 columns per uint32 but not the bit order or the
+ *   polarity; this is the reading the library uses.) Two word orders:
+ *     RB_ROWS    [N][M][K/32], row-major: the interchange order.
+ *     RB_SLICED  the order the matvec kernels stream: for each path k and each
+ *                512-column slice s (S = ceil(K/512) slices), the 16 words of
+ *                that slice of every row, row after row. Word v of slice s of
+ *                row i of path k sits at ((k*S + s)*M + i)*16 + v. In the last
+ *                slice the words past K/32 are padding (rb_pack writes 0).
  * - Scales: [N][M][K/G] with G = K (group = 0) or G = 128 (group = 128).
  * - K must be a positive multiple of 128, M positive, N in 1..8.
  * - Non-finite weights or activations are outside the contract.
@@ -62,14 +68,19 @@ typedef enum {
 
 typedef enum { RB_F32 = 0, RB_F16 = 1 } rb_dtype;
 
+typedef enum { RB_ROWS = 0, RB_SLICED = 1 } rb_order;
+
 typedef struct {
     int64_t M;        /* output rows (> 0) */
     int64_t K;        /* input columns (> 0, multiple of 128) */
     int32_t n_paths;  /* N, 1..8 */
     int32_t group;    /* 0: one scale per row; 128: one scale per 128 columns */
+    int32_t order;    /* plane word order, an rb_order */
+    int32_t reserved; /* must be 0 */
 } rb_layout;
 
-/* Number of uint32 plane words, N * M * K / 32 (0 for an invalid layout). */
+/* Number of uint32 plane words: N*M*K/32 (RB_ROWS) or N*M*16*ceil(K/512)
+ * (RB_SLICED); 0 for an invalid layout. */
 RB_API size_t rb_planes_words(rb_layout L);
 
 /* Number of scales, N * M * (K / G) (0 for an invalid layout). */
@@ -94,7 +105,7 @@ RB_API const char* rb_last_error(void);
  *
  * W         device, M rows of K elements, row pitch `ldw` elements (>= K);
  *           w_dtype RB_F16 or RB_F32. Base and row pitch 16-byte aligned.
- * planes    device, out, rb_planes_words(L) words, 16-byte aligned.
+ * planes    device, out, rb_planes_words(L) words in L.order, 16-byte aligned.
  * alpha     device, out, rb_scales_count(L) fp32 scales.
  * alpha_f16 device, out, nullable: the same scales rounded to nearest fp16.
  * Errors: RB_ERR_INVALID_ARG / UNSUPPORTED / ALIGNMENT before launch;
@@ -111,7 +122,8 @@ RB_API rb_status rb_pack(const void* W, rb_dtype w_dtype, int64_t ldw, rb_layout
  * shared-memory table of its 256 signed sums (built as 2 * masked sum - block
  * sum), and every plane byte then costs one table lookup and one add.
  *
- * planes    device, rb_planes_words(L) words in the layout above.
+ * planes    device, rb_planes_words(L) words in L.order (RB_SLICED streams
+ *           contiguous 32 KB tiles; RB_ROWS reads 64-byte pieces per row).
  * alpha     device, rb_scales_count(L) scales of type alpha_dtype.
  * x         device, T rows of K fp16 values, row pitch ldx elements (>= K);
  *           base and row pitch 16-byte aligned.
@@ -149,12 +161,13 @@ typedef struct {
  *
  * descs_host  host, n descriptors, read for validation and sizing only.
  * descs_dev   device, the same n descriptors (the caller uploads them once).
- * n           1..2047.  n_paths, group, alpha_dtype, y_dtype: shared by all.
+ * n           1..2047.  n_paths, group, order (an rb_order), alpha_dtype,
+ *             y_dtype: shared by all.
  * T           tokens, 1..64.
  * workspace   device scratch of rb_gemv_grouped_workspace_bytes(...) bytes.
  */
 RB_API rb_status rb_gemv_grouped(const rb_gemv_desc* descs_host, const rb_gemv_desc* descs_dev,
-                          int32_t n, int32_t n_paths, int32_t group,
+                          int32_t n, int32_t n_paths, int32_t group, int32_t order,
                           rb_dtype alpha_dtype, rb_dtype y_dtype, int32_t T,
                           void* workspace, size_t ws_bytes, void* stream);
 

@@ -17,6 +17,7 @@ RB_OK = 0
 STATUS_NAMES = {0: "RB_OK", 1: "RB_ERR_INVALID_ARG", 2: "RB_ERR_UNSUPPORTED", 3: "RB_ERR_ALIGNMENT",
                 4: "RB_ERR_WORKSPACE", 5: "RB_ERR_CUDA", 6: "RB_ERR_DEVICE"}
 RB_F32, RB_F16 = 0, 1
+RB_ROWS, RB_SLICED = 0, 1
 
 # every symbol include/rb_api.h declares
 EXPORTED = ("rb_planes_words", "rb_scales_count", "rb_status_string", "rb_last_error",
@@ -33,7 +34,8 @@ class RbError(RuntimeError):
 
 class Layout(ctypes.Structure):
     _fields_ = [("M", ctypes.c_int64), ("K", ctypes.c_int64),
-                ("n_paths", ctypes.c_int32), ("group", ctypes.c_int32)]
+                ("n_paths", ctypes.c_int32), ("group", ctypes.c_int32),
+                ("order", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
 class GemvDesc(ctypes.Structure):
@@ -71,7 +73,7 @@ def load() -> ctypes.CDLL:
         lib.rb_gemv.restype = st
         lib.rb_gemv_workspace_bytes.argtypes = [Layout, i32]
         lib.rb_gemv_workspace_bytes.restype = sz
-        lib.rb_gemv_grouped.argtypes = [vp, vp, i32, i32, i32, st, st, i32, vp, sz, vp]
+        lib.rb_gemv_grouped.argtypes = [vp, vp, i32, i32, i32, i32, st, st, i32, vp, sz, vp]
         lib.rb_gemv_grouped.restype = st
         lib.rb_gemv_grouped_workspace_bytes.argtypes = [vp, i32, i32, i32]
         lib.rb_gemv_grouped_workspace_bytes.restype = sz

@@ -20,16 +20,34 @@ def _p(t: Optional[torch.Tensor]):
     return ctypes.c_void_p(t.data_ptr()) if t is not None else None
 
 
-def layout(M: int, K: int, n_paths: int, group: int = 0) -> Layout:
-    return Layout(M, K, n_paths, group)
+_ORDERS = {"rows": _lib.RB_ROWS, "sliced": _lib.RB_SLICED}
 
 
-def planes_words(M: int, K: int, n_paths: int, group: int = 0) -> int:
-    return _lib.load().rb_planes_words(layout(M, K, n_paths, group))
+def layout(M: int, K: int, n_paths: int, group: int = 0, order: str = "rows") -> Layout:
+    return Layout(M, K, n_paths, group, _ORDERS[order], 0)
+
+
+def planes_words(M: int, K: int, n_paths: int, group: int = 0, order: str = "rows") -> int:
+    return _lib.load().rb_planes_words(layout(M, K, n_paths, group, order))
 
 
 def scales_count(M: int, K: int, n_paths: int, group: int = 0) -> int:
     return _lib.load().rb_scales_count(layout(M, K, n_paths, group))
+
+
+def _planes_geometry(planes: torch.Tensor, K: int):
+    """(N, M, order) of a planes tensor: [N, M, K/32] rows or [N, S, M, 16] sliced."""
+    if planes.dim() == 3:
+        N, M, W32 = planes.shape
+        if W32 * 32 != K:
+            raise ValueError("planes and x disagree on K")
+        return N, M, "rows"
+    if planes.dim() == 4:
+        N, S, M, sixteen = planes.shape
+        if sixteen != 16 or S != (K + 511) // 512:
+            raise ValueError("sliced planes and x disagree on K")
+        return N, M, "sliced"
+    raise ValueError("planes must be [N, M, K/32] (rows) or [N, S, M, 16] (sliced)")
 
 
 def _require_cuda(*ts: torch.Tensor) -> torch.device:
@@ -46,11 +64,13 @@ def _require_cuda(*ts: torch.Tensor) -> torch.device:
     return dev
 
 
-def pack(W: torch.Tensor, n_paths: int = 2, group: int = 0, alpha_f16: bool = False):
+def pack(W: torch.Tensor, n_paths: int = 2, group: int = 0, alpha_f16: bool = False, order: str = "rows"):
     """Derive N residual sign planes and scales from the shared weight W (M x K).
 
-    Returns (planes int32 [N, M, K/32] holding uint32 words, alpha fp32
-    [N, M, K/G], alpha16 fp16 [N, M, K/G] or None).
+    Returns (planes, alpha fp32 [N, M, K/G], alpha16 fp16 [N, M, K/G] or None).
+    planes holds uint32 words in an int32 tensor: [N, M, K/32] for
+    order="rows", [N, ceil(K/512), M, 16] for order="sliced" (the order the
+    matvec kernel streams fastest).
     """
     lib = _lib.load()
     dev = _require_cuda(W)
@@ -58,11 +78,12 @@ def pack(W: torch.Tensor, n_paths: int = 2, group: int = 0, alpha_f16: bool = Fa
         raise ValueError("W must be a 2-D fp16/fp32 tensor with unit column stride")
     M, K = W.shape
     G = K if group == 0 else group
-    planes = torch.empty((n_paths, M, K // 32), dtype=torch.int32, device=dev)
+    shape = (n_paths, M, K // 32) if order == "rows" else (n_paths, (K + 511) // 512, M, 16)
+    planes = torch.empty(shape, dtype=torch.int32, device=dev)
     alpha = torch.empty((n_paths, M, K // G), dtype=torch.float32, device=dev)
     a16 = torch.empty((n_paths, M, K // G), dtype=torch.float16, device=dev) if alpha_f16 else None
     with torch.cuda.device(dev):
-        check(lib.rb_pack(_p(W), _DT[W.dtype], W.stride(0), layout(M, K, n_paths, group),
+        check(lib.rb_pack(_p(W), _DT[W.dtype], W.stride(0), layout(M, K, n_paths, group, order),
                           _p(planes), _p(alpha), _p(a16), _stream(dev)))
     return planes, alpha, a16
 
@@ -86,12 +107,12 @@ def gemv(planes: torch.Tensor, alpha: torch.Tensor, x: torch.Tensor, group: int 
     lib = _lib.load()
     x = _x2d(x)
     dev = _require_cuda(planes, alpha, x, y, workspace)
-    N, M, W32 = planes.shape
-    K = W32 * 32
+    K = x.shape[1]
+    N, M, order = _planes_geometry(planes, K)
     T = x.shape[0]
     if y is None:
         y = torch.empty((T, M), dtype=y_dtype, device=dev)
-    L = layout(M, K, N, group)
+    L = layout(M, K, N, group, order)
     need = lib.rb_gemv_workspace_bytes(L, T)
     if workspace is None or workspace.numel() * workspace.element_size() < need:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
@@ -115,24 +136,27 @@ class GroupedGemv:
         self.items = list(items)   # keep tensors alive
         n = len(self.items)
         self.host = (GemvDesc * n)()
-        adt = ydt = None
+        adt = ydt = order = None
         dev = None
         for i, (planes, alpha, x, y) in enumerate(self.items):
             dev = _require_cuda(planes, alpha, x, y)
-            N, M, W32 = planes.shape
-            if N != n_paths or x.shape[-1] != W32 * 32 or y.shape[-1] != M:
-                raise ValueError(f"item {i}: inconsistent shapes")
+            K = x.shape[-1]
+            N, M, o = _planes_geometry(planes, K)
+            order = o if order is None else order
+            if N != n_paths or y.shape[-1] != M or o != order:
+                raise ValueError(f"item {i}: inconsistent shapes or plane orders")
             if not (x.is_contiguous() and y.is_contiguous()):
                 raise ValueError(f"item {i}: x and y must be contiguous [T, K] / [T, M]")
             adt = alpha.dtype if adt is None else adt
             ydt = y.dtype if ydt is None else ydt
             if alpha.dtype != adt or y.dtype != ydt:
                 raise ValueError("all items must share the scale and output dtypes")
-            self.host[i] = GemvDesc(planes.data_ptr(), alpha.data_ptr(), x.data_ptr(), y.data_ptr(), M, W32 * 32)
+            self.host[i] = GemvDesc(planes.data_ptr(), alpha.data_ptr(), x.data_ptr(), y.data_ptr(), M, K)
         self.device = dev
         raw = bytes(self.host)
         self.dev_descs = torch.frombuffer(bytearray(raw), dtype=torch.uint8).to(dev)
         self.alpha_dtype, self.y_dtype = _DT[adt], _DT[ydt]
+        self.order = _ORDERS[order]
         need = lib.rb_gemv_grouped_workspace_bytes(self.host, n, n_paths, T)
         self.workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
         self.n = n
@@ -141,7 +165,7 @@ class GroupedGemv:
         lib = _lib.load()
         with torch.cuda.device(self.device):
             check(lib.rb_gemv_grouped(ctypes.cast(self.host, ctypes.c_void_p), _p(self.dev_descs), self.n,
-                                      self.n_paths, self.group, self.alpha_dtype, self.y_dtype, self.T,
+                                      self.n_paths, self.group, self.order, self.alpha_dtype, self.y_dtype, self.T,
                                       _p(self.workspace), self.workspace.numel(), _stream(self.device)))
 
     def check_device_flag(self) -> None:
@@ -156,12 +180,12 @@ def gemm(planes: torch.Tensor, alpha: torch.Tensor, X: torch.Tensor, group: int 
         raise _lib.RbError(2, "this build has no rb_gemm")
     X = _x2d(X)
     dev = _require_cuda(planes, alpha, X, Y)
-    N, M, W32 = planes.shape
-    K = W32 * 32
+    K = X.shape[1]
+    N, M, order = _planes_geometry(planes, K)
     T = X.shape[0]
     if Y is None:
         Y = torch.empty((T, M), dtype=y_dtype, device=dev)
     with torch.cuda.device(dev):
-        check(lib.rb_gemm(_p(planes), _p(alpha), _DT[alpha.dtype], layout(M, K, N, group), _p(X), X.stride(0), T,
+        check(lib.rb_gemm(_p(planes), _p(alpha), _DT[alpha.dtype], layout(M, K, N, group, order), _p(X), X.stride(0), T,
                           _p(Y), _DT[Y.dtype], Y.stride(0), _stream(dev)))
     return Y

@@ -52,10 +52,12 @@ static rb_status check_layout(const rb_layout& L) {
     if (L.K % 128 != 0) return fail(RB_ERR_UNSUPPORTED, "K=%lld is not a multiple of 128", (long long)L.K);
     if (L.n_paths < 1 || L.n_paths > 8) return fail(RB_ERR_UNSUPPORTED, "n_paths=%d outside 1..8", L.n_paths);
     if (L.group != 0 && L.group != 128) return fail(RB_ERR_UNSUPPORTED, "group=%d (0 or 128)", L.group);
-    // plane word offsets and row indices are kept in 32 bits on the device
-    if (static_cast<double>(L.n_paths) * L.M * (L.K / 32) >= 4294967296.0 || L.M >= (1ll << 31) ||
+    if (L.order != RB_ROWS && L.order != RB_SLICED) return fail(RB_ERR_INVALID_ARG, "order=%d", L.order);
+    if (L.reserved != 0) return fail(RB_ERR_INVALID_ARG, "reserved field must be 0");
+    // byte offsets within one path's planes and scale indices are 32-bit on the device
+    if (static_cast<double>(L.M) * 64.0 * ((L.K + 511) / 512) >= 4294967296.0 || L.M >= (1ll << 31) ||
         static_cast<double>(L.n_paths) * L.M * (L.K / 128) >= 4294967296.0)
-        return fail(RB_ERR_UNSUPPORTED, "layout too large (N*M*K/32 must stay below 2^32)");
+        return fail(RB_ERR_UNSUPPORTED, "layout too large (planes of one path must stay below 4 GiB)");
     return RB_OK;
 }
 
@@ -76,6 +78,7 @@ extern "C" {
 
 size_t rb_planes_words(rb_layout L) {
     if (check_layout(L) != RB_OK) return 0;
+    if (L.order == RB_SLICED) return static_cast<size_t>(L.n_paths) * L.M * 16 * ((L.K + 511) / 512);
     return static_cast<size_t>(L.n_paths) * L.M * (L.K / 32);
 }
 
@@ -114,7 +117,7 @@ rb_status rb_pack(const void* W, rb_dtype w_dtype, int64_t ldw, rb_layout L,
     if ((reinterpret_cast<uintptr_t>(alpha) & 3u) || (reinterpret_cast<uintptr_t>(alpha_f16) & 1u))
         return fail(RB_ERR_ALIGNMENT, "alpha must be 4-byte aligned, alpha_f16 2-byte aligned");
     if (L.group == 0 && L.K > 65536) return fail(RB_ERR_UNSUPPORTED, "one scale per row supports K <= 65536");
-    PackArgs a{W, ldw, L.M, L.K, L.n_paths, L.group, w_dtype == RB_F16, planes, alpha,
+    PackArgs a{W, ldw, L.M, L.K, L.n_paths, L.group, w_dtype == RB_F16, L.order == RB_SLICED, planes, alpha,
                static_cast<__half*>(alpha_f16)};
     cudaError_t e = launch_pack(a, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "rb_pack launch");
@@ -163,6 +166,7 @@ rb_status rb_gemv(const uint32_t* planes, const void* alpha, rb_dtype alpha_dtyp
     a.n_jobs = 1;
     a.n_paths = L.n_paths;
     a.group = L.group;
+    a.sliced = L.order == RB_SLICED;
     a.alpha_f16 = alpha_dtype == RB_F16;
     a.y_f16 = y_dtype == RB_F16;
     a.T = T;
@@ -177,11 +181,11 @@ rb_status rb_gemv(const uint32_t* planes, const void* alpha, rb_dtype alpha_dtyp
     return RB_OK;
 }
 
-static rb_status check_descs(const rb_gemv_desc* d, int32_t n, int32_t n_paths, int32_t group) {
+static rb_status check_descs(const rb_gemv_desc* d, int32_t n, int32_t n_paths, int32_t group, int32_t order) {
     if (!d) return fail(RB_ERR_INVALID_ARG, "null descriptors");
     if (n < 1 || n > gemv_max_jobs()) return fail(RB_ERR_UNSUPPORTED, "n=%d outside 1..%d", n, gemv_max_jobs());
     for (int32_t i = 0; i < n; ++i) {
-        rb_layout L{d[i].M, d[i].K, n_paths, group};
+        rb_layout L{d[i].M, d[i].K, n_paths, group, order, 0};
         rb_status st = check_layout(L);
         if (st != RB_OK) return fail(st, "descriptor %d: %s", i, g_last_error.c_str());
         if (!d[i].planes || !d[i].alpha || !d[i].x || !d[i].y)
@@ -206,12 +210,12 @@ size_t rb_gemv_grouped_workspace_bytes(const rb_gemv_desc* descs_host, int32_t n
 }
 
 rb_status rb_gemv_grouped(const rb_gemv_desc* descs_host, const rb_gemv_desc* descs_dev,
-                          int32_t n, int32_t n_paths, int32_t group,
+                          int32_t n, int32_t n_paths, int32_t group, int32_t order,
                           rb_dtype alpha_dtype, rb_dtype y_dtype, int32_t T,
                           void* workspace, size_t ws_bytes, void* stream) {
     g_last_error.clear();
     static_assert(sizeof(rb_gemv_desc) == sizeof(GvJob), "descriptor layout");
-    rb_status st = check_descs(descs_host, n, n_paths, group);
+    rb_status st = check_descs(descs_host, n, n_paths, group, order);
     if (st != RB_OK) return st;
     if (!descs_dev || (reinterpret_cast<uintptr_t>(descs_dev) & 7u))
         return fail(RB_ERR_INVALID_ARG, "descs_dev must be a non-null, 8-byte aligned device pointer");
@@ -230,6 +234,7 @@ rb_status rb_gemv_grouped(const rb_gemv_desc* descs_host, const rb_gemv_desc* de
     a.n_jobs = n;
     a.n_paths = n_paths;
     a.group = group;
+    a.sliced = order == RB_SLICED;
     a.alpha_f16 = alpha_dtype == RB_F16;
     a.y_f16 = y_dtype == RB_F16;
     a.T = T;

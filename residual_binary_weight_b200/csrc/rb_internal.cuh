@@ -22,6 +22,7 @@ struct PackArgs {
     int n_paths;
     int group;          // 0 or 128
     bool w_f16;
+    bool sliced;        // plane words in the sliced order
     uint32_t* planes;
     float* alpha;
     __half* alpha16;    // nullable
@@ -45,6 +46,7 @@ struct GvArgs {
     int n_jobs;
     int n_paths;
     int group;              // 0 or 128
+    bool sliced;            // plane words in the sliced order
     bool alpha_f16;
     bool y_f16;
     int T;

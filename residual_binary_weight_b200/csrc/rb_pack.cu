@@ -76,15 +76,21 @@ __device__ __forceinline__ uint32_t sign_and_update8(float* r, float a, bool upd
 
 template <typename WT, int CPT, int MAXT>
 __global__ void __launch_bounds__(MAXT)
-pack_row_kernel(const WT* __restrict__ W, int64_t ldw, int M, int K, int N,
+pack_row_kernel(const WT* __restrict__ W, int64_t ldw, int M, int K, int N, bool sliced,
                 uint32_t* __restrict__ planes, float* __restrict__ alpha,
                 __half* __restrict__ alpha16) {
     __shared__ double red[32];
     const int row = blockIdx.x;
     const int chunks = K >> 3;
     const WT* wrow = W + static_cast<int64_t>(row) * ldw;
-    uint8_t* pbytes = reinterpret_cast<uint8_t*>(planes) + static_cast<size_t>(row) * chunks;
-    const size_t plane_stride = static_cast<size_t>(M) * chunks;
+    uint8_t* pb = reinterpret_cast<uint8_t*>(planes);
+    const size_t S = (static_cast<size_t>(K) + 511) / 512;
+    // byte `idx` (columns 8 idx .. 8 idx + 7) of path k of this row
+    auto byte_at = [&](int k, int idx) -> uint8_t* {
+        if (!sliced) return pb + (static_cast<size_t>(k) * M + row) * chunks + idx;
+        const int w = idx >> 2;
+        return pb + ((static_cast<size_t>(k) * S + (w >> 4)) * M + row) * 64 + 4 * (w & 15) + (idx & 3);
+    };
 
     float r[CPT][8];
 #pragma unroll
@@ -114,7 +120,7 @@ pack_row_kernel(const WT* __restrict__ W, int64_t ldw, int M, int K, int N,
             const int idx = threadIdx.x + c * blockDim.x;
             if (idx < chunks) {
                 const uint32_t bits = sign_and_update8(r[c], a, update);
-                pbytes[k * plane_stride + idx] = static_cast<uint8_t>(bits);
+                *byte_at(k, idx) = static_cast<uint8_t>(bits);
             }
         }
     }
@@ -135,11 +141,12 @@ __device__ __forceinline__ void load32(const WT* p, float (&v)[32]) {
 // (eight groups per warp per step); lane (4g + q) holds columns 32q..32q+31.
 template <typename WT>
 __global__ void __launch_bounds__(256)
-pack_g128_kernel(const WT* __restrict__ W, int64_t ldw, int M, int K, int N,
+pack_g128_kernel(const WT* __restrict__ W, int64_t ldw, int M, int K, int N, bool sliced,
                  uint32_t* __restrict__ planes, float* __restrict__ alpha,
                  __half* __restrict__ alpha16) {
     const int gpr = K >> 7;
     const int words = K >> 5;
+    const int64_t S = (K + 511) / 512;
     const int64_t total = static_cast<int64_t>(M) * gpr;
     const int lane = threadIdx.x & 31;
     const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
@@ -170,7 +177,9 @@ pack_g128_kernel(const WT* __restrict__ W, int64_t ldw, int M, int K, int N,
 #pragma unroll
             for (int i = 0; i < 4; ++i) word |= sign_and_update8(r + 8 * i, a, update) << (8 * i);
             if (valid) {
-                planes[(static_cast<int64_t>(k) * M + row) * words + wi] = word;
+                const int64_t wo = sliced ? ((k * S + (wi >> 4)) * M + row) * 16 + (wi & 15)
+                                          : (static_cast<int64_t>(k) * M + row) * words + wi;
+                planes[wo] = word;
                 if ((lane & 3) == 0) {
                     const int64_t ai = (static_cast<int64_t>(k) * M + row) * gpr + gi;
                     alpha[ai] = a;
@@ -185,7 +194,7 @@ template <typename WT, int CPT, int MAXT = 1024>
 cudaError_t launch_row(const PackArgs& a, int threads, cudaStream_t s) {
     pack_row_kernel<WT, CPT, MAXT><<<static_cast<unsigned>(a.M), threads, 0, s>>>(
         static_cast<const WT*>(a.W), a.ldw, static_cast<int>(a.M), static_cast<int>(a.K),
-        a.n_paths, a.planes, a.alpha, a.alpha16);
+        a.n_paths, a.sliced, a.planes, a.alpha, a.alpha16);
     return cudaGetLastError();
 }
 
@@ -216,13 +225,21 @@ cudaError_t launch_g128(const PackArgs& a, cudaStream_t s) {
     if (blocks < 1) blocks = 1;
     pack_g128_kernel<WT><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
         static_cast<const WT*>(a.W), a.ldw, static_cast<int>(a.M), static_cast<int>(a.K),
-        a.n_paths, a.planes, a.alpha, a.alpha16);
+        a.n_paths, a.sliced, a.planes, a.alpha, a.alpha16);
     return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_pack(const PackArgs& a, cudaStream_t s) {
+    if (a.sliced && a.K % 512 != 0) {
+        // zero the last slice of every path (its words past K/32 are padding)
+        const size_t S = static_cast<size_t>((a.K + 511) / 512);
+        const size_t pitch = S * static_cast<size_t>(a.M) * 64;
+        char* last = reinterpret_cast<char*>(a.planes) + (S - 1) * static_cast<size_t>(a.M) * 64;
+        cudaError_t e = cudaMemset2DAsync(last, pitch, 0, static_cast<size_t>(a.M) * 64, a.n_paths, s);
+        if (e != cudaSuccess) return e;
+    }
     if (a.group == 0)
         return a.w_f16 ? launch_row_any<__half>(a, s) : launch_row_any<float>(a, s);
     return a.w_f16 ? launch_g128<__half>(a, s) : launch_g128<float>(a, s);

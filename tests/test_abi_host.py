@@ -38,14 +38,19 @@ def test_library_hides_internal_symbols():
 
 def test_sizes():
     lib = _lib.load()
-    assert lib.rb_planes_words(Layout(4096, 4096, 2, 0)) == 2 * 4096 * 128
-    assert lib.rb_scales_count(Layout(4096, 4096, 2, 0)) == 2 * 4096
-    assert lib.rb_scales_count(Layout(11008, 4096, 4, 128)) == 4 * 11008 * 32
+    assert lib.rb_planes_words(Layout(4096, 4096, 2, 0, 0, 0)) == 2 * 4096 * 128
+    assert lib.rb_scales_count(Layout(4096, 4096, 2, 0, 0, 0)) == 2 * 4096
+    assert lib.rb_scales_count(Layout(11008, 4096, 4, 128, 0, 0)) == 4 * 11008 * 32
     # invalid layouts size to zero
-    assert lib.rb_planes_words(Layout(4096, 4000, 2, 0)) == 0
-    assert lib.rb_planes_words(Layout(0, 4096, 2, 0)) == 0
-    assert lib.rb_planes_words(Layout(16, 128, 9, 0)) == 0
-    assert lib.rb_scales_count(Layout(16, 128, 2, 64)) == 0
+    assert lib.rb_planes_words(Layout(4096, 4000, 2, 0, 0, 0)) == 0
+    assert lib.rb_planes_words(Layout(0, 4096, 2, 0, 0, 0)) == 0
+    assert lib.rb_planes_words(Layout(16, 128, 9, 0, 0, 0)) == 0
+    assert lib.rb_scales_count(Layout(16, 128, 2, 64, 0, 0)) == 0
+    # the sliced order pads the last 512-column slice
+    assert lib.rb_planes_words(Layout(4096, 11008, 2, 0, 1, 0)) == 2 * 4096 * 16 * 22
+    assert lib.rb_planes_words(Layout(4096, 4096, 2, 0, 1, 0)) == 2 * 4096 * 128
+    assert lib.rb_planes_words(Layout(16, 128, 2, 0, 2, 0)) == 0
+    assert lib.rb_planes_words(Layout(16, 128, 2, 0, 0, 1)) == 0
 
 
 def test_status_strings():
@@ -63,7 +68,7 @@ def _status(rc):
 
 def test_pack_rejects_bad_arguments_before_launch():
     lib = _lib.load()
-    L = Layout(64, 256, 2, 0)
+    L = Layout(64, 256, 2, 0, 0, 0)
     p = ctypes.c_void_p
     assert _status(lib.rb_pack(None, 0, 256, L, p(FAKE), p(FAKE), None, None)) == "RB_ERR_INVALID_ARG"
     assert _status(lib.rb_pack(p(FAKE), 0, 255, L, p(FAKE), p(FAKE), None, None)) == "RB_ERR_INVALID_ARG"
@@ -71,21 +76,21 @@ def test_pack_rejects_bad_arguments_before_launch():
     assert _status(lib.rb_pack(p(FAKE + 4), 0, 256, L, p(FAKE), p(FAKE), None, None)) == "RB_ERR_ALIGNMENT"
     assert _status(lib.rb_pack(p(FAKE), 1, 260, L, p(FAKE), p(FAKE), None, None)) == "RB_ERR_ALIGNMENT"
     assert _status(lib.rb_pack(p(FAKE), 0, 256, L, p(FAKE + 8), p(FAKE), None, None)) == "RB_ERR_ALIGNMENT"
-    assert _status(lib.rb_pack(p(FAKE), 0, 256, Layout(64, 200, 2, 0), p(FAKE), p(FAKE), None, None)) == \
+    assert _status(lib.rb_pack(p(FAKE), 0, 256, Layout(64, 200, 2, 0, 0, 0), p(FAKE), p(FAKE), None, None)) == \
         "RB_ERR_UNSUPPORTED"
-    assert _status(lib.rb_pack(p(FAKE), 0, 256, Layout(64, 256, 0, 0), p(FAKE), p(FAKE), None, None)) == \
+    assert _status(lib.rb_pack(p(FAKE), 0, 256, Layout(64, 256, 0, 0, 0, 0), p(FAKE), p(FAKE), None, None)) == \
         "RB_ERR_UNSUPPORTED"
-    assert _status(lib.rb_pack(p(FAKE), 0, 256, Layout(64, 256, 2, 32), p(FAKE), p(FAKE), None, None)) == \
+    assert _status(lib.rb_pack(p(FAKE), 0, 256, Layout(64, 256, 2, 32, 0, 0), p(FAKE), p(FAKE), None, None)) == \
         "RB_ERR_UNSUPPORTED"
-    assert _status(lib.rb_pack(p(FAKE), 0, 1 << 17, Layout(4, 1 << 17, 2, 0), p(FAKE), p(FAKE), None, None)) == \
+    assert _status(lib.rb_pack(p(FAKE), 0, 1 << 17, Layout(4, 1 << 17, 2, 0, 0, 0), p(FAKE), p(FAKE), None, None)) == \
         "RB_ERR_UNSUPPORTED"
-    lib.rb_pack(p(FAKE), 0, 256, Layout(64, 200, 2, 0), p(FAKE), p(FAKE), None, None)
+    lib.rb_pack(p(FAKE), 0, 256, Layout(64, 200, 2, 0, 0, 0), p(FAKE), p(FAKE), None, None)
     assert b"multiple of 128" in lib.rb_last_error()
 
 
 def test_gemv_rejects_bad_arguments_before_launch():
     lib = _lib.load()
-    L = Layout(64, 256, 2, 0)
+    L = Layout(64, 256, 2, 0, 0, 0)
     p = ctypes.c_void_p
     ok = (p(FAKE), p(FAKE), 0, L, p(FAKE), 256, 1, p(FAKE), 1, 64, p(FAKE), 1 << 20, None)
 
@@ -106,7 +111,7 @@ def test_gemv_rejects_bad_arguments_before_launch():
     assert call(ws=None) == "RB_ERR_WORKSPACE"
     assert call(wsb=8) == "RB_ERR_WORKSPACE"
     assert call(adt=5) == "RB_ERR_INVALID_ARG"
-    assert call(L=Layout(64, 256, 9, 0)) == "RB_ERR_UNSUPPORTED"
+    assert call(L=Layout(64, 256, 9, 0, 0, 0)) == "RB_ERR_UNSUPPORTED"
 
 
 def test_grouped_rejects_bad_descriptors():
@@ -116,16 +121,16 @@ def test_grouped_rejects_bad_descriptors():
     d[0] = GemvDesc(FAKE, FAKE, FAKE, FAKE, 128, 256)
     d[1] = GemvDesc(FAKE, FAKE, FAKE, FAKE, 128, 200)
     host = ctypes.cast(d, p)
-    rc = lib.rb_gemv_grouped(host, p(FAKE), 2, 2, 0, 0, 1, 1, p(FAKE), 1 << 20, None)
+    rc = lib.rb_gemv_grouped(host, p(FAKE), 2, 2, 0, 0, 0, 1, 1, p(FAKE), 1 << 20, None)
     assert _status(rc) == "RB_ERR_UNSUPPORTED"
     assert b"descriptor 1" in lib.rb_last_error()
     d[1] = GemvDesc(FAKE, None, FAKE, FAKE, 128, 256)
-    assert _status(lib.rb_gemv_grouped(host, p(FAKE), 2, 2, 0, 0, 1, 1, p(FAKE), 1 << 20, None)) == \
+    assert _status(lib.rb_gemv_grouped(host, p(FAKE), 2, 2, 0, 0, 0, 1, 1, p(FAKE), 1 << 20, None)) == \
         "RB_ERR_INVALID_ARG"
     d[1] = GemvDesc(FAKE, FAKE, FAKE, FAKE, 128, 256)
-    assert _status(lib.rb_gemv_grouped(host, None, 2, 2, 0, 0, 1, 1, p(FAKE), 1 << 20, None)) == \
+    assert _status(lib.rb_gemv_grouped(host, None, 2, 2, 0, 0, 0, 1, 1, p(FAKE), 1 << 20, None)) == \
         "RB_ERR_INVALID_ARG"
-    assert _status(lib.rb_gemv_grouped(host, p(FAKE), 0, 2, 0, 0, 1, 1, p(FAKE), 1 << 20, None)) == \
+    assert _status(lib.rb_gemv_grouped(host, p(FAKE), 0, 2, 0, 0, 0, 1, 1, p(FAKE), 1 << 20, None)) == \
         "RB_ERR_UNSUPPORTED"
     assert lib.rb_gemv_grouped_workspace_bytes(host, 2, 2, 1) >= 256
 
@@ -133,7 +138,7 @@ def test_grouped_rejects_bad_descriptors():
 def test_workspace_sizes_follow_the_split():
     lib = _lib.load()
     # one matrix with few rows is split along K, which needs counters and partial sums
-    small = lib.rb_gemv_workspace_bytes(Layout(512, 8192, 2, 0), 1)
+    small = lib.rb_gemv_workspace_bytes(Layout(512, 8192, 2, 0, 0, 0), 1)
     assert small > 256 + 4 * 512
     # a layout that is rejected needs nothing
-    assert lib.rb_gemv_workspace_bytes(Layout(512, 8000, 2, 0), 1) == 0
+    assert lib.rb_gemv_workspace_bytes(Layout(512, 8000, 2, 0, 0, 0), 1) == 0

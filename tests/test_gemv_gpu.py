@@ -29,30 +29,37 @@ def test_layer256_full():
     _ok(check_gemv_on_oracle_planes(W, x, 2, 0, alpha_f16=False), "layer256")
 
 
+ORDERS = ["rows", "sliced"]
+
+
+@pytest.mark.parametrize("order", ORDERS)
 @pytest.mark.parametrize("matrix,rows,T", [("q", 1000, 1), ("gate", 700, 2), ("down", 300, 3)])
-def test_llama2_shapes(matrix, rows, T):
+def test_llama2_shapes(matrix, rows, T, order):
     wl = synth.WORKLOADS["llama2_7b_decode"]
     W = synth.host_rows(wl, 1, matrix, range(rows))
     x = synth.host_activations(wl, 1, matrix, T)
-    _ok(check_gemv_on_oracle_planes(W, x, 2, 0, alpha_f16=False), matrix)
+    _ok(check_gemv_on_oracle_planes(W, x, 2, 0, alpha_f16=False, order=order), matrix)
 
 
+@pytest.mark.parametrize("order", ORDERS)
 @pytest.mark.parametrize("T", [1, 4, 16])
 @pytest.mark.parametrize("matrix,rows", [("up", 200), ("down", 150)])
-def test_qbb_g128(matrix, rows, T):
+def test_qbb_g128(matrix, rows, T, order):
     wl = synth.WORKLOADS["qbb_g128"]
     W = synth.host_rows(wl, 0, matrix, range(rows))
     x = synth.host_activations(wl, 0, matrix, T)
-    _ok(check_gemv_on_oracle_planes(W, x, 4, 128, alpha_f16=True), (matrix, T))
+    _ok(check_gemv_on_oracle_planes(W, x, 4, 128, alpha_f16=True, order=order), (matrix, T))
 
 
-@pytest.mark.parametrize("n_paths", [1, 3, 5, 8])
+@pytest.mark.parametrize("order", ORDERS)
+@pytest.mark.parametrize("n_paths", [1, 3, 5, 6, 8])
 @pytest.mark.parametrize("group", [0, 128])
-def test_path_counts(n_paths, group):
+def test_path_counts(n_paths, group, order):
     rng = np.random.default_rng(7 * n_paths + group)
     W = (rng.standard_normal((333, 1152)) * 0.02).astype(np.float16)
     x = rng.standard_normal((2, 1152)).astype(np.float16)
-    _ok(check_gemv_on_oracle_planes(W, x, n_paths, group, alpha_f16=(group == 128)), (n_paths, group))
+    _ok(check_gemv_on_oracle_planes(W, x, n_paths, group, alpha_f16=(group == 128), order=order),
+        (n_paths, group))
 
 
 @pytest.mark.parametrize("alpha_f16,y_dtype", [(True, torch.float32), (False, torch.float32), (True, torch.float16)])
@@ -64,24 +71,26 @@ def test_dtypes_and_pitches(alpha_f16, y_dtype):
     _ok(check_gemv_on_oracle_planes(W, x, 2, 128, alpha_f16, y_dtype, ldx_pad=8, ldy_pad=3), "pitch g128")
 
 
+@pytest.mark.parametrize("order", ORDERS)
 @pytest.mark.parametrize("K", [128, 384, 640])
-def test_small_and_ragged(K):
+def test_small_and_ragged(K, order):
     rng = np.random.default_rng(K)
-    for M in (1, 33):
+    for M in (1, 33, 514):
         W = (rng.standard_normal((M, K)) * 0.02).astype(np.float32)
         x = rng.standard_normal((1, K)).astype(np.float16)
-        _ok(check_gemv_on_oracle_planes(W, x, 2, 0, False), (M, K))
-        _ok(check_gemv_on_oracle_planes(W, x, 2, 128, False), (M, K, 128))
+        _ok(check_gemv_on_oracle_planes(W, x, 2, 0, False, order=order), (M, K))
+        _ok(check_gemv_on_oracle_planes(W, x, 2, 128, False, order=order), (M, K, 128))
 
 
-def test_split_k_single_matrix():
+@pytest.mark.parametrize("order", ORDERS)
+def test_split_k_single_matrix(order):
     """Few rows and long rows: the single-matrix plan splits K into chunks and
     the last CTA of a row block adds the partial sums."""
     rng = np.random.default_rng(11)
     W = (rng.standard_normal((64, 28672)) * 0.02).astype(np.float16)
     x = rng.standard_normal((1, 28672)).astype(np.float16)
-    _ok(check_gemv_on_oracle_planes(W, x, 2, 0, False), "split")
-    _ok(check_gemv_on_oracle_planes(W, x, 4, 128, True), "split g128")
+    _ok(check_gemv_on_oracle_planes(W, x, 2, 0, False, order=order), "split")
+    _ok(check_gemv_on_oracle_planes(W, x, 4, 128, True, order=order), "split g128")
 
 
 def test_x_equal_one_and_unit_vectors():
@@ -108,7 +117,7 @@ def test_x_equal_one_and_unit_vectors():
         assert np.allclose(y, col, rtol=1e-6, atol=1e-9)
 
 
-def _grouped_case(wl_name, layer, scale_rows, T, n_paths, group, alpha_f16):
+def _grouped_case(wl_name, layer, scale_rows, T, n_paths, group, alpha_f16, order="rows"):
     wl = synth.WORKLOADS[wl_name]
     items, refs = [], []
     for spec in wl.matrices:
@@ -119,14 +128,16 @@ def _grouped_case(wl_name, layer, scale_rows, T, n_paths, group, alpha_f16):
         stored = oracle.alpha_to_f16(ref_a) if alpha_f16 else ref_a.astype(np.float32)
         y_ref, den = oracle.matvec(ref_p, stored.astype(np.float64), x.astype(np.float64))
         y = torch.full((T, M), float("nan"), dtype=torch.float16, device="cuda")
-        items.append((to_dev_planes(ref_p), torch.from_numpy(stored).cuda(), torch.from_numpy(x).cuda(), y))
+        items.append((to_dev_planes(ref_p, order=order), torch.from_numpy(stored).cuda(),
+                      torch.from_numpy(x).cuda(), y))
         refs.append((y_ref, den))
     return items, refs
 
 
+@pytest.mark.parametrize("order", ORDERS)
 @pytest.mark.parametrize("T", [1, 2])
-def test_grouped_llama2_layer(T):
-    items, refs = _grouped_case("llama2_7b_decode", 2, 8, T, 2, 0, False)
+def test_grouped_llama2_layer(T, order):
+    items, refs = _grouped_case("llama2_7b_decode", 2, 8, T, 2, 0, False, order)
     g = rb.GroupedGemv(items, n_paths=2, group=0, T=T)
     for _ in range(2):              # the work counter is cleared on every call
         for it in items:
@@ -139,8 +150,9 @@ def test_grouped_llama2_layer(T):
             assert nbad == 0, worst
 
 
-def test_grouped_qbb_g128():
-    items, refs = _grouped_case("qbb_g128", 0, 16, 1, 4, 128, True)
+@pytest.mark.parametrize("order", ORDERS)
+def test_grouped_qbb_g128(order):
+    items, refs = _grouped_case("qbb_g128", 0, 16, 1, 4, 128, True, order)
     g = rb.GroupedGemv(items, n_paths=4, group=128, T=1)
     g.run()
     torch.cuda.synchronize()
@@ -152,7 +164,8 @@ def test_grouped_qbb_g128():
 
 def test_full_size_layer_sampled_rows():
     """One full Llama-2-7B-shaped layer (7 matrices) drawn on the device,
-    packed and evaluated by one grouped launch. For 48 sampled rows per
+    packed in the sliced order and evaluated by one grouped launch (the
+    bench's configuration). For 48 sampled rows per
     matrix the oracle packs the host copy of the weight row; the GPU planes of
     those rows must match, and after the rows are replaced by the oracle's
     planes and scales, the GPU outputs must match the oracle's."""
@@ -162,15 +175,15 @@ def test_full_size_layer_sampled_rows():
     for spec in wl.matrices:
         W = synth.device_weight(wl, 0, spec.name, "cuda")
         x = synth.device_activations(wl, 0, spec.name, 1, "cuda")
-        planes, alpha, _ = rb.pack(W, 2, 0)
+        planes, alpha, _ = rb.pack(W, 2, 0, order="sliced")       # [N, S, M, 16]
         rows = np.sort(rng.choice(spec.M, 48, replace=False))
         idx = torch.from_numpy(rows).cuda()
         Wr = W.index_select(0, idx).cpu().numpy()
         ref_p, ref_a, rabs = oracle.pack(Wr, 2, 0, want_rabs=True)
-        rep = oracle.compare_planes(planes_np(planes[:, idx]), ref_p, rabs, ref_a)
+        rep = oracle.compare_planes(planes_np(planes[:, :, idx], spec.K), ref_p, rabs, ref_a)
         assert rep.bad == 0, (spec.name, rep)
         assert oracle.compare_scales(alpha[:, idx].cpu().numpy(), ref_a)[0] == 0
-        planes[:, idx] = to_dev_planes(ref_p)
+        planes[:, :, idx] = to_dev_planes(ref_p, order="sliced")
         a32 = ref_a.astype(np.float32)
         alpha[:, idx] = torch.from_numpy(a32).cuda()
         del W

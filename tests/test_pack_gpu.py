@@ -17,27 +17,30 @@ def _ok(res, what):
     assert nbad16 == 0, what
 
 
-def test_layer256_full():
+@pytest.mark.parametrize("order", ["rows", "sliced"])
+def test_layer256_full(order):
     wl = synth.WORKLOADS["layer256"]
     W = synth.host_weight(wl, 0, "w")
     assert W.dtype == np.float32
-    _ok(check_pack(W, 2, 0), "layer256")
+    _ok(check_pack(W, 2, 0, order=order), "layer256")
 
 
+@pytest.mark.parametrize("order", ["rows", "sliced"])
 @pytest.mark.parametrize("matrix,rows", [("q", 256), ("gate", 192), ("down", 160)])
-def test_llama2_shapes_row_scales(matrix, rows):
+def test_llama2_shapes_row_scales(matrix, rows, order):
     wl = synth.WORKLOADS["llama2_7b_decode"]
     spec = {m.name: m for m in wl.matrices}[matrix]
     W = synth.host_rows(wl, 3, matrix, range(rows))
     assert W.shape == (rows, spec.K)
-    _ok(check_pack(W, 2, 0), matrix)
+    _ok(check_pack(W, 2, 0, order=order), matrix)
 
 
+@pytest.mark.parametrize("order", ["rows", "sliced"])
 @pytest.mark.parametrize("matrix,rows", [("up", 192), ("down", 96)])
-def test_qbb_g128_four_paths(matrix, rows):
+def test_qbb_g128_four_paths(matrix, rows, order):
     wl = synth.WORKLOADS["qbb_g128"]
     W = synth.host_rows(wl, 0, matrix, range(rows))
-    _ok(check_pack(W, 4, 128), matrix)
+    _ok(check_pack(W, 4, 128, order=order), matrix)
 
 
 @pytest.mark.parametrize("matrix,rows", [("attn", 48), ("down", 24)])
@@ -55,14 +58,15 @@ def test_path_counts(n_paths, group):
     _ok(check_pack(W, n_paths, group), (n_paths, group))
 
 
+@pytest.mark.parametrize("order", ["rows", "sliced"])
 @pytest.mark.parametrize("K", [128, 384, 1152])
 @pytest.mark.parametrize("group", [0, 128])
-def test_ragged_and_minimum_shapes(K, group):
+def test_ragged_and_minimum_shapes(K, group, order):
     rng = np.random.default_rng(K)
     W = (rng.standard_normal((3, K)) * 0.05).astype(np.float32)
-    _ok(check_pack(W, 2, group), (K, group))
+    _ok(check_pack(W, 2, group, order=order), (K, group))
     W1 = W[:1]
-    _ok(check_pack(W1, 2, group), (1, K, group))
+    _ok(check_pack(W1, 2, group, order=order), (1, K, group))
 
 
 def test_row_pitch_and_fp32_groups():
