@@ -175,6 +175,34 @@ RB_API size_t rb_gemv_grouped_workspace_bytes(const rb_gemv_desc* descs_host, in
                                        int32_t n_paths, int32_t T);
 
 /*
+ * rb_gemv_noalloc -- rb_gemv for callers that cannot allocate device memory.
+ * (An addition of this library; the paper has no counterpart.) Some callers
+ * have no way to obtain a workspace: code that runs where cudaMalloc is not
+ * allowed or not wanted -- a real-time decode loop that must not take the
+ * implicit device synchronisation of an allocation, a plug-in inside a host
+ * framework that owns every device buffer, or a fixed-budget deployment that
+ * forbids allocations after start-up. For them the scratch rb_gemv keeps in
+ * the workspace (work counters and K-split partial sums) lives in one static
+ * 2 MiB device array per GPU, held by every GPU that loads the library until
+ * the process exits. The caller still passes planes, scales, x and y, with
+ * the same meaning, layout and checks as rb_gemv.
+ *
+ * - Shapes whose scratch would exceed 2 MiB (rb_gemv_workspace_bytes(L, T) >
+ *   2 MiB) are refused with RB_ERR_UNSUPPORTED before any CUDA call.
+ * - The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.
+ * - Every call on a device shares the array, and a call clears the part that
+ *   must start at zero (a memset on `stream`). Calls whose work may overlap
+ *   on the GPU -- on different streams of one device -- race on the array and
+ *   must be ordered by the caller.
+ * - Nothing here calls cudaMalloc, cudaFree or any allocating routine.
+ */
+RB_API rb_status rb_gemv_noalloc(const uint32_t* planes, const void* alpha, rb_dtype alpha_dtype,
+                                 rb_layout L, const void* x, int64_t ldx, int32_t T,
+                                 void* y, rb_dtype y_dtype, int64_t ldy, void* stream);
+
+/*
  * rb_gemv_check -- wait for `stream`, then report RB_ERR_DEVICE if a matvec
  * kernel that used `workspace` recorded a failure, else RB_OK.
  */

@@ -22,7 +22,7 @@ RB_ROWS, RB_SLICED = 0, 1
 # every symbol include/rb_api.h declares
 EXPORTED = ("rb_planes_words", "rb_scales_count", "rb_status_string", "rb_last_error",
             "rb_pack", "rb_gemv", "rb_gemv_workspace_bytes", "rb_gemv_grouped",
-            "rb_gemv_grouped_workspace_bytes", "rb_gemv_check",
+            "rb_gemv_grouped_workspace_bytes", "rb_gemv_check", "rb_gemv_noalloc",
             "rb_gemm")
 
 
@@ -79,6 +79,8 @@ def load() -> ctypes.CDLL:
         lib.rb_gemv_grouped_workspace_bytes.restype = sz
         lib.rb_gemv_check.argtypes = [vp, vp]
         lib.rb_gemv_check.restype = st
+        lib.rb_gemv_noalloc.argtypes = [vp, vp, st, Layout, vp, i64, i32, vp, st, i64, vp]
+        lib.rb_gemv_noalloc.restype = st
         if hasattr(lib, "rb_gemm"):
             lib.rb_gemm.argtypes = [vp, vp, st, Layout, vp, i64, i32, vp, st, i64, vp]
             lib.rb_gemm.restype = st

@@ -25,6 +25,8 @@ static rb_status fail(rb_status s, const char* fmt, ...) {
     return s;
 }
 
+void set_error_message(const char* msg) { g_last_error = msg; }
+
 static rb_status cuda_fail(cudaError_t e, const char* where) {
     return fail(RB_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
 }
