@@ -175,6 +175,31 @@ RB_API size_t rb_gemv_grouped_workspace_bytes(const rb_gemv_desc* descs_host, in
                                        int32_t n_paths, int32_t T);
 
 /*
+ * rb_gemm -- Y_t = sum_k alpha_k (.) (B_k X_t) for a prefill block of T
+ * tokens on the tcgen05 tensor cores. The plane bits are expanded exactly to
+ * fp16 +-1 (one scale per row: one fp32 accumulator per path in tensor
+ * memory, scaled by alpha_k in the epilogue) or to +-alpha_k in fp16 (one
+ * scale per 128 columns; alpha is then read as fp16, exact when alpha_dtype
+ * is RB_F16), multiplied with fp16 X and accumulated in fp32.
+ *
+ * planes    device, rb_planes_words(L) words in L.order; 16-byte aligned.
+ * alpha     device, rb_scales_count(L) scales of type alpha_dtype.
+ * X         device, fp16 [T][ldx], ldx >= K, base and row pitch 16-byte aligned.
+ * Y         device, out, [T][ldy] of type y_dtype, ldy >= M.
+ * L         1..4 paths.  T >= 1.
+ * Errors: validation as rb_gemv; RB_ERR_CUDA if the tensor-map encoder or the
+ *         launch fails. A kernel whose pipeline waits ran out records a code
+ *         that rb_gemm_check() reports.
+ */
+RB_API rb_status rb_gemm(const uint32_t* planes, const void* alpha, rb_dtype alpha_dtype, rb_layout L,
+                         const void* X, int64_t ldx, int32_t T, void* Y, rb_dtype y_dtype, int64_t ldy,
+                         void* stream);
+
+/* rb_gemm_check -- wait for `stream`, then report RB_ERR_DEVICE (and clear
+ * the record) if an rb_gemm kernel recorded a failure, else RB_OK. */
+RB_API rb_status rb_gemm_check(void* stream);
+
+/*
  * rb_gemv_noalloc -- rb_gemv for callers that cannot allocate device memory.
  * (An addition of this library; the paper has no counterpart.) Some callers
  * have no way to obtain a workspace: code that runs where cudaMalloc is not

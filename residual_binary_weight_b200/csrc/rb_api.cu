@@ -251,6 +251,39 @@ rb_status rb_gemv_grouped(const rb_gemv_desc* descs_host, const rb_gemv_desc* de
     return RB_OK;
 }
 
+rb_status rb_gemm(const uint32_t* planes, const void* alpha, rb_dtype alpha_dtype, rb_layout L,
+                  const void* X, int64_t ldx, int32_t T, void* Y, rb_dtype y_dtype, int64_t ldy, void* stream) {
+    g_last_error.clear();
+    rb_status st = check_layout(L);
+    if (st != RB_OK) return st;
+    if (!planes || !alpha || !X || !Y) return fail(RB_ERR_INVALID_ARG, "null planes, alpha, X or Y");
+    if (!valid_dtype(alpha_dtype) || !valid_dtype(y_dtype)) return fail(RB_ERR_INVALID_ARG, "bad dtype");
+    if (!gemm_supported(L.n_paths, L.group)) return fail(RB_ERR_UNSUPPORTED, "rb_gemm supports 1..4 paths");
+    if (T < 1 || T > (1 << 24)) return fail(RB_ERR_UNSUPPORTED, "T=%d outside 1..2^24", T);
+    if (ldx < L.K || ldy < L.M) return fail(RB_ERR_INVALID_ARG, "ldx < K or ldy < M");
+    if (!aligned16(planes) || !aligned16(X) || (ldx * 2) % 16 != 0)
+        return fail(RB_ERR_ALIGNMENT, "planes, X and the row pitch of X must be 16-byte aligned");
+    if (reinterpret_cast<uintptr_t>(alpha) & (dtype_size(alpha_dtype) - 1))
+        return fail(RB_ERR_ALIGNMENT, "alpha misaligned for its dtype");
+    if (reinterpret_cast<uintptr_t>(Y) & (dtype_size(y_dtype) - 1)) return fail(RB_ERR_ALIGNMENT, "Y misaligned");
+    cudaError_t e = launch_gemm(planes, alpha, alpha_dtype == RB_F16, L.M, L.K, L.n_paths, L.group,
+                                L.order == RB_SLICED, X, ldx, T, Y, y_dtype == RB_F16, ldy,
+                                static_cast<cudaStream_t>(stream));
+    if (e == cudaErrorNotSupported) return fail(RB_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+    if (e != cudaSuccess) return cuda_fail(e, "rb_gemm launch");
+    return RB_OK;
+}
+
+rb_status rb_gemm_check(void* stream) {
+    g_last_error.clear();
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    unsigned int code = 0;
+    if (e == cudaSuccess) e = gemm_read_error(&code);
+    if (e != cudaSuccess) return cuda_fail(e, "rb_gemm_check");
+    if (code) return fail(RB_ERR_DEVICE, "rb_gemm kernel wait ran out (code 0x%x)", code);
+    return RB_OK;
+}
+
 rb_status rb_gemv_check(const void* workspace, void* stream) {
     g_last_error.clear();
     if (!workspace) return fail(RB_ERR_INVALID_ARG, "null workspace");

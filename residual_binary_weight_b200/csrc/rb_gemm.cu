@@ -1,0 +1,452 @@
+// rb_gemm: Y = sum_k alpha_k (.) (B_k X^T) for a block of T tokens on the
+// tcgen05 tensor cores (sm_100a).
+//
+// The per-path contraction B_k X^T is a dense GEMM with a +-1 operand: the
+// plane bits are expanded exactly to fp16 +-1.0 (or, with one scale per 128
+// columns, to +-alpha_k in fp16, which is exact because alpha_k is stored in
+// fp16) and multiplied on the tensor cores with fp32 accumulation in tensor
+// memory; per-row scales multiply the per-path accumulators in the epilogue
+// (RaBiT section 4.1: y = sum_k alpha_k (.) (B_k x); QBB W(4x1)A16g128).
+//
+// One CTA computes a 128-row x BN-token tile over all of K:
+//   warp 0     one thread issues TMA loads of X tiles (BN tokens x 64 columns,
+//              128-byte swizzle) into a STAGES-deep ring;
+//   warp 1     allocates tensor memory and one thread issues
+//              tcgen05.mma.cta_group::1.kind::f16 (M=128, N=BN, K=16), one
+//              accumulator per path (per-row scales) or one in all;
+//   warps 4-7  expand the plane bits of their row (thread = row) into the
+//              K-major 128-byte-swizzled fp16 A tile of every path, then run
+//              the epilogue: tcgen05.ld of the accumulators, scale, fp16/fp32
+//              store.
+// Stages are handed over with mbarriers: full[s] (TMA bytes + 128 expansion
+// arrivals) and empty[s] (tcgen05.commit after the MMAs that read stage s).
+// Every wait is bounded; a wait that runs out records an error code, raises
+// a CTA-wide abort flag and the kernel winds down instead of hanging.
+#include "rb_internal.cuh"
+
+#include <cuda.h>
+
+namespace rb {
+namespace {
+
+constexpr int BM = 128;          // rows per tile (UMMA M)
+constexpr int BK = 64;           // columns per stage (one 128-byte swizzle row of fp16)
+constexpr int THREADS = 256;
+constexpr int EXP_WARP0 = 4;     // first expansion/epilogue warp
+constexpr uint32_t A_TILE_BYTES = BM * BK * 2;   // 16 KB
+constexpr uint32_t WAIT_LIMIT = 1u << 26;
+
+__device__ unsigned int g_gemm_error;   // first failure code of any rb_gemm launch
+
+__device__ __forceinline__ uint32_t elect_lane0() { return (threadIdx.x & 31) == 0; }
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait for phase `parity` of barrier `bar`. Returns false (after
+// recording `code` and raising the CTA abort flag) if it runs out, or at once
+// if another thread already aborted.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile uint32_t* abort_flag,
+                                          uint32_t code) {
+    for (uint32_t i = 0; i < WAIT_LIMIT; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+    }
+    atomicOr(&g_gemm_error, code);
+    *abort_flag = 1u;
+    return false;
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// UMMA shared-memory descriptor of a K-major tile in the 128-byte swizzle
+// layout: 8-row atoms of 1024 bytes (leading offset 16 B, stride 1024 B).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr) {
+    return static_cast<uint64_t>((addr >> 4) & 0x3FFFu) | (static_cast<uint64_t>(1) << 16) |
+           (static_cast<uint64_t>(1024 >> 4) << 32) | (static_cast<uint64_t>(1) << 46) |
+           (static_cast<uint64_t>(2) << 61);
+}
+
+// kind::f16 instruction descriptor: fp32 accumulator, fp16 A and B, both
+// K-major, M = 128, N = BN.
+__host__ __device__ constexpr uint32_t instr_desc(int bn) {
+    return (1u << 4) | (static_cast<uint32_t>(bn >> 3) << 17) | (static_cast<uint32_t>(BM >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(dst), "l"(map), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+                 : "memory");
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t lop_sign(uint32_t value, uint32_t mask) {
+    // value | (~mask & 0x80008000): clear bit -> negative half
+    return value | (~mask & 0x80008000u);
+}
+
+// Expand one 32-column word of plane bits into 16 half2 (+-v, v = `val2`
+// in both halves): half2 i holds columns 2i, 2i+1. Bit c sits at the most
+// significant bit of byte c/8 of (w << (7 - c % 8)); PRMT replicates those
+// sign bits into a mask, which decides the sign of each half.
+__device__ __forceinline__ void expand_word(uint32_t w, uint32_t val2, uint32_t (&h)[16]) {
+    uint32_t s[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) s[k] = w << (7 - k);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const int m = i & 3, b = i >> 2;
+        // byte 1 <- sign of byte b of s[2m] (column 2i); byte 3 <- sign of byte b of s[2m+1] (column 2i+1)
+        const uint32_t sel = (static_cast<uint32_t>(8 | b) << 4) | (static_cast<uint32_t>(8 | (4 + b)) << 12);
+        h[i] = lop_sign(val2, prmt(s[2 * m], s[2 * m + 1], sel));
+    }
+}
+
+struct GemmArgs {
+    const uint32_t* planes;
+    const void* alpha;
+    void* y;
+    int64_t M, K, ldy;
+    int T;
+    int n_paths;
+    bool g128;
+    bool sliced;
+    bool alpha_f16;
+    bool y_f16;
+};
+
+template <int NP, int BN, int STAGES, bool G128>
+struct GemmCfg {
+    static constexpr int NACC = G128 ? 1 : NP;                         // accumulators
+    static constexpr uint32_t B_TILE_BYTES = BN * BK * 2;
+    static constexpr uint32_t STAGE_BYTES = NP * A_TILE_BYTES + B_TILE_BYTES;
+    static constexpr uint32_t TMEM_COLS = (NACC * BN <= 32) ? 32 : (NACC * BN <= 64) ? 64 :
+                                          (NACC * BN <= 128) ? 128 : (NACC * BN <= 256) ? 256 : 512;
+    static constexpr uint32_t SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+    static_assert(NACC * BN <= 512, "accumulators exceed tensor memory");
+};
+
+template <int NP, int BN, int STAGES, bool G128>
+__global__ void __launch_bounds__(THREADS, 1)
+gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, GemmArgs a) {
+    using C = GemmCfg<NP, BN, STAGES, G128>;
+    extern __shared__ __align__(1024) unsigned char dsm[];
+    // 1024-byte aligned tile area (the 128-byte swizzle repeats every 1024 B)
+    const uint32_t raw = smem_addr(dsm);
+    const uint32_t tiles = (raw + 1023u) & ~1023u;
+    const uint32_t bars = tiles + STAGES * C::STAGE_BYTES;     // full[STAGES], empty[STAGES], accf
+    auto full_bar = [&](int s) { return bars + 8u * s; };
+    auto empty_bar = [&](int s) { return bars + 8u * (STAGES + s); };
+    const uint32_t acc_bar = bars + 8u * (2 * STAGES);
+    const uint32_t tmem_slot = acc_bar + 8u;
+    const uint32_t abort_slot = tmem_slot + 4u;
+    volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(dsm + (abort_slot - raw));
+    auto a_tile = [&](int s, int p) { return tiles + s * C::STAGE_BYTES + p * A_TILE_BYTES; };
+    auto b_tile = [&](int s) { return tiles + s * C::STAGE_BYTES + NP * A_TILE_BYTES; };
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int row_tile = blockIdx.x, tok_tile = blockIdx.y;
+    const int64_t M = a.M, K = a.K;
+    const int nk = static_cast<int>(K / BK);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(full_bar(s), 1 + 128);
+            mbar_init(empty_bar(s), 1);
+        }
+        mbar_init(acc_bar, 1);
+        *abort_flag = 0u;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(tmem_slot),
+                     "r"(C::TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(dsm + (tmem_slot - raw));
+
+    if (warp == 0) {
+        // ---------------------------------------------------------- TMA producer
+        if (elect_lane0()) {
+            for (int kb = 0; kb < nk; ++kb) {
+                const int s = kb % STAGES;
+                const uint32_t ph = static_cast<uint32_t>(kb / STAGES) & 1u;
+                if (!mbar_wait(empty_bar(s), ph ^ 1u, abort_flag, 1u)) break;
+                mbar_arrive_expect_tx(full_bar(s), C::B_TILE_BYTES);
+                tma_load_2d(b_tile(s), &xmap, kb * BK, tok_tile * BN, full_bar(s));
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------- MMA issuer
+        if (elect_lane0()) {
+            constexpr uint32_t idesc = instr_desc(BN);
+            bool ok = true;
+            for (int kb = 0; kb < nk && ok; ++kb) {
+                const int s = kb % STAGES;
+                const uint32_t ph = static_cast<uint32_t>(kb / STAGES) & 1u;
+                if (!mbar_wait(full_bar(s), ph, abort_flag, 2u)) { ok = false; break; }
+                tc_fence_after();
+#pragma unroll
+                for (int p = 0; p < NP; ++p) {
+                    const uint32_t d = tmem_base + static_cast<uint32_t>(G128 ? 0 : p * BN);
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        const uint64_t ad = smem_desc(a_tile(s, p) + 32u * kk);
+                        const uint64_t bd = smem_desc(b_tile(s) + 32u * kk);
+                        const uint32_t acc = (kb > 0 || kk > 0 || (G128 && p > 0)) ? 1u : 0u;
+                        umma_f16(d, ad, bd, idesc, acc);
+                    }
+                }
+                umma_commit(empty_bar(s));      // stage s is free once these MMAs completed
+            }
+            umma_commit(acc_bar);               // accumulators complete
+        }
+    } else if (warp >= EXP_WARP0) {
+        // ------------------------------------------------- expansion, then epilogue
+        const int r = (warp - EXP_WARP0) * 32 + lane;            // row within the tile
+        const int64_t row = static_cast<int64_t>(row_tile) * BM + r;
+        const int64_t crow = row < M ? row : M - 1;               // rows past M read a real row
+        const int64_t W32 = K >> 5;
+        const int64_t S = (K + 511) >> 9;
+        const int64_t gpr = K >> 7;
+        // the two words (64 columns) of stage kb of path p of this row
+        auto words_at = [&](int p, int kb) -> uint2 {
+            const int64_t w = 2 * static_cast<int64_t>(kb);
+            const uint32_t* src = a.sliced ? a.planes + ((p * S + (w >> 4)) * M + crow) * 16 + (w & 15)
+                                           : a.planes + (p * M + crow) * W32 + w;
+            return __ldg(reinterpret_cast<const uint2*>(src));
+        };
+        auto alpha_h2 = [&](int p, int kb) -> uint32_t {
+            if (!G128) return 0x3C003C00u;                             // +1.0 in both halves
+            const int64_t ai = (p * M + crow) * gpr + (static_cast<int64_t>(kb) * BK >> 7);
+            uint32_t hv;
+            if (a.alpha_f16) hv = static_cast<const unsigned short*>(a.alpha)[ai];
+            else hv = __half_as_ushort(__float2half_rn(static_cast<const float*>(a.alpha)[ai]));
+            return hv | (hv << 16);
+        };
+        const uint32_t rsw = static_cast<uint32_t>(r & 7);
+        const uint32_t row_off = static_cast<uint32_t>(r >> 3) * 1024u + rsw * 128u;
+        uint2 nxt[NP];
+#pragma unroll
+        for (int p = 0; p < NP; ++p) nxt[p] = words_at(p, 0);
+        for (int kb = 0; kb < nk; ++kb) {
+            const int s = kb % STAGES;
+            const uint32_t ph = static_cast<uint32_t>(kb / STAGES) & 1u;
+            uint2 cur[NP];
+#pragma unroll
+            for (int p = 0; p < NP; ++p) {
+                cur[p] = nxt[p];
+                if (kb + 1 < nk) nxt[p] = words_at(p, kb + 1);
+            }
+            if (!mbar_wait(empty_bar(s), ph ^ 1u, abort_flag, 4u)) break;
+#pragma unroll
+            for (int p = 0; p < NP; ++p) {
+                const uint32_t v2 = alpha_h2(p, kb);
+                const uint32_t base = a_tile(s, p) + row_off;
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t h[16];
+                    expand_word(half ? cur[p].y : cur[p].x, v2, h);
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        const uint32_t chunk = static_cast<uint32_t>(4 * half + c4);   // 16-byte chunk 0..7
+                        sts128(base + ((chunk ^ rsw) << 4), h[4 * c4], h[4 * c4 + 1], h[4 * c4 + 2], h[4 * c4 + 3]);
+                    }
+                }
+            }
+            fence_proxy_async_smem();          // make the generic-proxy stores visible to the tensor core
+            mbar_arrive(full_bar(s));
+        }
+
+        // ------------------------------------------------------------ epilogue
+        const bool ok = mbar_wait(acc_bar, 0u, abort_flag, 8u);
+        tc_fence_after();
+        if (ok) {
+            float al[C::NACC];
+#pragma unroll
+            for (int p = 0; p < C::NACC; ++p) {
+                if (G128) al[p] = 1.0f;
+                else al[p] = a.alpha_f16 ? __half2float(static_cast<const __half*>(a.alpha)[p * M + crow])
+                                         : static_cast<const float*>(a.alpha)[p * M + crow];
+            }
+            const uint32_t lane_addr = static_cast<uint32_t>((warp - EXP_WARP0) * 32) << 16;
+            const int t_base = tok_tile * BN;
+            for (int c0 = 0; c0 < BN; c0 += 32) {
+                float yv[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) yv[i] = 0.0f;
+#pragma unroll
+                for (int p = 0; p < C::NACC; ++p) {
+                    uint32_t v[32];
+                    const uint32_t taddr = tmem_base + lane_addr + static_cast<uint32_t>(p * BN + c0);
+                    asm volatile(
+                        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+                        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+                        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+                        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+                          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+                          "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]),
+                          "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]),
+                          "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+                        : "r"(taddr));
+                    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) yv[i] = fmaf(al[p], __uint_as_float(v[i]), yv[i]);
+                }
+                if (row < M) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int t = t_base + c0 + i;
+                        if (t < a.T) {
+                            if (a.y_f16) static_cast<__half*>(a.y)[t * a.ldy + row] = __float2half_rn(yv[i]);
+                            else static_cast<float*>(a.y)[t * a.ldy + row] = yv[i];
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    __syncwarp();            // lanes 1..31 of warps 0 and 1 wait for their lane 0
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(C::TMEM_COLS)
+                     : "memory");
+    }
+}
+
+// ---------------------------------------------------------------- host side
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+template <int NP, int BN, int STAGES, bool G128>
+cudaError_t launch_cfg(const GemmArgs& a, const void* X, int64_t ldx, cudaStream_t s) {
+    using C = GemmCfg<NP, BN, STAGES, G128>;
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return cudaErrorNotSupported;
+    CUtensorMap map;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.K), static_cast<cuuint64_t>(a.T)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ldx) * 2};
+    const cuuint32_t box[2] = {BK, BN};
+    const cuuint32_t estr[2] = {1, 1};
+    if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(X), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    auto kern = gemm_tc_kernel<NP, BN, STAGES, G128>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    dim3 grid(static_cast<unsigned>((a.M + BM - 1) / BM), static_cast<unsigned>((a.T + BN - 1) / BN));
+    kern<<<grid, THREADS, C::SMEM_BYTES, s>>>(map, a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool gemm_supported(int n_paths, int group) { return n_paths >= 1 && n_paths <= 4 && (group == 0 || group == 128); }
+
+cudaError_t launch_gemm(const uint32_t* planes, const void* alpha, bool alpha_f16, int64_t M, int64_t K, int n_paths,
+                        int group, bool sliced, const void* X, int64_t ldx, int T, void* Y, bool y_f16, int64_t ldy,
+                        cudaStream_t s) {
+    GemmArgs a{planes, alpha, Y, M, K, ldy, T, n_paths, group == 128, sliced, alpha_f16, y_f16};
+    if (group == 0) {
+        switch (n_paths) {
+            case 1: return launch_cfg<1, 256, 4, false>(a, X, ldx, s);
+            case 2: return launch_cfg<2, 256, 3, false>(a, X, ldx, s);
+            case 3: return launch_cfg<3, 128, 3, false>(a, X, ldx, s);
+            case 4: return launch_cfg<4, 128, 2, false>(a, X, ldx, s);
+        }
+    } else {
+        switch (n_paths) {
+            case 1: return launch_cfg<1, 256, 4, true>(a, X, ldx, s);
+            case 2: return launch_cfg<2, 256, 3, true>(a, X, ldx, s);
+            case 3: return launch_cfg<3, 256, 2, true>(a, X, ldx, s);
+            case 4: return launch_cfg<4, 256, 2, true>(a, X, ldx, s);
+        }
+    }
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t gemm_read_error(unsigned int* code) {
+    cudaError_t e = cudaMemcpyFromSymbol(code, g_gemm_error, sizeof(unsigned int));
+    if (e != cudaSuccess) return e;
+    if (*code) {
+        const unsigned int zero = 0;
+        e = cudaMemcpyToSymbol(g_gemm_error, &zero, sizeof(zero));
+    }
+    return e;
+}
+
+}  // namespace rb

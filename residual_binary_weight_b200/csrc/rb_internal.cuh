@@ -76,6 +76,13 @@ GvPlan gemv_plan_grouped(const GvJob* host_jobs, int n, int n_paths, int group, 
 cudaError_t launch_gemv(const GvArgs& a, const GvPlan& plan, cudaStream_t s);
 int gemv_max_jobs();
 
+// ---------------------------------------------------------------- rb_gemm
+bool gemm_supported(int n_paths, int group);
+cudaError_t launch_gemm(const uint32_t* planes, const void* alpha, bool alpha_f16, int64_t M, int64_t K, int n_paths,
+                        int group, bool sliced, const void* X, int64_t ldx, int T, void* Y, bool y_f16, int64_t ldy,
+                        cudaStream_t s);
+cudaError_t gemm_read_error(unsigned int* code);
+
 int device_sm_count();
 
 }  // namespace rb

@@ -1,0 +1,122 @@
+"""rb_gemm (tcgen05 prefill kernel) on the GPU against the fp64 oracle.
+
+As for the matvec, the oracle packs the weight and both sides evaluate the
+same planes and stored scales on the same X; outputs must be within
+1e-3 * sum_k sum_j |alpha_k x_j| per element.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import residual_binary_weight_b200 as rb
+import synth
+from gpu_util import planes_np, to_dev_planes
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(W, X, n_paths, group, alpha_f16, order="rows", y_dtype=torch.float16, ldx_pad=0, ldy_pad=0):
+    ref_p, ref_a, _ = oracle.pack(W, n_paths, group)
+    stored = oracle.alpha_to_f16(ref_a) if alpha_f16 else ref_a.astype(np.float32)
+    if group == 128 and not alpha_f16:
+        # with per-group scales the kernel multiplies by the fp16 rounding of fp32 scales
+        used = stored.astype(np.float16).astype(np.float64)
+    else:
+        used = stored.astype(np.float64)
+    y_ref, den = oracle.matvec(ref_p, used, X.astype(np.float64))
+    T, K = X.shape
+    M = W.shape[0]
+    xt = torch.zeros((T, K + ldx_pad), dtype=torch.float16)
+    xt[:, :K] = torch.from_numpy(X)
+    Xd = xt.cuda()[:, :K]
+    Yd = torch.full((T, M + ldy_pad), float("nan"), dtype=y_dtype, device="cuda")
+    rb.gemm(to_dev_planes(ref_p, order=order), torch.from_numpy(stored).cuda(), Xd, group=group, Y=Yd[:, :M])
+    torch.cuda.synchronize()
+    rb.load()
+    from residual_binary_weight_b200._lib import check
+    check(rb.load().rb_gemm_check(None))
+    Yh = Yd.float().cpu().numpy()
+    if ldy_pad:
+        assert np.all(np.isnan(Yh[:, M:])), "wrote past the row"
+    return oracle.compare_outputs(Yh[:, :M], y_ref, den)
+
+
+def _ok(res, what):
+    nbad, worst = res
+    assert nbad == 0, (what, worst)
+
+
+@pytest.mark.parametrize("order", ["rows", "sliced"])
+def test_small_two_paths(order):
+    rng = np.random.default_rng(1)
+    W = (rng.standard_normal((256, 512)) * 0.02).astype(np.float16)
+    X = rng.standard_normal((300, 512)).astype(np.float16)          # one full and one partial token tile
+    _ok(_run(W, X, 2, 0, False, order), order)
+
+
+@pytest.mark.parametrize("M,K,T", [(1, 128, 1), (130, 128, 7), (200, 384, 257), (129, 640, 64)])
+def test_ragged_shapes(M, K, T):
+    rng = np.random.default_rng(M + K + T)
+    W = (rng.standard_normal((M, K)) * 0.02).astype(np.float32)
+    X = rng.standard_normal((T, K)).astype(np.float16)
+    _ok(_run(W, X, 2, 0, False), (M, K, T))
+    _ok(_run(W, X, 2, 0, False, "sliced"), (M, K, T, "sliced"))
+
+
+@pytest.mark.parametrize("n_paths", [1, 2, 3, 4])
+@pytest.mark.parametrize("group,alpha_f16", [(0, False), (0, True), (128, True), (128, False)])
+def test_paths_and_scales(n_paths, group, alpha_f16):
+    rng = np.random.default_rng(10 * n_paths + group)
+    W = (rng.standard_t(4, (260, 1024)) * 0.014).astype(np.float16)
+    X = rng.standard_normal((130, 1024)).astype(np.float16)
+    _ok(_run(W, X, n_paths, group, alpha_f16), (n_paths, group, alpha_f16))
+
+
+def test_dtypes_and_pitches():
+    rng = np.random.default_rng(5)
+    W = (rng.standard_normal((160, 768)) * 0.02).astype(np.float16)
+    X = rng.standard_normal((96, 768)).astype(np.float16)
+    _ok(_run(W, X, 2, 0, False, y_dtype=torch.float32, ldx_pad=8, ldy_pad=3), "f32 out, pitches")
+    _ok(_run(W, X, 4, 128, True, "sliced", ldx_pad=16, ldy_pad=1), "g128 pitches")
+
+
+def test_qbb_batch16():
+    wl = synth.WORKLOADS["qbb_g128"]
+    W = synth.host_rows(wl, 0, "down", range(256))
+    X = synth.host_activations(wl, 0, "down", 16)
+    _ok(_run(W, X, 4, 128, True, "sliced"), "qbb down T=16")
+
+
+@pytest.mark.parametrize("matrix", ["up", "down"])
+def test_prefill_full_size_sampled(matrix):
+    """The 2048-token prefill block through a full 14336-wide projection.
+    The weight is drawn on the device and packed by the GPU; 64 sampled rows
+    are replaced by the oracle's planes and scales, and their outputs for 48
+    sampled tokens are checked against the oracle."""
+    wl = synth.WORKLOADS["prefill"]
+    spec = {m.name: m for m in wl.matrices}[matrix]
+    W = synth.device_weight(wl, 0, matrix, "cuda")
+    planes, alpha, _ = rb.pack(W, 2, 0, order="sliced")
+    rng = np.random.default_rng(9)
+    rows = np.sort(rng.choice(spec.M, 64, replace=False))
+    idx = torch.from_numpy(rows).cuda()
+    Wr = W.index_select(0, idx).cpu().numpy()
+    del W
+    ref_p, ref_a, rabs = oracle.pack(Wr, 2, 0, want_rabs=True)
+    rep = oracle.compare_planes(planes_np(planes[:, :, idx], spec.K), ref_p, rabs, ref_a)
+    assert rep.bad == 0, rep
+    planes[:, :, idx] = to_dev_planes(ref_p, order="sliced")
+    a32 = ref_a.astype(np.float32)
+    alpha[:, idx] = torch.from_numpy(a32).cuda()
+    X = synth.device_activations(wl, 0, matrix, 2048, "cuda")
+    Y = rb.gemm(planes, alpha, X)
+    torch.cuda.synchronize()
+    from residual_binary_weight_b200._lib import check
+    check(rb.load().rb_gemm_check(None))
+    toks = np.sort(rng.choice(2048, 48, replace=False))
+    Xs = X[torch.from_numpy(toks).cuda()].cpu().numpy().astype(np.float64)
+    y_ref, den = oracle.matvec(ref_p, a32.astype(np.float64), Xs)
+    got = Y[torch.from_numpy(toks).cuda()][:, idx].float().cpu().numpy()
+    nbad, worst = oracle.compare_outputs(got, y_ref, den)
+    assert nbad == 0, worst
