@@ -176,7 +176,7 @@ def time_gemm(torch, rb, synth, device, peak_tf):
     for name in ("up", "down"):
         sp = {m.name: m for m in wl.matrices}[name]
         W = synth.device_weight(wl, 0, name, device)
-        planes, alpha, _ = rb.pack(W, 2, 0)
+        planes, alpha, _ = rb.pack(W, 2, 0, order="sliced")
         del W
         X = synth.device_activations(wl, 0, name, 2048, device)
         Y = torch.empty((2048, sp.M), dtype=torch.float16, device=device)
@@ -274,7 +274,7 @@ def run_gpu(args):
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
     hbm_peak, bf16_peak, _, peak_kind = _peaks()
 
-    items, xbuf, ybuf, alg_bytes = build_stack(torch, rb, synth, device)
+    items, xbuf, ybuf, alg_bytes = build_stack(torch, rb, synth, device, layers=args.layers)
     g = rb.GroupedGemv(items, n_paths=2, group=0, T=1)
     stream = torch.cuda.current_stream(device)
 
@@ -339,7 +339,7 @@ def run_gpu(args):
            "h2d_bytes_per_step": xbuf.numel() * 2, "d2h_bytes_per_step": ybuf.numel() * 2}
 
     parts = {}
-    if rank == 0:
+    if rank == 0 and not args.no_parts:
         parts["rb_pack"] = time_pack(torch, rb, synth, device)
         gm = time_gemm(torch, rb, synth, device, bf16_peak)
         if gm is not None:
@@ -360,8 +360,9 @@ def run_gpu(args):
         "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded device draws: per-row sigma log-uniform [0.005, 0.05], 0.1% entries x10; "
                 "x N(0,1) with 0.5% channels x20)",
-        "config": {"workload": "Llama-2-7B-shaped decode linears, batch 1: 32 layers x (4 x 4096x4096, "
-                               "2 x 11008x4096, 1 x 4096x11008), 2 paths, fp32 per-row scales, fp16 x/y",
+        "config": {"workload": f"Llama-2-7B-shaped decode linears, batch 1: {args.layers} layers x (4 x 4096x4096, "
+                               "2 x 11008x4096, 1 x 4096x11008), 2 paths, fp32 per-row scales, fp16 x/y, "
+                               "sliced plane order",
                    "bytes_per_step": alg_bytes, "l2": "inputs larger than L2 (1.6 GB streamed per step)",
                    "parallelism": f"replicas x{ws}"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
@@ -386,6 +387,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline leg")
+    ap.add_argument("--layers", type=int, default=32,
+                    help="decoder layers in the stack (32 for the benchmark; fewer for profiling captures)")
+    ap.add_argument("--no-parts", action="store_true", help="skip the rb_pack / rb_gemm sub-measurements")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)

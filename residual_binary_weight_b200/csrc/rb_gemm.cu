@@ -153,6 +153,37 @@ __device__ __forceinline__ void expand_word(uint32_t w, uint32_t val2, uint32_t 
     }
 }
 
+// 32 lanes x CW columns of fp32 from tensor memory (this warp's lane quarter)
+template <int CW>
+__device__ __forceinline__ void tmem_load(uint32_t taddr, uint32_t (&v)[CW]);
+
+template <>
+__device__ __forceinline__ void tmem_load<32>(uint32_t taddr, uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+          "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]),
+          "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]),
+          "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+template <>
+__device__ __forceinline__ void tmem_load<16>(uint32_t taddr, uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+          "=r"(v[14]), "=r"(v[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
 struct GemmArgs {
     const uint32_t* planes;
     const void* alpha;
@@ -326,31 +357,22 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, GemmArgs a) {
             }
             const uint32_t lane_addr = static_cast<uint32_t>((warp - EXP_WARP0) * 32) << 16;
             const int t_base = tok_tile * BN;
-            for (int c0 = 0; c0 < BN; c0 += 32) {
-                float yv[32];
+            constexpr int CW = BN < 32 ? BN : 32;          // columns per tensor-memory load
+            for (int c0 = 0; c0 < BN; c0 += CW) {
+                float yv[CW];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) yv[i] = 0.0f;
+                for (int i = 0; i < CW; ++i) yv[i] = 0.0f;
 #pragma unroll
                 for (int p = 0; p < C::NACC; ++p) {
-                    uint32_t v[32];
+                    uint32_t v[CW];
                     const uint32_t taddr = tmem_base + lane_addr + static_cast<uint32_t>(p * BN + c0);
-                    asm volatile(
-                        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-                        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-                        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-                        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
-                          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
-                          "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]),
-                          "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]),
-                          "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-                        : "r"(taddr));
-                    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+                    tmem_load<CW>(taddr, v);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) yv[i] = fmaf(al[p], __uint_as_float(v[i]), yv[i]);
+                    for (int i = 0; i < CW; ++i) yv[i] = fmaf(al[p], __uint_as_float(v[i]), yv[i]);
                 }
                 if (row < M) {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
+                    for (int i = 0; i < CW; ++i) {
                         const int t = t_base + c0 + i;
                         if (t < a.T) {
                             if (a.y_f16) static_cast<__half*>(a.y)[t * a.ldy + row] = __float2half_rn(yv[i]);
@@ -417,23 +439,44 @@ cudaError_t launch_cfg(const GemmArgs& a, const void* X, int64_t ldx, cudaStream
 
 bool gemm_supported(int n_paths, int group) { return n_paths >= 1 && n_paths <= 4 && (group == 0 || group == 128); }
 
+// stages that fit in shared memory for a configuration (at most 8)
+constexpr int stages_for(int np, int bn) {
+    return ((210 * 1024) / static_cast<int>(np * A_TILE_BYTES + bn * BK * 2)) < 8
+               ? ((210 * 1024) / static_cast<int>(np * A_TILE_BYTES + bn * BK * 2))
+               : 8;
+}
+
+template <int NP, bool G128>
+cudaError_t launch_np(const GemmArgs& a, const void* X, int64_t ldx, cudaStream_t s) {
+    // token tile: the narrowest of 16..256 that covers T (MMA N), so small
+    // batches do not pay for unused columns; NP accumulators must fit in
+    // 512 tensor-memory columns
+    constexpr int BN_MAX = G128 ? 256 : (NP <= 2 ? 256 : 128);
+    const int T = a.T;
+    if (T <= 16) return launch_cfg<NP, 16, stages_for(NP, 16), G128>(a, X, ldx, s);
+    if (T <= 32) return launch_cfg<NP, 32, stages_for(NP, 32), G128>(a, X, ldx, s);
+    if (T <= 64) return launch_cfg<NP, 64, stages_for(NP, 64), G128>(a, X, ldx, s);
+    if (T <= 128 || BN_MAX == 128) return launch_cfg<NP, 128, stages_for(NP, 128), G128>(a, X, ldx, s);
+    return launch_cfg<NP, BN_MAX, stages_for(NP, BN_MAX), G128>(a, X, ldx, s);
+}
+
 cudaError_t launch_gemm(const uint32_t* planes, const void* alpha, bool alpha_f16, int64_t M, int64_t K, int n_paths,
                         int group, bool sliced, const void* X, int64_t ldx, int T, void* Y, bool y_f16, int64_t ldy,
                         cudaStream_t s) {
     GemmArgs a{planes, alpha, Y, M, K, ldy, T, n_paths, group == 128, sliced, alpha_f16, y_f16};
     if (group == 0) {
         switch (n_paths) {
-            case 1: return launch_cfg<1, 256, 4, false>(a, X, ldx, s);
-            case 2: return launch_cfg<2, 256, 3, false>(a, X, ldx, s);
-            case 3: return launch_cfg<3, 128, 3, false>(a, X, ldx, s);
-            case 4: return launch_cfg<4, 128, 2, false>(a, X, ldx, s);
+            case 1: return launch_np<1, false>(a, X, ldx, s);
+            case 2: return launch_np<2, false>(a, X, ldx, s);
+            case 3: return launch_np<3, false>(a, X, ldx, s);
+            case 4: return launch_np<4, false>(a, X, ldx, s);
         }
     } else {
         switch (n_paths) {
-            case 1: return launch_cfg<1, 256, 4, true>(a, X, ldx, s);
-            case 2: return launch_cfg<2, 256, 3, true>(a, X, ldx, s);
-            case 3: return launch_cfg<3, 256, 2, true>(a, X, ldx, s);
-            case 4: return launch_cfg<4, 256, 2, true>(a, X, ldx, s);
+            case 1: return launch_np<1, true>(a, X, ldx, s);
+            case 2: return launch_np<2, true>(a, X, ldx, s);
+            case 3: return launch_np<3, true>(a, X, ldx, s);
+            case 4: return launch_np<4, true>(a, X, ldx, s);
         }
     }
     return cudaErrorInvalidValue;
