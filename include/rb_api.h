@@ -208,12 +208,12 @@ RB_API rb_status rb_gemm_check(void* stream);
  * framework that owns every device buffer, or a fixed-budget deployment that
  * forbids allocations after start-up. For them the scratch rb_gemv keeps in
  * the workspace (work counters and K-split partial sums) lives in one static
- * 2 MiB device array per GPU, held by every GPU that loads the library until
+ * 1 MiB device array per GPU, held by every GPU that loads the library until
  * the process exits. The caller still passes planes, scales, x and y, with
  * the same meaning, layout and checks as rb_gemv.
  *
- * - Shapes whose scratch would exceed 2 MiB (rb_gemv_workspace_bytes(L, T) >
- *   2 MiB) are refused with RB_ERR_UNSUPPORTED before any CUDA call.
+ * - Shapes whose scratch would exceed 1 MiB (rb_gemv_workspace_bytes(L, T) >
+ *   1 MiB) are refused with RB_ERR_UNSUPPORTED before any CUDA call.
  * - The first call on a device looks up the array's device address
  *   (cudaGetSymbolAddress) with that device current; make that first call
  *   before any stream capture.

@@ -61,7 +61,7 @@ struct GvArgs {
 // arrival counter per (job, row block, token) of every K-split job, then the
 // fp32 partial sums of the split jobs.
 constexpr size_t GV_HEADER_BYTES = 256;
-enum : uint32_t { GV_ERR_SMEM_LAYOUT = 1u, GV_ERR_BAD_JOB = 2u, GV_ERR_TOO_MANY_JOBS = 4u };
+enum : uint32_t { GV_ERR_SMEM_LAYOUT = 1u, GV_ERR_BAD_JOB = 2u, GV_ERR_TOO_MANY_JOBS = 4u, GV_ERR_WAIT = 8u };
 
 struct GvPlan {
     int rows_per_cta;       // R

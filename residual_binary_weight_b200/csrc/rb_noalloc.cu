@@ -15,7 +15,7 @@ void set_error_message(const char* msg);
 namespace {
 
 // Every GPU that loads the library holds this array until the process exits.
-constexpr size_t kNoallocScratchBytes = size_t(2) << 20;   // 2 MiB
+constexpr size_t kNoallocScratchBytes = size_t(1) << 20;   // 1 MiB
 __device__ __align__(256) unsigned char rb_noalloc_scratch[kNoallocScratchBytes];
 
 constexpr int kMaxDevices = 64;

@@ -56,12 +56,23 @@ def test_noalloc_matches_workspace_entry_point():
         assert nbad == 0, (call, worst)
 
 
+def _shape_beyond_scratch(lib):
+    """A layout whose K-split scratch is larger than the static 1 MiB array."""
+    for n_paths in (1, 2, 4):
+        for M in (1024, 2048, 3072, 4096, 6144, 8192, 12288, 16384):
+            for T in (64, 32, 16):
+                L = rb.layout(M, 8192, n_paths, 0, "sliced")
+                if lib.rb_gemv_workspace_bytes(L, T) > (1 << 20):
+                    return L, M, T
+    return None
+
+
 def test_noalloc_refuses_shapes_beyond_its_scratch():
     lib = _lib.load()
-    # one path, 64 tokens, 4096 rows: the K split needs just over 2 MiB
-    L = rb.layout(4096, 8192, 1, 0, "sliced")
-    assert lib.rb_gemv_workspace_bytes(L, 64) > (2 << 20)
+    found = _shape_beyond_scratch(lib)
+    assert found is not None
+    L, M, T = found
     p = ctypes.c_void_p(1 << 40)
-    rc = lib.rb_gemv_noalloc(p, p, _lib.RB_F32, L, p, 8192, 64, p, _lib.RB_F16, 4096, None)
+    rc = lib.rb_gemv_noalloc(p, p, _lib.RB_F32, L, p, 8192, T, p, _lib.RB_F16, M, None)
     assert _lib.STATUS_NAMES[rc] == "RB_ERR_UNSUPPORTED"
     assert b"static array" in lib.rb_last_error()
