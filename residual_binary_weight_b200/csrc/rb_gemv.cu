@@ -17,15 +17,16 @@
 // the lane's base register and byte 1 from the plane word.
 //
 // Work split. A CTA (32 warps) owns R rows of one matrix for a K chunk and
-// walks its 512-column slices. A warp holds 2J (row, path) items; an
-// item-slice is 16 consecutive plane words, one per lane of a half-warp, so a
-// warp-wide 32-bit load covers two items: rows 2r and 2r + 1 of one path,
-// which are adjacent in memory in the sliced plane layout (so one load
-// instruction reads 128 contiguous bytes and the items of one path sit at
-// immediate offsets from one pointer). Lane l reads byte (q + (l >> 3)) & 3
-// of its word at step q, which puts the 32 lanes of every LDS on 32
-// distinct banks. Partial sums stay in registers across the slices of the
-// chunk and are reduced over the 16 lanes of each item at the end.
+// walks its 512-column slices. An item (row, path) of a slice is 16 plane
+// words; 8 lanes hold one item, two consecutive words per lane, so one
+// warp-wide 64-bit load covers 4 items: 4 consecutive rows of one path, which
+// in the sliced plane layout are 256 contiguous bytes (and the items of one
+// path sit at immediate offsets from one pointer). Each lane issues J such
+// loads per slice. Lanes whose words would share banks process their two
+// words in opposite order and rotate the byte order, which puts the 32 lanes
+// of every LDS on 32 distinct banks. Partial sums stay in registers across
+// the slices of the chunk and are reduced over the 8 lanes of each item at
+// the end.
 //
 // Per-row scales are applied once per row at the end; per-128-column scales
 // (the QBB layout) multiply each word's partial sum as it is accumulated.
@@ -86,6 +87,19 @@ __device__ __forceinline__ const char* mad_ptr(uint32_t a, uint32_t b, const voi
     return reinterpret_cast<const char*>(r);
 }
 
+// m ? b : a, bitwise (m is all ones or all zeros): one LOP3
+__device__ __forceinline__ uint32_t sel_mask(uint32_t a, uint32_t b, uint32_t m) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xD8;" : "=r"(d) : "r"(a), "r"(b), "r"(m));
+    return d;
+}
+
+__device__ __forceinline__ uint2 ldg_words2(const void* p) {
+    uint2 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+    return v;
+}
+
 __device__ __forceinline__ uint32_t ldg_word(const void* p) {
     uint32_t v;
     asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
@@ -98,12 +112,14 @@ struct BoolC { static constexpr bool value = B; };
 template <int J>
 struct Log2 { static constexpr int v = J == 16 ? 4 : J == 8 ? 3 : J == 4 ? 2 : J == 2 ? 1 : 0; };
 
+// A warp-wide 64-bit load reads 4 items (consecutive rows of one path, 8
+// lanes per item, 2 words per lane); J such loads per lane and slice.
 template <int NP, bool G128>
 struct Cfg {
-    static constexpr int J = G128 ? 8 : 16;           // item pairs per warp
-    static constexpr int HR = (2 * J / NP) / 2;       // row pairs per path per warp
-    static constexpr int RW = 2 * HR;                 // rows per warp
-    static constexpr int JV = NP * HR;                // item pairs in use (<= J)
+    static constexpr int J = G128 && NP <= 4 ? 4 : 8;  // item loads per lane per slice (>= NP)
+    static constexpr int HR = J / NP > 0 ? J / NP : 1; // row quads per path per warp
+    static constexpr int RW = 4 * HR;                 // rows per warp
+    static constexpr int JV = NP * HR <= J ? NP * HR : J;   // loads in use
     static constexpr int R = WARPS * RW;              // rows per CTA
 };
 
@@ -160,16 +176,17 @@ __device__ __forceinline__ void build_table(const uint4* xs, uint32_t tbl) {
     for (int lo = 0; lo < 16; ++lo) sts(a0 + (lo << 8), q01[lo & 3] + p23[lo >> 2]);
 }
 
-// Reduce acc[0..J) over the 16 lanes of a half-warp; afterwards lane wd holds
-// the sum of item pair j = wd >> (4 - log2 J) in acc[0].
+// Reduce acc[0..J) over the 8 lanes of an item group (lane bits 0-2); J is
+// a power of two <= 8. Afterwards lane t of the group holds the sum of item
+// load j = t >> (3 - log2 J) in acc[0].
 template <int J>
-__device__ __forceinline__ void halfwarp_transpose_reduce(float (&acc)[J], int wd) {
+__device__ __forceinline__ void group8_transpose_reduce(float (&acc)[J], int t) {
     int cnt = J;
 #pragma unroll
-    for (int off = 8; off >= 1; off >>= 1) {
+    for (int off = 4; off >= 1; off >>= 1) {
         if (cnt > 1) {
             const int half = cnt >> 1;
-            const bool up = (wd & off) != 0;
+            const bool up = (t & off) != 0;
 #pragma unroll
             for (int i = 0; i < J / 2; ++i) {
                 if (i < half) {
@@ -289,7 +306,8 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_lut_kernel(GvArgs p, uint32_t
         return;
     }
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int h = lane >> 4, wd = lane & 15;
+    // lane -> item q4 of each 4-item load, word pair t (words 2t, 2t + 1)
+    const int q4 = lane >> 3, t8 = lane & 7;
     const int T = p.T;
     const int n_jobs = p.jobs ? p.n_jobs : 1;
     if (n_jobs > MAX_JOBS) {
@@ -299,10 +317,16 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_lut_kernel(GvArgs p, uint32_t
     scan_jobs<C::R>(p, lo, n_jobs);
     const uint32_t total_units = lo.unit_prefix[n_jobs];
 
-    const int rot = (lane >> 3) & 3;
+    // The 8 lanes sharing t8 & 3 (t8 in {a, a + 4}, 4 items) would hit the
+    // same banks; lane z = (t8 >> 2) + 2 q4 swaps its two words when z is odd
+    // (rv) and rotates the byte order by rq = z >> 1, so every LDS touches 32
+    // distinct banks.
+    const uint32_t zr = static_cast<uint32_t>((t8 >> 2) + 2 * q4);
+    const uint32_t rv = zr & 1u, rq = zr >> 1;
+    const uint32_t swap_mask = 0u - rv;
     uint32_t sel[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) sel[q] = 0x7604u | (static_cast<uint32_t>((q + rot) & 3) << 4);
+    for (int q = 0; q < 4; ++q) sel[q] = 0x7604u | (((static_cast<uint32_t>(q) + rq) & 3u) << 4);
 
     uint32_t iter = 0;
     while (true) {
@@ -335,67 +359,75 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_lut_kernel(GvArgs p, uint32_t
         const bool full = row0 + C::RW <= uM;
 
         float acc[J];
-        uint32_t wv[J];
+        uint2 wv[J];
         float av[J];
 #pragma unroll
         for (int j = 0; j < J; ++j) {
             acc[j] = 0.0f;
             av[j] = 0.0f;
         }
-        uint32_t cur_base[4];
+        // table address base of step (word v, byte q): column 8 t8 + 4 (v ^ rv) + (q + rq) & 3
+        uint32_t cur_base[8];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) cur_base[q] = TBL0 + 4u * (4u * wd + static_cast<uint32_t>((q + rot) & 3));
+        for (int v = 0; v < 2; ++v)
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                cur_base[4 * v + q] = TBL0 + 4u * (8u * t8 + 4u * (static_cast<uint32_t>(v) ^ rv) +
+                                                   ((static_cast<uint32_t>(q) + rq) & 3u));
 
-        // word of lane wd in slice s, clamped in a partial last slice (the
-        // table entries past K are 0, so a clamped word adds nothing); the
-        // sliced layout pads the last slice, so only the scale index needs it
-        auto lane_word = [&](int s) -> uint32_t {
+        // word pair of lane t8 in slice s, clamped in a partial last slice
+        // (the table entries past K are 0, so a clamped pair adds nothing);
+        // the sliced layout pads the last slice, so only the scale index and
+        // the row layout need it
+        auto lane_pair = [&](int s) -> uint32_t {
             const int ws = min(16, static_cast<int>((K - static_cast<int64_t>(s) * SLICE_COLS) >> 5));
-            return wd < ws ? static_cast<uint32_t>(wd) : 0u;
+            return 2 * t8 < ws ? static_cast<uint32_t>(t8) : 0u;
         };
         auto alpha_at = [&](size_t ai) -> float {
             return A16 ? __half2float(static_cast<const __half*>(jb.alpha)[ai]) : static_cast<const float*>(jb.alpha)[ai];
         };
-        // Item pair j (of this half-warp): path j / HR, row 2 (j % HR) + h.
-        // Word address = lane pointer of the path + (j % HR) * row-pair
-        // stride, an immediate offset in the sliced layout. The per-slice row
-        // goes through an empty asm so the compiler cannot hoist per-item values.
+        // Item load j: path j / HR, rows row0 + 4 (j % HR) + q4. Its lane
+        // pointer = path pointer + (j % HR) * (4 rows): an immediate offset in
+        // the sliced layout. The per-slice row goes through an empty asm so
+        // the compiler cannot hoist per-item values.
         struct SliceAddr {
-            const char* slice0;   // (path 0, row 0, word wsel) of the slice
-            const char* lane0;    // (path 0, row r0 + h, word wsel): full warps
-            uint32_t r0, lw;
+            const char* slice0;   // (path 0, row 0, pair tsel) of the slice
+            const char* lane0;    // (path 0, row r0 + q4, pair tsel): full warps
+            uint32_t r0, tp;
         };
+        const uint32_t row_bytes = SLICED ? 64u : uW32 * 4u;
         auto slice_addr = [&](int s) {
             SliceAddr a;
-            a.lw = lane_word(s);
+            a.tp = lane_pair(s);
             a.r0 = row0;
             asm volatile("" : "+r"(a.r0));
-            const uint32_t wsel = SLICED ? static_cast<uint32_t>(wd) : a.lw;
-            const uint32_t row_bytes = SLICED ? 64u : uW32 * 4u;
+            const uint32_t tsel = SLICED ? static_cast<uint32_t>(t8) : a.tp;
             a.slice0 = reinterpret_cast<const char*>(jb.planes) +
-                       (SLICED ? (static_cast<size_t>(s) * uM * 16u + wsel) * 4u
-                               : (16u * static_cast<uint32_t>(s) + wsel) * 4u);
-            a.lane0 = mad_ptr(a.r0 + h, row_bytes, a.slice0);
+                       (SLICED ? (static_cast<size_t>(s) * uM * 16u + 2u * tsel) * 4u
+                               : (16u * static_cast<uint32_t>(s) + 2u * tsel) * 4u);
+            a.lane0 = mad_ptr(a.r0 + q4, row_bytes, a.slice0);
             return a;
         };
-        // load item pair j of the slice at `a`
+        // load item j of the slice at `a` (words swapped on lanes with rv)
         auto fetch = [&](int j, int s, const SliceAddr& a, auto full_tag) {
             constexpr bool F = decltype(full_tag)::value;
-            const uint32_t row_bytes = SLICED ? 64u : uW32 * 4u;
-            const uint32_t path = j / HR, rp = j % HR;
+            const uint32_t path = j / HR, rr = j % HR;
             uint32_t row;
             const char* wp;
             if (F) {
-                row = a.r0 + h + 2u * rp;
+                row = a.r0 + q4 + 4u * rr;
                 const char* pb = path ? mad_ptr(path, path_bytes, a.lane0) : a.lane0;
-                wp = SLICED ? pb + rp * 128u : mad_ptr(2u * rp, row_bytes, pb);
+                wp = SLICED ? pb + rr * 256u : mad_ptr(4u * rr, row_bytes, pb);
             } else {
                 // rows past M are clamped to the last row (absolute address)
-                row = min(a.r0 + h + 2u * rp, uM - 1u);
+                row = min(a.r0 + q4 + 4u * rr, uM - 1u);
                 wp = mad_ptr(row, row_bytes, path ? mad_ptr(path, path_bytes, a.slice0) : a.slice0);
             }
-            wv[j] = ldg_word(wp);
-            if (G128) av[j] = alpha_at(static_cast<size_t>(path * uM + row) * gpr + 4u * s + (a.lw >> 2));
+            // K is a multiple of 128, so rows of either layout are a multiple
+            // of 16 bytes, the planes are 16-byte aligned and a slice holds an
+            // even number of words: the pair is one aligned 8-byte load
+            wv[j] = ldg_words2(wp);
+            if (G128) av[j] = alpha_at(static_cast<size_t>(path * uM + row) * gpr + 4u * s + (a.tp >> 1));
         };
         auto fetch_slice = [&](int s, auto full_tag) {
             const SliceAddr a = slice_addr(s);
@@ -413,12 +445,20 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_lut_kernel(GvArgs p, uint32_t
 #pragma unroll
             for (int j = 0; j < J; ++j) {
                 if (j >= C::JV) continue;
-                const uint32_t w = wv[j];
-                const float v0 = lds(prmt(w, cur_base[0], sel[0]));
-                const float v1 = lds(prmt(w, cur_base[1], sel[1]));
-                const float v2 = lds(prmt(w, cur_base[2], sel[2]));
-                const float v3 = lds(prmt(w, cur_base[3], sel[3]));
-                const float ps = (v0 + v1) + (v2 + v3);
+                // the word swap of lanes with rv happens here, where the words
+                // are used, not where they are loaded (a use right after the
+                // load would wait for it)
+                const uint32_t w0 = sel_mask(wv[j].x, wv[j].y, swap_mask);
+                const uint32_t w1 = sel_mask(wv[j].y, wv[j].x, swap_mask);
+                const float v0 = lds(prmt(w0, cur_base[0], sel[0]));
+                const float v1 = lds(prmt(w0, cur_base[1], sel[1]));
+                const float v2 = lds(prmt(w0, cur_base[2], sel[2]));
+                const float v3 = lds(prmt(w0, cur_base[3], sel[3]));
+                const float v4 = lds(prmt(w1, cur_base[4], sel[0]));
+                const float v5 = lds(prmt(w1, cur_base[5], sel[1]));
+                const float v6 = lds(prmt(w1, cur_base[6], sel[2]));
+                const float v7 = lds(prmt(w1, cur_base[7], sel[3]));
+                const float ps = ((v0 + v1) + (v2 + v3)) + ((v4 + v5) + (v6 + v7));
                 if (G128) acc[j] = fmaf(av[j], ps, acc[j]);
                 else acc[j] += ps;
                 if (PF) fetch(j, s + 1, an, full_tag);
@@ -445,7 +485,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_lut_kernel(GvArgs p, uint32_t
                 if (s + 2 < s_end) stage_x(xt, K, s + 2, lo.xstage[par]);
                 consume(s, full_tag, BoolC<true>{});
 #pragma unroll
-                for (int q = 0; q < 4; ++q) cur_base[q] ^= TBL_TOGGLE;
+                for (int q = 0; q < 8; ++q) cur_base[q] ^= TBL_TOGGLE;
                 stage_wait_all();
                 cta_sync_any();
             }
@@ -460,21 +500,21 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_lut_kernel(GvArgs p, uint32_t
         asm volatile("" : "+r"(u));
         const UnitInfo ue = decode_unit(p, lo, n_jobs, u);
 
-        // ---- reduce over the half-warp; lane wd owns item pair j = wd >> shift
-        halfwarp_transpose_reduce<J>(acc, wd);
-        constexpr int shift = 4 - Log2<J>::v;
-        if ((wd & ((1 << shift) - 1)) == 0) lo.tot[warp][2 * (wd >> shift) + h] = acc[0];
+        // ---- reduce over the 8 lanes of each item; lane t8 owns load j = t8 >> shift
+        group8_transpose_reduce<J>(acc, t8);
+        constexpr int shift = 3 - Log2<J>::v;
+        if ((t8 & ((1 << shift) - 1)) == 0) lo.tot[warp][4 * (t8 >> shift) + q4] = acc[0];
         __syncwarp();
 
         // ---- per-row output of this chunk: lane r < RW owns row r of the warp,
-        // whose path-k item is pair k * HR + r / 2 of half-warp r % 2
+        // whose path-k item is load k * HR + r / 4 of item group r % 4
         float yv = 0.0f;
         const int64_t my_row = static_cast<int64_t>(ue.rb) * C::R + warp * C::RW + lane;
         const bool row_ok = lane < C::RW && my_row < ue.jb.M;
         if (row_ok) {
 #pragma unroll
             for (int k = 0; k < NP; ++k) {
-                const float tk = lo.tot[warp][2 * (k * HR + (lane >> 1)) + (lane & 1)];
+                const float tk = lo.tot[warp][4 * (k * HR + (lane >> 2)) + (lane & 3)];
                 if (G128) {
                     yv += tk;
                 } else {
@@ -560,8 +600,9 @@ cudaError_t launch_order(const GvArgs& a, const GvPlan& plan, cudaStream_t s) {
 int gemv_max_jobs() { return MAX_JOBS; }
 
 int gemv_rows_per_cta(int n_paths, int group) {
-    const int J = group ? 8 : 16;
-    return WARPS * 2 * ((2 * J / n_paths) / 2);
+    const int J = group && n_paths <= 4 ? 4 : 8;
+    const int hr = J / n_paths > 0 ? J / n_paths : 1;
+    return WARPS * 4 * hr;
 }
 
 static void count_job(int64_t M, int64_t K, int R, int chunk, int T, GvPlan& pl) {
