@@ -175,7 +175,6 @@ rb_status rb_gemv(const uint32_t* planes, const void* alpha, rb_dtype alpha_dtyp
     a.ldx = ldx;
     a.ldy = ldy;
     a.chunk_slices = pl.chunk_slices;
-    a.dynamic = false;
     a.workspace = workspace;
     a.ws_bytes = ws_bytes;
     e = launch_gemv(a, pl, s);
@@ -243,7 +242,6 @@ rb_status rb_gemv_grouped(const rb_gemv_desc* descs_host, const rb_gemv_desc* de
     a.ldx = 0;
     a.ldy = 0;
     a.chunk_slices = pl.chunk_slices;
-    a.dynamic = true;
     a.workspace = workspace;
     a.ws_bytes = ws_bytes;
     e = launch_gemv(a, pl, s);

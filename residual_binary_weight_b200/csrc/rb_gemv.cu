@@ -45,7 +45,22 @@ constexpr uint32_t TBL_TOGGLE = 0x30000u;   // 0x10000 <-> 0x20000
 constexpr int SMEM_BYTES = 0x30000;          // covers both tables whatever the window base
 constexpr int MAX_JOBS = 2 * THREADS - 1;    // each thread scans two descriptors
 
-// Low shared region (below 0x10000): totals, job prefix sums, staged x.
+// One work unit of a CTA, decoded once into shared memory: (job, row block,
+// K chunk, token), with the token fastest, so CTAs that run together share
+// plane rows in L2.
+struct __align__(16) UnitRec {
+    const uint32_t* planes;
+    const void* alpha;
+    const __half* x;        // the unit's token row of x
+    void* y;                // the unit's token row of y
+    int64_t M, K;
+    uint32_t rb, j, t, ch, nch, s_begin, s_end, pad;
+};
+
+constexpr int UCAP = 128;   // unit records held at a time (a ring)
+
+// Low shared region (below 0x10000): totals, job prefix sums, unit records,
+// staged x.
 struct __align__(16) LowSmem {
     float tot[WARPS][32];
     uint32_t unit_prefix[MAX_JOBS + 1];
@@ -53,7 +68,7 @@ struct __align__(16) LowSmem {
     uint32_t part_prefix[MAX_JOBS + 1];
     uint32_t wsum[3][WARPS];
     uint4 xstage[2][64];      // x of the next slices, staged by cp.async
-    uint32_t bcast;
+    UnitRec units[UCAP];      // this CTA's units k at k % UCAP
     uint32_t last;
 };
 
@@ -87,10 +102,27 @@ __device__ __forceinline__ const char* mad_ptr(uint32_t a, uint32_t b, const voi
     return reinterpret_cast<const char*>(r);
 }
 
-// m ? b : a, bitwise (m is all ones or all zeros): one LOP3
-__device__ __forceinline__ uint32_t sel_mask(uint32_t a, uint32_t b, uint32_t m) {
-    uint32_t d;
-    asm("lop3.b32 %0, %1, %2, %3, 0xD8;" : "=r"(d) : "r"(a), "r"(b), "r"(m));
+// Packed fp32 pairs (sm_100 add/fma .f32x2): one instruction adds two
+// independent sums.
+__device__ __forceinline__ uint64_t pack_f2(float lo, float hi) {
+    uint64_t d;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+    return d;
+}
+
+__device__ __forceinline__ void unpack_f2(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+__device__ __forceinline__ uint64_t add_f2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+__device__ __forceinline__ uint64_t fma_f2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
     return d;
 }
 
@@ -202,35 +234,36 @@ __device__ __forceinline__ void group8_transpose_reduce(float (&acc)[J], int t) 
     }
 }
 
-struct UnitInfo {
-    GvJob jb;
-    int j, t, ch, rb, nch, s_begin, s_end;
-    int64_t ldx, ldy;
-};
-
-// Unit u -> job (binary search of the prefix), then (row block, chunk, token)
-// with the token fastest, so CTAs that run together share plane rows in L2.
-__device__ __forceinline__ UnitInfo decode_unit(const GvArgs& p, const LowSmem& lo, int n_jobs, uint32_t u) {
-    UnitInfo ui;
+__device__ __forceinline__ void decode_rec(const GvArgs& p, const uint32_t* unit_prefix, int n_jobs, uint32_t u,
+                                           UnitRec& r) {
     int jlo = 0, jhi = n_jobs - 1;
     while (jlo < jhi) {
         const int mid = (jlo + jhi + 1) >> 1;
-        if (lo.unit_prefix[mid] <= u) jlo = mid; else jhi = mid - 1;
+        if (unit_prefix[mid] <= u) jlo = mid; else jhi = mid - 1;
     }
-    ui.j = jlo;
-    ui.jb = p.jobs ? p.jobs[jlo] : p.one;
-    ui.ldx = p.jobs ? ui.jb.K : p.ldx;
-    ui.ldy = p.jobs ? ui.jb.M : p.ldy;
-    const int S = slices_of(ui.jb.K);
-    ui.nch = (S + p.chunk_slices - 1) / p.chunk_slices;
-    uint32_t r = u - lo.unit_prefix[jlo];
-    ui.t = static_cast<int>(r % static_cast<uint32_t>(p.T));
-    r /= static_cast<uint32_t>(p.T);
-    ui.ch = static_cast<int>(r % static_cast<uint32_t>(ui.nch));
-    ui.rb = static_cast<int>(r / static_cast<uint32_t>(ui.nch));
-    ui.s_begin = ui.ch * p.chunk_slices;
-    ui.s_end = min(S, ui.s_begin + p.chunk_slices);
-    return ui;
+    const GvJob jb = p.jobs ? p.jobs[jlo] : p.one;
+    const int64_t ldx = p.jobs ? jb.K : p.ldx;
+    const int64_t ldy = p.jobs ? jb.M : p.ldy;
+    const int S = slices_of(jb.K);
+    const uint32_t nch = static_cast<uint32_t>((S + p.chunk_slices - 1) / p.chunk_slices);
+    uint32_t q = u - unit_prefix[jlo];
+    const uint32_t t = q % static_cast<uint32_t>(p.T);
+    q /= static_cast<uint32_t>(p.T);
+    const uint32_t ch = q % nch;
+    r.planes = jb.planes;
+    r.alpha = jb.alpha;
+    r.x = static_cast<const __half*>(jb.x) + t * ldx;
+    r.y = static_cast<char*>(jb.y) + t * ldy * (p.y_f16 ? 2 : 4);
+    r.M = jb.M;
+    r.K = jb.K;
+    r.rb = q / nch;
+    r.j = static_cast<uint32_t>(jlo);
+    r.t = t;
+    r.ch = ch;
+    r.nch = nch;
+    r.s_begin = ch * static_cast<uint32_t>(p.chunk_slices);
+    r.s_end = min(static_cast<uint32_t>(S), r.s_begin + static_cast<uint32_t>(p.chunk_slices));
+    r.pad = 0;
 }
 
 // Every CTA computes the same unit prefix sums over the jobs: each thread
@@ -320,187 +353,261 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_lut_kernel(GvArgs p, uint32_t
     // The 8 lanes sharing t8 & 3 (t8 in {a, a + 4}, 4 items) would hit the
     // same banks; lane z = (t8 >> 2) + 2 q4 swaps its two words when z is odd
     // (rv) and rotates the byte order by rq = z >> 1, so every LDS touches 32
-    // distinct banks.
+    // distinct banks. One PRMT per word does both: word v' of the lane is
+    // (rv ? word 1 - v : word v) with byte q taken from byte (q + rq) & 3.
     const uint32_t zr = static_cast<uint32_t>((t8 >> 2) + 2 * q4);
     const uint32_t rv = zr & 1u, rq = zr >> 1;
-    const uint32_t swap_mask = 0u - rv;
-    uint32_t sel[4];
+    uint32_t perm0 = 0, perm1 = 0;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) sel[q] = 0x7604u | (((static_cast<uint32_t>(q) + rq) & 3u) << 4);
+    for (int q = 0; q < 4; ++q) {
+        const uint32_t byte = (static_cast<uint32_t>(q) + rq) & 3u;
+        perm0 |= (byte + 4u * rv) << (4 * q);
+        perm1 |= (byte + 4u * (rv ^ 1u)) << (4 * q);
+    }
 
-    uint32_t iter = 0;
-    while (true) {
-        uint32_t u;
-        if (p.dynamic) {
-            if (tid == 0) lo.bcast = atomicAdd(hdr, 1u);
-            cta_sync();
-            u = lo.bcast;
-            cta_sync();
-        } else {
-            u = blockIdx.x + iter * gridDim.x;
+    // ---- this CTA's units: u = blockIdx.x + k * gridDim.x, k < n_my, decoded
+    // into the ring of unit records ahead of use
+    const uint32_t G = gridDim.x, bid = blockIdx.x;
+    const uint32_t n_my = total_units > bid ? (total_units - bid + G - 1) / G : 0u;
+    if (n_my == 0) return;   // uniform over the CTA
+    uint32_t decoded = 0;
+    auto decode_upto = [&](uint32_t to) {
+        for (uint32_t k = decoded + tid; k < to; k += THREADS)
+            decode_rec(p, lo.unit_prefix, n_jobs, bid + k * G, lo.units[k % UCAP]);
+        decoded = to;
+        cta_sync();
+    };
+    decode_upto(min(n_my, static_cast<uint32_t>(UCAP)));
+
+    // The step `d` steps after (unit k, slice s) in this CTA's sequence of
+    // (unit, slice) steps; false past the last unit. Needs units up to k + d
+    // decoded (every unit has at least one slice).
+    auto step_after = [&](uint32_t k, int s, int d, uint32_t& ko, int& so) -> bool {
+        while (true) {
+            const UnitRec& r = lo.units[k % UCAP];
+            if (s + d < static_cast<int>(r.s_end)) {
+                ko = k;
+                so = s + d;
+                return true;
+            }
+            d -= static_cast<int>(r.s_end) - s;
+            if (++k >= n_my) return false;
+            s = static_cast<int>(lo.units[k % UCAP].s_begin);
         }
-        ++iter;
-        if (u >= total_units) break;
+    };
+    // threads 0..63 stage the x of step (k, s) + d into `dst`
+    auto stage_step = [&](uint32_t k, int s, int d, uint4* dst) {
+        if (tid < 64) {
+            uint32_t ko;
+            int so;
+            if (step_after(k, s, d, ko, so)) {
+                const UnitRec& r = lo.units[ko % UCAP];
+                stage_x(r.x, r.K, so, dst);
+            }
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
 
-        const UnitInfo ui = decode_unit(p, lo, n_jobs, u);
-        const GvJob& jb = ui.jb;
-        const int64_t M = jb.M, K = jb.K;
-        const int S = slices_of(K);
-        const int s_begin = ui.s_begin, s_end = ui.s_end;
-        const uint32_t uM = static_cast<uint32_t>(M);
+    // items 2i and 2i + 1 accumulate as one fp32 pair (add.f32x2)
+    uint64_t acc2[J / 2];
+    uint2 wv[J];
+    float av[J];
+#pragma unroll
+    for (int j = 0; j < J; ++j) av[j] = 0.0f;
+    // Table address of lookup step i = 4 v + q (byte q of permuted word
+    // v): TBL | b << 8 | 4c with c = 8 t8 + 4 (v ^ rv) + (q + rq) & 3.
+    // Register pb[i / 2] holds 4c of steps i and i + 1 in bytes 0 and 1,
+    // the table's 64 KB page in byte 2 and 0 in byte 3; the address PRMT
+    // takes byte 0 or 1 of it, the plane byte, then bytes 2 and 3.
+    uint32_t pb[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        uint32_t r = TBL0;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const uint32_t v = static_cast<uint32_t>((2 * k + h) >> 2), q = static_cast<uint32_t>((2 * k + h) & 3);
+            r |= (4u * (8u * t8 + 4u * (v ^ rv) + ((q + rq) & 3u))) << (8 * h);
+        }
+        pb[k] = r;
+    }
+    uint32_t tbl_next = TBL0 + 0x10000u;   // buffer of the next step's table
+
+    // Where item loads of one slice of one unit come from. Item load j: path
+    // j / HR, rows r0 + 4 (j % HR) + q4. In a full warp its lane pointer is
+    // the path pointer + (j % HR) * (4 rows), an immediate offset in the
+    // sliced layout; other warps clamp rows to M - 1 (absolute addresses).
+    struct SliceAddr {
+        const char* slice0;   // (path 0, row 0, pair tsel) of the slice
+        const char* lane0;    // (path 0, row r0 + q4, pair tsel)
+        const void* alpha;
+        uint32_t r0, tp, uM, path_bytes, row_bytes, aoff, gpr;
+    };
+    auto make_addr = [&](const uint32_t* planes, const void* alpha, uint32_t uM, int64_t K, uint32_t rb, int s) {
+        SliceAddr a;
+        // word pair of lane t8, clamped in a partial last slice (the table
+        // entries past K are 0, so a clamped pair adds nothing); the sliced
+        // layout pads the last slice, so only the scale index and the row
+        // layout need it
+        const int ws = min(16, static_cast<int>((K - static_cast<int64_t>(s) * SLICE_COLS) >> 5));
+        a.tp = 2 * t8 < ws ? static_cast<uint32_t>(t8) : 0u;
+        a.r0 = rb * C::R + warp * C::RW;
+        asm volatile("" : "+r"(a.r0));
+        a.uM = uM;
+        const uint32_t S = static_cast<uint32_t>(slices_of(K));
         const uint32_t uW32 = static_cast<uint32_t>(K >> 5);
-        const uint32_t gpr = static_cast<uint32_t>(K >> 7);
-        const uint32_t row0 = static_cast<uint32_t>(ui.rb) * C::R + warp * C::RW;
-        const __half* xt = static_cast<const __half*>(jb.x) + ui.t * ui.ldx;
-        // plane bytes per path in each layout
-        const uint32_t path_bytes = SLICED ? static_cast<uint32_t>(S) * 64u * uM : uM * uW32 * 4u;
-        // a full warp has every row of its items below M; others clamp rows
-        // (the sums of the extra rows are computed and dropped)
-        const bool full = row0 + C::RW <= uM;
-
-        float acc[J];
-        uint2 wv[J];
-        float av[J];
-#pragma unroll
-        for (int j = 0; j < J; ++j) {
-            acc[j] = 0.0f;
-            av[j] = 0.0f;
+        a.path_bytes = SLICED ? S * 64u * uM : uM * uW32 * 4u;
+        a.row_bytes = SLICED ? 64u : uW32 * 4u;
+        a.alpha = alpha;
+        a.gpr = static_cast<uint32_t>(K >> 7);
+        a.aoff = 4u * static_cast<uint32_t>(s) + (a.tp >> 1);
+        const uint32_t tsel = SLICED ? static_cast<uint32_t>(t8) : a.tp;
+        a.slice0 = reinterpret_cast<const char*>(planes) +
+                   (SLICED ? (static_cast<size_t>(s) * uM * 16u + 2u * tsel) * 4u
+                           : (16u * static_cast<uint32_t>(s) + 2u * tsel) * 4u);
+        a.lane0 = mad_ptr(a.r0 + q4, a.row_bytes, a.slice0);
+        return a;
+    };
+    auto fetch = [&](int j, const SliceAddr& a, auto full_tag) {
+        constexpr bool F = decltype(full_tag)::value;
+        const uint32_t path = j / HR, rr = j % HR;
+        uint32_t row;
+        const char* wp;
+        if (F) {
+            row = a.r0 + q4 + 4u * rr;
+            const char* pp = path ? mad_ptr(path, a.path_bytes, a.lane0) : a.lane0;
+            wp = SLICED ? pp + rr * 256u : mad_ptr(4u * rr, a.row_bytes, pp);
+        } else {
+            row = min(a.r0 + q4 + 4u * rr, a.uM - 1u);
+            wp = mad_ptr(row, a.row_bytes, path ? mad_ptr(path, a.path_bytes, a.slice0) : a.slice0);
         }
-        // table address base of step (word v, byte q): column 8 t8 + 4 (v ^ rv) + (q + rq) & 3
-        uint32_t cur_base[8];
+        // K is a multiple of 128, so rows of either layout are a multiple
+        // of 16 bytes, the planes are 16-byte aligned and a slice holds an
+        // even number of words: the pair is one aligned 8-byte load
+        wv[j] = ldg_words2(wp);
+        if (G128) {
+            const size_t ai = static_cast<size_t>(path * a.uM + row) * a.gpr + a.aoff;
+            av[j] = A16 ? __half2float(static_cast<const __half*>(a.alpha)[ai]) : static_cast<const float*>(a.alpha)[ai];
+        }
+    };
+    auto fetch_all = [&](const SliceAddr& a, auto full_tag) {
 #pragma unroll
-        for (int v = 0; v < 2; ++v)
+        for (int j = 0; j < J; ++j)
+            if (j < C::JV) fetch(j, a, full_tag);
+    };
+    // consume the current slice from the current table; with PF, items of
+    // the next step (at `an`) are loaded right after the same items of this
+    // slice were used, so each load has about one slice of time to arrive
+    auto consume = [&](const SliceAddr& an, auto pf_tag, auto full_tag) {
+        constexpr bool PF = decltype(pf_tag)::value;
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-                cur_base[4 * v + q] = TBL0 + 4u * (8u * t8 + 4u * (static_cast<uint32_t>(v) ^ rv) +
-                                                   ((static_cast<uint32_t>(q) + rq) & 3u));
-
-        // word pair of lane t8 in slice s, clamped in a partial last slice
-        // (the table entries past K are 0, so a clamped pair adds nothing);
-        // the sliced layout pads the last slice, so only the scale index and
-        // the row layout need it
-        auto lane_pair = [&](int s) -> uint32_t {
-            const int ws = min(16, static_cast<int>((K - static_cast<int64_t>(s) * SLICE_COLS) >> 5));
-            return 2 * t8 < ws ? static_cast<uint32_t>(t8) : 0u;
-        };
-        auto alpha_at = [&](size_t ai) -> float {
-            return A16 ? __half2float(static_cast<const __half*>(jb.alpha)[ai]) : static_cast<const float*>(jb.alpha)[ai];
-        };
-        // Item load j: path j / HR, rows row0 + 4 (j % HR) + q4. Its lane
-        // pointer = path pointer + (j % HR) * (4 rows): an immediate offset in
-        // the sliced layout. The per-slice row goes through an empty asm so
-        // the compiler cannot hoist per-item values.
-        struct SliceAddr {
-            const char* slice0;   // (path 0, row 0, pair tsel) of the slice
-            const char* lane0;    // (path 0, row r0 + q4, pair tsel): full warps
-            uint32_t r0, tp;
-        };
-        const uint32_t row_bytes = SLICED ? 64u : uW32 * 4u;
-        auto slice_addr = [&](int s) {
-            SliceAddr a;
-            a.tp = lane_pair(s);
-            a.r0 = row0;
-            asm volatile("" : "+r"(a.r0));
-            const uint32_t tsel = SLICED ? static_cast<uint32_t>(t8) : a.tp;
-            a.slice0 = reinterpret_cast<const char*>(jb.planes) +
-                       (SLICED ? (static_cast<size_t>(s) * uM * 16u + 2u * tsel) * 4u
-                               : (16u * static_cast<uint32_t>(s) + 2u * tsel) * 4u);
-            a.lane0 = mad_ptr(a.r0 + q4, row_bytes, a.slice0);
-            return a;
-        };
-        // load item j of the slice at `a` (words swapped on lanes with rv)
-        auto fetch = [&](int j, int s, const SliceAddr& a, auto full_tag) {
-            constexpr bool F = decltype(full_tag)::value;
-            const uint32_t path = j / HR, rr = j % HR;
-            uint32_t row;
-            const char* wp;
-            if (F) {
-                row = a.r0 + q4 + 4u * rr;
-                const char* pb = path ? mad_ptr(path, path_bytes, a.lane0) : a.lane0;
-                wp = SLICED ? pb + rr * 256u : mad_ptr(4u * rr, row_bytes, pb);
-            } else {
-                // rows past M are clamped to the last row (absolute address)
-                row = min(a.r0 + q4 + 4u * rr, uM - 1u);
-                wp = mad_ptr(row, row_bytes, path ? mad_ptr(path, path_bytes, a.slice0) : a.slice0);
+        for (int i = 0; i < J / 2; ++i) {
+            const int j0 = 2 * i, j1 = 2 * i + 1;
+            if (j0 >= C::JV) continue;
+            const bool has1 = j1 < C::JV;
+            // the word permutation happens here, where the words are
+            // used, not where they are loaded (a use right after the load
+            // would wait for it)
+            const uint32_t a0 = prmt(wv[j0].x, wv[j0].y, perm0), a1 = prmt(wv[j0].x, wv[j0].y, perm1);
+            uint32_t b0 = 0, b1 = 0;
+            if (has1) {
+                b0 = prmt(wv[j1].x, wv[j1].y, perm0);
+                b1 = prmt(wv[j1].x, wv[j1].y, perm1);
             }
-            // K is a multiple of 128, so rows of either layout are a multiple
-            // of 16 bytes, the planes are 16-byte aligned and a slice holds an
-            // even number of words: the pair is one aligned 8-byte load
-            wv[j] = ldg_words2(wp);
-            if (G128) av[j] = alpha_at(static_cast<size_t>(path * uM + row) * gpr + 4u * s + (a.tp >> 1));
-        };
-        auto fetch_slice = [&](int s, auto full_tag) {
-            const SliceAddr a = slice_addr(s);
+            uint64_t pr[8];
 #pragma unroll
-            for (int j = 0; j < J; ++j)
-                if (j < C::JV) fetch(j, s, a, full_tag);
-        };
-        // consume slice s from the current table; with PF, item j of slice
-        // s + 1 is loaded right after item j of slice s was used, so each load
-        // has about one slice of time to arrive
-        auto consume = [&](int s, auto full_tag, auto pf_tag) {
-            constexpr bool PF = decltype(pf_tag)::value;
-            SliceAddr an;
-            if (PF) an = slice_addr(s + 1);
-#pragma unroll
-            for (int j = 0; j < J; ++j) {
-                if (j >= C::JV) continue;
-                // the word swap of lanes with rv happens here, where the words
-                // are used, not where they are loaded (a use right after the
-                // load would wait for it)
-                const uint32_t w0 = sel_mask(wv[j].x, wv[j].y, swap_mask);
-                const uint32_t w1 = sel_mask(wv[j].y, wv[j].x, swap_mask);
-                const float v0 = lds(prmt(w0, cur_base[0], sel[0]));
-                const float v1 = lds(prmt(w0, cur_base[1], sel[1]));
-                const float v2 = lds(prmt(w0, cur_base[2], sel[2]));
-                const float v3 = lds(prmt(w0, cur_base[3], sel[3]));
-                const float v4 = lds(prmt(w1, cur_base[4], sel[0]));
-                const float v5 = lds(prmt(w1, cur_base[5], sel[1]));
-                const float v6 = lds(prmt(w1, cur_base[6], sel[2]));
-                const float v7 = lds(prmt(w1, cur_base[7], sel[3]));
-                const float ps = ((v0 + v1) + (v2 + v3)) + ((v4 + v5) + (v6 + v7));
-                if (G128) acc[j] = fmaf(av[j], ps, acc[j]);
-                else acc[j] += ps;
-                if (PF) fetch(j, s + 1, an, full_tag);
+            for (int st = 0; st < 8; ++st) {
+                const uint32_t q = st & 3;
+                const uint32_t sel = 0x7600u | (q << 4) | (4u + (st & 1));
+                const float e0 = lds(prmt(st < 4 ? a0 : a1, pb[st >> 1], sel));
+                const float e1 = has1 ? lds(prmt(st < 4 ? b0 : b1, pb[st >> 1], sel)) : 0.0f;
+                pr[st] = pack_f2(e0, e1);
             }
-        };
+            const uint64_t ps = add_f2(add_f2(add_f2(pr[0], pr[1]), add_f2(pr[2], pr[3])),
+                                       add_f2(add_f2(pr[4], pr[5]), add_f2(pr[6], pr[7])));
+            if (G128) acc2[i] = fma_f2(pack_f2(av[j0], av[j1]), ps, acc2[i]);
+            else acc2[i] = add_f2(acc2[i], ps);
+            if (PF) {
+                fetch(j0, an, full_tag);
+                if (has1) fetch(j1, an, full_tag);
+            }
+        }
+    };
 
-        // ---- slice pipeline: table of slice s in buffer (s - s_begin) & 1;
-        // the x of slice s + 2 is staged while slice s is consumed, so each
-        // slice needs one CTA barrier. Full and partial warps run separate
-        // copies of the whole loop (non-aligned barriers), the last slice is
-        // peeled, so the steady-state loop is one straight-line block.
+    // ---- prologue: words, x and table of the first step, x of the second
+    uint32_t g = 0;   // global step counter: x of step g in xstage[g & 1]
+    {
+        const UnitRec& r = lo.units[0];
+        fetch_all(make_addr(r.planes, r.alpha, static_cast<uint32_t>(r.M), r.K, r.rb, static_cast<int>(r.s_begin)),
+                  BoolC<false>{});
+        stage_step(0, static_cast<int>(r.s_begin), 0, lo.xstage[0]);
+        stage_step(0, static_cast<int>(r.s_begin), 1, lo.xstage[1]);
+        stage_wait_all();
+        cta_sync();
+        build_table(lo.xstage[0], TBL0);
+        cta_sync();
+    }
+
+    for (uint32_t k = 0; k < n_my; ++k) {
+        if (decoded < n_my && decoded < k + 3) decode_upto(min(n_my, decoded + UCAP / 2));
+        const UnitRec& ur = lo.units[k % UCAP];
+        const uint32_t* planes = ur.planes;
+        const void* alpha = ur.alpha;
+        const uint32_t uM = static_cast<uint32_t>(ur.M);
+        const int64_t K = ur.K;
+        const uint32_t rb = ur.rb;
+        const int s_begin = static_cast<int>(ur.s_begin), s_end = static_cast<int>(ur.s_end);
+        const bool has_next = k + 1 < n_my;
+        const uint32_t row0 = rb * C::R + warp * C::RW;
+        // a full warp has every row of its items below M
+        const bool full = row0 + C::RW <= uM;
+#pragma unroll
+        for (int i = 0; i < J / 2; ++i) acc2[i] = 0ull;
+        // the per-row scales of this warp's rows, read in the epilogue, are
+        // brought into L1 now
+        if (!G128 && lane < 2 * NP) {
+            const uint32_t row = min(row0 + (lane & 1) * (C::RW - 1), uM - 1u);
+            const size_t ai = static_cast<size_t>(lane >> 1) * uM + row;
+            const char* ap = static_cast<const char*>(alpha) + ai * (p.alpha_f16 ? 2 : 4);
+            asm volatile("prefetch.global.L1 [%0];" ::"l"(ap));
+        }
+
+        // one step: build the next step's table, stage x two steps ahead,
+        // consume this slice (loading the next step's words), one barrier
+        auto step = [&](int s, bool build_next, const SliceAddr& an, auto pf_tag, auto full_tag) {
+            if (build_next) build_table(lo.xstage[(g + 1) & 1], tbl_next);
+            stage_step(k, s, 2, lo.xstage[g & 1]);
+            consume(an, pf_tag, full_tag);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) pb[q] ^= TBL_TOGGLE;
+            tbl_next ^= TBL_TOGGLE;
+            ++g;
+            stage_wait_all();
+            cta_sync_any();
+        };
+        // Full and partial warps run separate copies of the unit's steps
+        // (non-aligned barriers); the last step is peeled: it loads the next
+        // unit's first words (rows clamped, whatever that unit's shape)
         auto run_unit = [&](auto full_tag) {
-            fetch_slice(s_begin, full_tag);
-            stage_x(xt, K, s_begin, lo.xstage[0]);
-            stage_wait_all();
-            cta_sync_any();
-            build_table(lo.xstage[0], TBL0);
-            if (s_begin + 1 < s_end) stage_x(xt, K, s_begin + 1, lo.xstage[1]);
-            stage_wait_all();
-            cta_sync_any();
-            for (int s = s_begin; s < s_end - 1; ++s) {
-                const int par = (s - s_begin) & 1;
-                build_table(lo.xstage[par ^ 1], par ? TBL0 : TBL0 + 0x10000u);
-                if (s + 2 < s_end) stage_x(xt, K, s + 2, lo.xstage[par]);
-                consume(s, full_tag, BoolC<true>{});
-#pragma unroll
-                for (int q = 0; q < 8; ++q) cur_base[q] ^= TBL_TOGGLE;
-                stage_wait_all();
-                cta_sync_any();
+            for (int s = s_begin; s < s_end - 1; ++s)
+                step(s, true, make_addr(planes, alpha, uM, K, rb, s + 1), BoolC<true>{}, full_tag);
+            if (has_next) {
+                const UnitRec& rn = lo.units[(k + 1) % UCAP];
+                step(s_end - 1, true,
+                     make_addr(rn.planes, rn.alpha, static_cast<uint32_t>(rn.M), rn.K, rn.rb,
+                               static_cast<int>(rn.s_begin)),
+                     BoolC<true>{}, BoolC<false>{});
+            } else {
+                SliceAddr none{};
+                step(s_end - 1, false, none, BoolC<false>{}, full_tag);
             }
-            consume(s_end - 1, full_tag, BoolC<false>{});
-            cta_sync_any();
         };
         if (full) run_unit(BoolC<true>{});
         else run_unit(BoolC<false>{});
 
-        // the unit's indices are decoded again rather than kept live across
-        // the slice loop, which leaves the registers to the accumulators
-        asm volatile("" : "+r"(u));
-        const UnitInfo ue = decode_unit(p, lo, n_jobs, u);
-
         // ---- reduce over the 8 lanes of each item; lane t8 owns load j = t8 >> shift
+        float acc[J];
+#pragma unroll
+        for (int i = 0; i < J / 2; ++i) unpack_f2(acc2[i], acc[2 * i], acc[2 * i + 1]);
         group8_transpose_reduce<J>(acc, t8);
         constexpr int shift = 3 - Log2<J>::v;
         if ((t8 & ((1 << shift) - 1)) == 0) lo.tot[warp][4 * (t8 >> shift) + q4] = acc[0];
@@ -508,36 +615,39 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_lut_kernel(GvArgs p, uint32_t
 
         // ---- per-row output of this chunk: lane r < RW owns row r of the warp,
         // whose path-k item is load k * HR + r / 4 of item group r % 4
+        const UnitRec& ue = lo.units[k % UCAP];
+        const int64_t M = ue.M;
         float yv = 0.0f;
         const int64_t my_row = static_cast<int64_t>(ue.rb) * C::R + warp * C::RW + lane;
-        const bool row_ok = lane < C::RW && my_row < ue.jb.M;
+        const bool row_ok = lane < C::RW && my_row < M;
         if (row_ok) {
 #pragma unroll
-            for (int k = 0; k < NP; ++k) {
-                const float tk = lo.tot[warp][4 * (k * HR + (lane >> 2)) + (lane & 3)];
+            for (int kk = 0; kk < NP; ++kk) {
+                const float tk = lo.tot[warp][4 * (kk * HR + (lane >> 2)) + (lane & 3)];
                 if (G128) {
                     yv += tk;
                 } else {
-                    const size_t ai = static_cast<size_t>(k) * ue.jb.M + my_row;
-                    const float a = p.alpha_f16 ? __half2float(static_cast<const __half*>(ue.jb.alpha)[ai])
-                                                : static_cast<const float*>(ue.jb.alpha)[ai];
+                    const size_t ai = static_cast<size_t>(kk) * M + my_row;
+                    const float a = p.alpha_f16 ? __half2float(static_cast<const __half*>(ue.alpha)[ai])
+                                                : static_cast<const float*>(ue.alpha)[ai];
                     yv = fmaf(a, tk, yv);
                 }
             }
         }
-        if (ue.nch == 1) {
+        const uint32_t nch = ue.nch;
+        if (nch == 1) {
             if (row_ok) {
-                if (p.y_f16) static_cast<__half*>(ue.jb.y)[ue.t * ue.ldy + my_row] = __float2half_rn(yv);
-                else static_cast<float*>(ue.jb.y)[ue.t * ue.ldy + my_row] = yv;
+                if (p.y_f16) static_cast<__half*>(ue.y)[my_row] = __float2half_rn(yv);
+                else static_cast<float*>(ue.y)[my_row] = yv;
             }
         } else {
-            float* part = parts + lo.part_prefix[ue.j] + (static_cast<size_t>(ue.t) * ue.nch) * ue.jb.M;
-            if (row_ok) part[static_cast<size_t>(ue.ch) * ue.jb.M + my_row] = yv;
+            float* part = parts + lo.part_prefix[ue.j] + (static_cast<size_t>(ue.t) * nch) * M;
+            if (row_ok) part[static_cast<size_t>(ue.ch) * M + my_row] = yv;
             __threadfence();
             cta_sync();
             if (tid == 0) {
                 const uint32_t prev = atomicAdd(ctrs + lo.ctr_prefix[ue.j] + ue.rb * T + ue.t, 1u);
-                lo.last = (prev == static_cast<uint32_t>(ue.nch - 1)) ? 1u : 0u;
+                lo.last = (prev == nch - 1) ? 1u : 0u;
             }
             cta_sync();
             if (lo.last) {
@@ -545,11 +655,11 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_lut_kernel(GvArgs p, uint32_t
                 const int64_t rbase = static_cast<int64_t>(ue.rb) * C::R;
                 for (int i = tid; i < C::R; i += THREADS) {
                     const int64_t row = rbase + i;
-                    if (row < ue.jb.M) {
+                    if (row < M) {
                         float sum = 0.0f;
-                        for (int c = 0; c < ue.nch; ++c) sum += __ldcg(part + static_cast<size_t>(c) * ue.jb.M + row);
-                        if (p.y_f16) static_cast<__half*>(ue.jb.y)[ue.t * ue.ldy + row] = __float2half_rn(sum);
-                        else static_cast<float*>(ue.jb.y)[ue.t * ue.ldy + row] = sum;
+                        for (uint32_t c = 0; c < nch; ++c) sum += __ldcg(part + static_cast<size_t>(c) * M + row);
+                        if (p.y_f16) static_cast<__half*>(ue.y)[row] = __float2half_rn(sum);
+                        else static_cast<float*>(ue.y)[row] = sum;
                     }
                 }
             }
@@ -567,7 +677,7 @@ cudaError_t launch_one(const GvArgs& a, const GvPlan& plan, cudaStream_t s) {
     uint32_t* ctrs = reinterpret_cast<uint32_t*>(static_cast<char*>(a.workspace) + GV_HEADER_BYTES);
     float* parts = reinterpret_cast<float*>(ctrs + ((plan.counters + 3) & ~size_t(3)));
     const int sms = device_sm_count();
-    size_t grid = a.dynamic ? static_cast<size_t>(sms) : plan.units;
+    size_t grid = plan.units;
     if (grid > static_cast<size_t>(sms)) grid = sms;
     if (grid < 1) grid = 1;
     kern<<<static_cast<unsigned>(grid), THREADS, SMEM_BYTES, s>>>(a, hdr, ctrs, parts);

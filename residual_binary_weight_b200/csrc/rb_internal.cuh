@@ -52,12 +52,11 @@ struct GvArgs {
     int T;
     int64_t ldx, ldy;       // pitches of the single matrix (grouped: K and M)
     int chunk_slices;       // 512-column slices per K chunk
-    bool dynamic;           // hand out units from the workspace counter
     void* workspace;
     size_t ws_bytes;
 };
 
-// Workspace layout: a 256-byte header (unit counter, error flag), then one
+// Workspace layout: a 256-byte header (word 1: error flags), then one
 // arrival counter per (job, row block, token) of every K-split job, then the
 // fp32 partial sums of the split jobs.
 constexpr size_t GV_HEADER_BYTES = 256;
