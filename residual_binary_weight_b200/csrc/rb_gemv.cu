@@ -261,8 +261,9 @@ __device__ __forceinline__ void decode_rec(const GvArgs& p, const uint32_t* unit
     r.t = t;
     r.ch = ch;
     r.nch = nch;
-    r.s_begin = ch * static_cast<uint32_t>(p.chunk_slices);
-    r.s_end = min(static_cast<uint32_t>(S), r.s_begin + static_cast<uint32_t>(p.chunk_slices));
+    // the S slices split into nch chunks of equal size (+-1)
+    r.s_begin = (ch * static_cast<uint32_t>(S)) / nch;
+    r.s_end = ((ch + 1) * static_cast<uint32_t>(S)) / nch;
     r.pad = 0;
 }
 
