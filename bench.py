@@ -198,13 +198,12 @@ def time_gemm(torch, rb, synth, device, peak_tf):
     return out
 
 
-def cpu_oracle_sample(budget_s: float = 12.0):
-    """The fp64 oracle's matvec on rows sampled from every matrix of layer 0."""
+def oracle_sample_inputs(rows_per: int = 96):
+    """Rows sampled from every matrix of layer 0, packed by the oracle."""
     import numpy as np
     import oracle
     import synth
     wl = synth.WORKLOADS[WORKLOAD]
-    rows_per = 96
     prepared = []
     for name in ORDER:
         sp = {m.name: m for m in wl.matrices}[name]
@@ -213,6 +212,14 @@ def cpu_oracle_sample(budget_s: float = 12.0):
         p, a, _ = oracle.pack(W, wl.n_paths, wl.group)
         x = synth.host_activations(wl, 0, name, 1).astype(np.float64)
         prepared.append((p, a.astype(np.float32).astype(np.float64), x, sp))
+    return prepared, rows_per
+
+
+def cpu_oracle_sample(budget_s: float = 12.0, inputs=None):
+    """The fp64 oracle's matvec on rows sampled from every matrix of layer 0,
+    repeated for about `budget_s` seconds; GB/s of the same algorithmic bytes."""
+    import oracle
+    prepared, rows_per = inputs if inputs is not None else oracle_sample_inputs()
     done_bytes, t0, reps = 0, time.perf_counter(), 0
     while True:
         for p, a, x, sp in prepared:
@@ -229,17 +236,27 @@ def cpu_oracle_sample(budget_s: float = 12.0):
                       f"OpenMP threads = {cores}"}
 
 
+def workload_config(layers: int) -> dict:
+    return {"workload": f"Llama-2-7B-shaped decode linears, batch 1: {layers} layers x (4 x 4096x4096, "
+                        "2 x 11008x4096, 1 x 4096x11008), 2 paths, fp32 per-row scales, fp16 x/y, "
+                        "sliced plane order",
+            "l2": "inputs larger than L2 (1.6 GB streamed per step)"}
+
+
 def run_reference(args):
     ws, rank, _ = _dist_env()
     if rank != 0:
         return 0
-    per_step = []
+    # each step is a bounded sample of the workload, sized so that the whole
+    # run stays within a few minutes whatever --steps is
+    budget = min(8.0, max(0.3, 150.0 / max(1, args.steps + args.warmup)))
+    inputs = oracle_sample_inputs()
     for _ in range(args.warmup):
-        cpu_oracle_sample(budget_s=2.0)
+        cpu_oracle_sample(budget_s=budget, inputs=inputs)
     t_all = time.perf_counter()
     vals = []
     for _ in range(args.steps):
-        r = cpu_oracle_sample(budget_s=8.0)
+        r = cpu_oracle_sample(budget_s=budget, inputs=inputs)
         vals.append(r["value"])
     dt = time.perf_counter() - t_all
     v = sorted(vals)[len(vals) // 2]
@@ -247,8 +264,7 @@ def run_reference(args):
             "warmup": args.warmup, "ms_per_step": round(dt / max(args.steps, 1) * 1e3, 1),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
-            "config": {"workload": "Llama-2-7B-shaped decode linears, batch 1, 2 paths, per-row scales "
-                                   "(sampled rows, fp64 CPU oracle)"},
+            "config": workload_config(args.layers),
             "cpu_baseline": {"value": v, "unit": "GB/s", "cores": r["cores"], "kind": "oracle",
                              "sample": r["sample"]},
             "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -360,14 +376,10 @@ def run_gpu(args):
         "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded device draws: per-row sigma log-uniform [0.005, 0.05], 0.1% entries x10; "
                 "x N(0,1) with 0.5% channels x20)",
-        "config": {"workload": f"Llama-2-7B-shaped decode linears, batch 1: {args.layers} layers x (4 x 4096x4096, "
-                               "2 x 11008x4096, 1 x 4096x11008), 2 paths, fp32 per-row scales, fp16 x/y, "
-                               "sliced plane order",
-                   "bytes_per_step": alg_bytes, "l2": "inputs larger than L2 (1.6 GB streamed per step)",
-                   "parallelism": f"replicas x{ws}"},
+        "config": dict(workload_config(args.layers), bytes_per_step=alg_bytes, parallelism=f"replicas x{ws}"),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                      "frac": round(achieved / hbm_peak, 4), "traffic": _traffic_per_launch(),
-                     "peak_kind": f"{peak_kind} copy bandwidth", "kernel": "gemv_lut_kernel<2,0,0>",
+                     "peak_kind": f"{peak_kind} copy bandwidth", "kernel": "gemv_lut_kernel<2,0,0,1>",
                      "kernel_us": round(kern_ms * 1e3, 1)},
         "e2e": e2e,
         "gpu_launches": args.steps,
