@@ -147,24 +147,48 @@ def build_stack(torch, rb, synth, device, layers=32):
     return items, xbuf, ybuf, alg_bytes
 
 
-def time_pack(torch, rb, synth, device):
-    wl = synth.WORKLOADS[WORKLOAD]
-    W = synth.device_weight(wl, 0, "gate", device)
-    M, K = W.shape
+def _graph_time_us(torch, fn, n=20):
+    """Device time of fn() replayed from a CUDA graph (no host overhead between
+    launches); fn must only enqueue work on the current stream."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for _ in range(3):
+            fn()
+    torch.cuda.current_stream().wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        fn()
     for _ in range(3):
-        rb.pack(W, 2, 0)
+        graph.replay()
     torch.cuda.synchronize()
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    n = 20
     s.record()
     for _ in range(n):
-        rb.pack(W, 2, 0)
+        graph.replay()
     e.record()
     torch.cuda.synchronize()
-    ms = s.elapsed_time(e) / n
-    b = M * K * 2 + 2 * M * K // 8 + 2 * M * 4
-    return {"shape": [M, K], "n_paths": 2, "us": round(ms * 1e3, 2), "GB/s": round(b / ms / 1e6, 1),
-            "bytes": b}
+    us = s.elapsed_time(e) / n * 1e3
+    del graph
+    return us
+
+
+def time_pack(torch, rb, synth, device):
+    """rb_pack on the 7B gate matrix (2 paths, per-row scales) and on the QBB
+    up matrix (4 paths, fp16 scales per 128 columns)."""
+    out = {}
+    for wl_name, name, n_paths, group in (("llama2_7b_decode", "gate", 2, 0), ("qbb_g128", "up", 4, 128)):
+        wl = synth.WORKLOADS[wl_name]
+        W = synth.device_weight(wl, 0, name, device)
+        M, K = W.shape
+        a16 = group == 128
+        us = _graph_time_us(torch, lambda: rb.pack(W, n_paths, group, alpha_f16=a16))
+        G = K if group == 0 else group
+        b = M * K * W.element_size() + n_paths * M * K // 8 + n_paths * M * (K // G) * (4 + (2 if a16 else 0))
+        out[f"{wl_name}/{name}"] = {"shape": [M, K], "n_paths": n_paths, "group": group, "us": round(us, 2),
+                                   "GB/s": round(b / us / 1e3, 1), "bytes": b}
+        del W
+    return out
 
 
 def time_gemm(torch, rb, synth, device, peak_tf):

@@ -137,6 +137,83 @@ __device__ __forceinline__ void load32(const WT* p, float (&v)[32]) {
     }
 }
 
+// One scale per row, K <= 32768: thread tr of a row's `tpr` threads owns
+// plane word tr (columns 32 tr .. 32 tr + 31) for every path, so the sign
+// bits of a word are packed in registers and stored as one 32-bit word. A
+// CTA packs rows_per_cta rows; |R| is summed in fp32 over the 32 values of
+// a word (balanced tree), then in fp64 over the words of the row (warp
+// shuffles, then the row's warps through shared memory, in a fixed order).
+template <typename WT>
+__global__ void __launch_bounds__(1024)
+pack_words_kernel(const WT* __restrict__ W, int64_t ldw, int M, int K, int N, bool sliced, int tpr,
+                  int rows_per_cta, uint32_t* __restrict__ planes, float* __restrict__ alpha,
+                  __half* __restrict__ alpha16) {
+    __shared__ double red[2][32];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int rl = tid / tpr, tr = tid - rl * tpr;
+    const int row = blockIdx.x * rows_per_cta + rl;
+    const int words = K >> 5;
+    const bool active = row < M && tr < words;
+    const int wpr = tpr >> 5;   // warps per row when tpr >= 32
+    const size_t S = (static_cast<size_t>(K) + 511) / 512;
+
+    float r[32];
+    if (active) {
+        load32(W + static_cast<int64_t>(row) * ldw + 32 * tr, r);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) r[e] = __fadd_rn(r[e], 0.0f);   // -0.0 -> +0.0 (sign(0) = +1)
+    } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) r[e] = 0.0f;
+    }
+    for (int k = 0; k < N; ++k) {
+        float t[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) t[e] = fabsf(r[2 * e]) + fabsf(r[2 * e + 1]);
+#pragma unroll
+        for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+            for (int e = 0; e < w; ++e) t[e] = t[2 * e] + t[2 * e + 1];
+        double sum = static_cast<double>(t[0]);
+        if (tpr <= 32) {
+            for (int o = 1; o < tpr; o <<= 1) sum += __shfl_xor_sync(FULL_MASK, sum, o);
+        } else {
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) sum += __shfl_xor_sync(FULL_MASK, sum, o);
+            if (lane == 0) red[k & 1][warp] = sum;
+            __syncthreads();
+            sum = 0.0;
+            for (int w = 0; w < wpr; ++w) sum += red[k & 1][rl * wpr + w];
+        }
+        // every lane of a row holds the same sum; one lane per warp divides
+        float a = 0.0f;
+        if ((lane & (min(tpr, 32) - 1)) == 0) a = static_cast<float>(sum / static_cast<double>(K));
+        a = __shfl_sync(FULL_MASK, a, lane & ~(min(tpr, 32) - 1));
+        if (active && tr == 0) {
+            alpha[static_cast<size_t>(k) * M + row] = a;
+            if (alpha16) alpha16[static_cast<size_t>(k) * M + row] = __float2half_rn(a);
+        }
+        // B = +1 where R >= 0 (R is never -0.0: the input was cleared of it
+        // and x + (-x) rounds to +0.0); R <- R + (-a B)
+        uint32_t word = 0;
+        // threads past the row's last word keep R = 0, so they add nothing
+        // to the next path's sum
+        const bool update = active && k + 1 < N;
+        const uint32_t neg_a = __float_as_uint(-a);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+            const uint32_t neg = __float_as_uint(r[e]) & 0x80000000u;
+            word |= (neg ? 0u : 1u) << e;
+            if (update) r[e] = __fadd_rn(r[e], __uint_as_float(neg_a ^ neg));
+        }
+        if (active) {
+            const size_t wo = sliced ? ((static_cast<size_t>(k) * S + (tr >> 4)) * M + row) * 16 + (tr & 15)
+                                     : (static_cast<size_t>(k) * M + row) * words + tr;
+            planes[wo] = word;
+        }
+    }
+}
+
 // One scale per (path, row, 128 columns): lanes 4g..4g+3 of a warp own group g
 // (eight groups per warp per step); lane (4g + q) holds columns 32q..32q+31.
 template <typename WT>
@@ -199,7 +276,25 @@ cudaError_t launch_row(const PackArgs& a, int threads, cudaStream_t s) {
 }
 
 template <typename WT>
+cudaError_t launch_words(const PackArgs& a, cudaStream_t s) {
+    const int words = static_cast<int>(a.K >> 5);
+    int tpr = 4;
+    if (words <= 32) {
+        while (tpr < words) tpr <<= 1;
+    } else {
+        tpr = (words + 31) & ~31;
+    }
+    const int rows_per_cta = tpr >= 512 ? 1 : 512 / tpr;   // 512-thread CTAs: two per SM
+    const int64_t blocks = (a.M + rows_per_cta - 1) / rows_per_cta;
+    pack_words_kernel<WT><<<static_cast<unsigned>(blocks), rows_per_cta * tpr, 0, s>>>(
+        static_cast<const WT*>(a.W), a.ldw, static_cast<int>(a.M), static_cast<int>(a.K), a.n_paths, a.sliced, tpr,
+        rows_per_cta, a.planes, a.alpha, a.alpha16);
+    return cudaGetLastError();
+}
+
+template <typename WT>
 cudaError_t launch_row_any(const PackArgs& a, cudaStream_t s) {
+    if (a.K <= 32768) return launch_words<WT>(a, s);
     const int chunks = static_cast<int>(a.K >> 3);
     int cpt = 1;
     while (cpt < 8 && (chunks + cpt - 1) / cpt > 512) cpt *= 2;
