@@ -130,3 +130,33 @@ def test_token_tile_widths(T, n_paths, group):
     W = (rng.standard_normal((160, 512)) * 0.02).astype(np.float16)
     X = rng.standard_normal((T, 512)).astype(np.float16)
     _ok(_run(W, X, n_paths, group, group == 128, "sliced"), (T, n_paths, group))
+
+
+@pytest.mark.parametrize("T", [16, 64])
+@pytest.mark.parametrize("matrix", ["attn", "up", "down"])
+def test_llama3_full_size_sampled(matrix, T):
+    """The Llama-3-70B-shaped projections at batch 16 and 64 on the tensor-core
+    path: weight drawn and packed on the device, 32 sampled rows replaced by
+    the oracle's planes and scales, all tokens of those rows checked."""
+    wl = synth.WORKLOADS["llama3_70b_decode"]
+    spec = {m.name: m for m in wl.matrices}[matrix]
+    W = synth.device_weight(wl, 0, matrix, "cuda")
+    planes, alpha, _ = rb.pack(W, 2, 0, order="sliced")
+    rng = np.random.default_rng(3 * T + spec.K)
+    rows = np.sort(rng.choice(spec.M, 32, replace=False))
+    idx = torch.from_numpy(rows).cuda()
+    Wr = W.index_select(0, idx).cpu().numpy()
+    del W
+    ref_p, ref_a, _ = oracle.pack(Wr, 2, 0)
+    planes[:, :, idx] = to_dev_planes(ref_p, order="sliced")
+    a32 = ref_a.astype(np.float32)
+    alpha[:, idx] = torch.from_numpy(a32).cuda()
+    X = synth.device_activations(wl, 0, matrix, T, "cuda")
+    Y = rb.gemm(planes, alpha, X)
+    torch.cuda.synchronize()
+    from residual_binary_weight_b200._lib import check
+    check(rb.load().rb_gemm_check(None))
+    y_ref, den = oracle.matvec(ref_p, a32.astype(np.float64), X.cpu().numpy().astype(np.float64))
+    got = Y[:, idx].float().cpu().numpy()
+    nbad, worst = oracle.compare_outputs(got, y_ref, den)
+    assert nbad == 0, worst

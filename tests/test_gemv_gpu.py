@@ -199,3 +199,34 @@ def test_full_size_layer_sampled_rows():
         got = y[:, idx].float().cpu().numpy()
         nbad, worst = oracle.compare_outputs(got, y_ref, den)
         assert nbad == 0, worst
+
+
+@pytest.mark.parametrize("T", [1, 4, 16, 64])
+@pytest.mark.parametrize("matrix", ["attn", "up", "down"])
+def test_llama3_full_size_sampled(matrix, T):
+    """A full Llama-3-70B-shaped projection at batch T through the single-matrix
+    launch (K split into chunks, partial sums reduced by the last CTA). The
+    weight is drawn and packed on the device; 32 sampled rows get the oracle's
+    planes and scales, and their outputs for every token (at most 16 sampled
+    tokens) are checked against the oracle."""
+    wl = synth.WORKLOADS["llama3_70b_decode"]
+    spec = {m.name: m for m in wl.matrices}[matrix]
+    W = synth.device_weight(wl, 0, matrix, "cuda")
+    planes, alpha, _ = rb.pack(W, 2, 0, order="sliced")
+    rng = np.random.default_rng(T + spec.M)
+    rows = np.sort(rng.choice(spec.M, 32, replace=False))
+    idx = torch.from_numpy(rows).cuda()
+    Wr = W.index_select(0, idx).cpu().numpy()
+    del W
+    ref_p, ref_a, _ = oracle.pack(Wr, 2, 0)
+    planes[:, :, idx] = to_dev_planes(ref_p, order="sliced")
+    a32 = ref_a.astype(np.float32)
+    alpha[:, idx] = torch.from_numpy(a32).cuda()
+    x = synth.device_activations(wl, 0, matrix, T, "cuda")
+    y = rb.gemv(planes, alpha, x)
+    torch.cuda.synchronize()
+    toks = np.sort(rng.choice(T, min(T, 16), replace=False))
+    xs = x[torch.from_numpy(toks).cuda()].cpu().numpy().astype(np.float64)
+    y_ref, den = oracle.matvec(ref_p, a32.astype(np.float64), xs)
+    got = y[torch.from_numpy(toks).cuda()][:, idx].float().cpu().numpy()
+    _ok(oracle.compare_outputs(got, y_ref, den), (matrix, T))
