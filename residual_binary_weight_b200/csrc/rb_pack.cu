@@ -195,16 +195,19 @@ pack_words_kernel(const WT* __restrict__ W, int64_t ldw, int M, int K, int N, bo
         }
         // B = +1 where R >= 0 (R is never -0.0: the input was cleared of it
         // and x + (-x) rounds to +0.0); R <- R + (-a B)
-        uint32_t word = 0;
+        // The sign bits are gathered with one funnel shift per value (bit e of
+        // `neg` = sign of R[e]); the word is their complement.
+        uint32_t neg = 0;
+#pragma unroll
+        for (int e = 31; e >= 0; --e) neg = __funnelshift_l(__float_as_uint(r[e]), neg, 1);
+        const uint32_t word = ~neg;
         // threads past the row's last word keep R = 0, so they add nothing
         // to the next path's sum
-        const bool update = active && k + 1 < N;
-        const uint32_t neg_a = __float_as_uint(-a);
+        if (active && k + 1 < N) {
+            const uint32_t neg_a = __float_as_uint(-a);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-            const uint32_t neg = __float_as_uint(r[e]) & 0x80000000u;
-            word |= (neg ? 0u : 1u) << e;
-            if (update) r[e] = __fadd_rn(r[e], __uint_as_float(neg_a ^ neg));
+            for (int e = 0; e < 32; ++e)
+                r[e] = __fadd_rn(r[e], __uint_as_float((__float_as_uint(r[e]) & 0x80000000u) ^ neg_a));
         }
         if (active) {
             const size_t wo = sliced ? ((static_cast<size_t>(k) * S + (tr >> 4)) * M + row) * 16 + (tr & 15)
@@ -237,6 +240,8 @@ pack_g128_kernel(const WT* __restrict__ W, int64_t ldw, int M, int K, int N, boo
         float r[32];
         if (valid) {
             load32(W + row * ldw + 32 * wi, r);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) r[e] = __fadd_rn(r[e], 0.0f);   // -0.0 -> +0.0 (sign(0) = +1)
         } else {
 #pragma unroll
             for (int e = 0; e < 32; ++e) r[e] = 0.0f;
@@ -249,10 +254,17 @@ pack_g128_kernel(const WT* __restrict__ W, int64_t ldw, int M, int K, int N, boo
             s += __shfl_xor_sync(FULL_MASK, s, 1);
             s += __shfl_xor_sync(FULL_MASK, s, 2);
             const float a = static_cast<float>(s * (1.0 / 128.0));
-            const bool update = k + 1 < N;
-            uint32_t word = 0;
+            // sign bits by one funnel shift per value; R <- R + (-a B)
+            uint32_t neg = 0;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) word |= sign_and_update8(r + 8 * i, a, update) << (8 * i);
+            for (int e = 31; e >= 0; --e) neg = __funnelshift_l(__float_as_uint(r[e]), neg, 1);
+            const uint32_t word = ~neg;
+            if (k + 1 < N) {
+                const uint32_t neg_a = __float_as_uint(-a);
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                    r[e] = __fadd_rn(r[e], __uint_as_float((__float_as_uint(r[e]) & 0x80000000u) ^ neg_a));
+            }
             if (valid) {
                 const int64_t wo = sliced ? ((k * S + (wi >> 4)) * M + row) * 16 + (wi & 15)
                                           : (static_cast<int64_t>(k) * M + row) * words + wi;
