@@ -200,12 +200,17 @@ struct GemmArgs {
 template <int NP, int BN, int STAGES, bool G128>
 struct GemmCfg {
     static constexpr int NACC = G128 ? 1 : NP;                         // accumulators
+    // tensor-memory columns between accumulators: BN rounded up to a power of two
+    static constexpr int ACC_STRIDE = BN <= 16 ? 16 : BN <= 32 ? 32 : BN <= 64 ? 64 : BN <= 128 ? 128 : 256;
     static constexpr uint32_t B_TILE_BYTES = BN * BK * 2;
     static constexpr uint32_t STAGE_BYTES = NP * A_TILE_BYTES + B_TILE_BYTES;
-    static constexpr uint32_t TMEM_COLS = (NACC * BN <= 32) ? 32 : (NACC * BN <= 64) ? 64 :
-                                          (NACC * BN <= 128) ? 128 : (NACC * BN <= 256) ? 256 : 512;
+    static constexpr int ACC_COLS = NACC * ACC_STRIDE;
+    static constexpr uint32_t TMEM_COLS = (ACC_COLS <= 32) ? 32 : (ACC_COLS <= 64) ? 64 :
+                                          (ACC_COLS <= 128) ? 128 : (ACC_COLS <= 256) ? 256 : 512;
     static constexpr uint32_t SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
-    static_assert(NACC * BN <= 512, "accumulators exceed tensor memory");
+    static_assert(ACC_COLS <= 512, "accumulators exceed tensor memory");
+    static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M = 128");
+    static_assert(B_TILE_BYTES % 1024 == 0, "B tile must keep the 1024-byte swizzle alignment");
 };
 
 template <int NP, int BN, int STAGES, bool G128>
@@ -274,7 +279,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, GemmArgs a) {
                 tc_fence_after();
 #pragma unroll
                 for (int p = 0; p < NP; ++p) {
-                    const uint32_t d = tmem_base + static_cast<uint32_t>(G128 ? 0 : p * BN);
+                    const uint32_t d = tmem_base + static_cast<uint32_t>(G128 ? 0 : p * C::ACC_STRIDE);
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk) {
                         const uint64_t ad = smem_desc(a_tile(s, p) + 32u * kk);
@@ -357,7 +362,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, GemmArgs a) {
             }
             const uint32_t lane_addr = static_cast<uint32_t>((warp - EXP_WARP0) * 32) << 16;
             const int t_base = tok_tile * BN;
-            constexpr int CW = BN < 32 ? BN : 32;          // columns per tensor-memory load
+            // columns per tensor-memory load (a divisor of BN)
+            constexpr int CW = BN < 32 ? BN : (BN % 32 == 0 ? 32 : 16);
             for (int c0 = 0; c0 < BN; c0 += CW) {
                 float yv[CW];
 #pragma unroll
@@ -365,7 +371,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, GemmArgs a) {
 #pragma unroll
                 for (int p = 0; p < C::NACC; ++p) {
                     uint32_t v[CW];
-                    const uint32_t taddr = tmem_base + lane_addr + static_cast<uint32_t>(p * BN + c0);
+                    const uint32_t taddr = tmem_base + lane_addr + static_cast<uint32_t>(p * C::ACC_STRIDE + c0);
                     tmem_load<CW>(taddr, v);
 #pragma unroll
                     for (int i = 0; i < CW; ++i) yv[i] = fmaf(al[p], __uint_as_float(v[i]), yv[i]);
@@ -456,8 +462,24 @@ cudaError_t launch_np(const GemmArgs& a, const void* X, int64_t ldx, cudaStream_
     if (T <= 16) return launch_cfg<NP, 16, stages_for(NP, 16), G128>(a, X, ldx, s);
     if (T <= 32) return launch_cfg<NP, 32, stages_for(NP, 32), G128>(a, X, ldx, s);
     if (T <= 64) return launch_cfg<NP, 64, stages_for(NP, 64), G128>(a, X, ldx, s);
-    if (T <= 128 || BN_MAX == 128) return launch_cfg<NP, 128, stages_for(NP, 128), G128>(a, X, ldx, s);
+    if constexpr (BN_MAX == 128) {
+        return launch_cfg<NP, 128, stages_for(NP, 128), G128>(a, X, ldx, s);
+    } else {
+    if (T <= 128) return launch_cfg<NP, 128, stages_for(NP, 128), G128>(a, X, ldx, s);
+    // Wide token tiles: 240 instead of 256 when the last wave of 256-wide
+    // tiles would leave most SMs idle and 240 needs no extra wave: e.g. 112
+    // row tiles x 2048 tokens are 896 tiles of 256 (6 full waves on 148 SMs
+    // and 8 tiles in a seventh) or 1008 of 240 (7 waves, the last 81 % full).
+    // Measured: 14336 x 4096 x 2048 tokens 374 -> 350 us; 4096 x 14336 (256
+    // tiles of 256, last wave 73 % full) is slower with 240 and keeps 256.
+    const int64_t rows = (a.M + BM - 1) / BM, sms = device_sm_count();
+    const int64_t tiles256 = rows * ((T + 255) / 256), tiles240 = rows * ((T + 239) / 240);
+    const int64_t waves256 = (tiles256 + sms - 1) / sms, waves240 = (tiles240 + sms - 1) / sms;
+    const int64_t last256 = tiles256 - (waves256 - 1) * sms;
+    if (waves240 <= waves256 && 2 * last256 < sms)
+        return launch_cfg<NP, 240, stages_for(NP, 240), G128>(a, X, ldx, s);
     return launch_cfg<NP, BN_MAX, stages_for(NP, BN_MAX), G128>(a, X, ldx, s);
+    }
 }
 
 cudaError_t launch_gemm(const uint32_t* planes, const void* alpha, bool alpha_f16, int64_t M, int64_t K, int n_paths,

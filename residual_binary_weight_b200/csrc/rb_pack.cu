@@ -157,6 +157,10 @@ pack_words_kernel(const WT* __restrict__ W, int64_t ldw, int M, int K, int N, bo
     const int wpr = tpr >> 5;   // warps per row when tpr >= 32
     const size_t S = (static_cast<size_t>(K) + 511) / 512;
 
+    // mean = sum / K; for K a power of two the product with 1/K is the same
+    // number and avoids the fp64 division
+    const bool k_pow2 = (K & (K - 1)) == 0;
+    const double inv_k = 1.0 / static_cast<double>(K);
     float r[32];
     if (active) {
         load32(W + static_cast<int64_t>(row) * ldw + 32 * tr, r);
@@ -187,7 +191,8 @@ pack_words_kernel(const WT* __restrict__ W, int64_t ldw, int M, int K, int N, bo
         }
         // every lane of a row holds the same sum; one lane per warp divides
         float a = 0.0f;
-        if ((lane & (min(tpr, 32) - 1)) == 0) a = static_cast<float>(sum / static_cast<double>(K));
+        if ((lane & (min(tpr, 32) - 1)) == 0)
+            a = static_cast<float>(k_pow2 ? sum * inv_k : sum / static_cast<double>(K));
         a = __shfl_sync(FULL_MASK, a, lane & ~(min(tpr, 32) - 1));
         if (active && tr == 0) {
             alpha[static_cast<size_t>(k) * M + row] = a;

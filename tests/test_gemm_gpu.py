@@ -122,10 +122,11 @@ def test_prefill_full_size_sampled(matrix):
     assert nbad == 0, worst
 
 
-@pytest.mark.parametrize("T", [1, 5, 16, 17, 33, 64, 100, 129])
+@pytest.mark.parametrize("T", [1, 5, 16, 17, 33, 64, 100, 129, 241, 300, 481])
 @pytest.mark.parametrize("n_paths,group", [(2, 0), (4, 0), (4, 128), (3, 128)])
 def test_token_tile_widths(T, n_paths, group):
-    """Every token-tile width (16..256) the launcher picks from T."""
+    """Every token-tile width (16..256, and 240 when it saves a wave) the
+    launcher picks from T, with partial last token tiles."""
     rng = np.random.default_rng(T * 7 + n_paths)
     W = (rng.standard_normal((160, 512)) * 0.02).astype(np.float16)
     X = rng.standard_normal((T, 512)).astype(np.float16)
