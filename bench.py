@@ -44,6 +44,26 @@ def _peaks():
     return 6650.0, 1590.0, 1400.0, "fallback"
 
 
+def max_over_ranks(value: float, device) -> float:
+    """The largest `value` of all ranks (the job's time is its slowest rank's);
+    `device` is where the collective runs (a CUDA device under NCCL, "cpu"
+    under gloo)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(world_size: int, bytes_per_rank_step: int, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank streams its own copy of the stack
+    (replicas), so the job moves world_size x the bytes in the slowest rank's
+    time."""
+    return world_size * bytes_per_rank_step / (ms_per_step * 1e-3) / 1e9
+
+
 def _dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -341,15 +361,11 @@ def run_gpu(args):
             ev[i][1].record(stream)
         t1.record(stream)
         barrier()
-    total_ms = t0.elapsed_time(t1)
+    total_ms = max_over_ranks(t0.elapsed_time(t1), device)
     launch_ms = [a.elapsed_time(b) for a, b in ev]
     clocks = clk.summary()
-    if ws > 1:
-        t = torch.tensor([total_ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
     ms_step = total_ms / args.steps
-    value = ws * alg_bytes / (ms_step * 1e-3) / 1e9
+    value = whole_job_gbs(ws, alg_bytes, ms_step)
     kern_ms = sum(launch_ms) / len(launch_ms)
     achieved = alg_bytes / (kern_ms * 1e-3) / 1e9
 
@@ -370,12 +386,8 @@ def run_gpu(args):
         yh.copy_(ybuf, non_blocking=True)
     e1.record(stream)
     barrier()
-    e2e_ms = e0.elapsed_time(e1) / args.steps
-    if ws > 1:
-        t = torch.tensor([e2e_ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e = {"value": round(ws * alg_bytes / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, device)
+    e2e = {"value": round(whole_job_gbs(ws, alg_bytes, e2e_ms), 1), "unit": "GB/s",
            "h2d_bytes_per_step": xbuf.numel() * 2, "d2h_bytes_per_step": ybuf.numel() * 2}
 
     parts = {}
