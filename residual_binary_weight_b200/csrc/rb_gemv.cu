@@ -731,10 +731,23 @@ GvPlan gemv_plan_single(int64_t M, int64_t K, int n_paths, int group, int T, int
     const int R = gemv_rows_per_cta(n_paths, group);
     const int64_t S = (K + SLICE_COLS - 1) / SLICE_COLS;
     const int64_t nrb = (M + R - 1) / R;
-    // split K until there are at least two units per SM (or one slice per unit)
-    int64_t nch = 1;
-    while (nch < S && nrb * nch * T < 2 * num_sms) ++nch;
-    const int chunk = static_cast<int>((S + nch - 1) / nch);
+    // Choose the number of K chunks that minimises the busiest CTA's work:
+    // (units it gets) x (slices per unit + about half a slice for the
+    // partial-sum epilogue of a split unit); ties go to fewer chunks.
+    const int64_t sms = num_sms > 0 ? num_sms : 1;
+    int64_t best_nch = 1;
+    double best = -1.0;
+    for (int64_t nch = 1; nch <= S; ++nch) {
+        const int64_t units = nrb * nch * T;
+        const int64_t per_cta = (units + sms - 1) / sms;
+        const int64_t slices = (S + nch - 1) / nch;
+        const double cost = static_cast<double>(per_cta) * (static_cast<double>(slices) + (nch > 1 ? 0.5 : 0.0));
+        if (best < 0.0 || cost < best) {
+            best = cost;
+            best_nch = nch;
+        }
+    }
+    const int chunk = static_cast<int>((S + best_nch - 1) / best_nch);
     GvPlan pl{R, chunk, 0, 0, 0};
     count_job(M, K, R, chunk, T, pl);
     return pl;
