@@ -755,7 +755,12 @@ GvPlan gemv_plan_single(int64_t M, int64_t K, int n_paths, int group, int T, int
 
 GvPlan gemv_plan_grouped(const GvJob* jobs, int n, int n_paths, int group, int T) {
     const int R = gemv_rows_per_cta(n_paths, group);
-    const int chunk = 8;   // 4096 columns: wider matrices are split so units stay small
+    // up to 12 slices (6144 columns) per unit: wider matrices are split in
+    // equal parts. Each split adds a partial-sum epilogue (fp32 partials, an
+    // arrival counter, the last CTA's reduction), which costs more than the
+    // load imbalance of longer units (7B stack: 8 -> 408 us, 12 -> 402 us;
+    // 4 or 6, which split the 4096-wide matrices too: 519 and 506 us)
+    const int chunk = 12;
     GvPlan pl{R, chunk, 0, 0, 0};
     for (int i = 0; i < n; ++i) count_job(jobs[i].M, jobs[i].K, R, chunk, T, pl);
     return pl;
