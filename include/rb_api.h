@@ -146,7 +146,7 @@ RB_API size_t rb_gemv_workspace_bytes(rb_layout L, int32_t T);
 
 /* One matrix of a grouped matvec; x is [T][K] and y is [T][M], both dense. */
 typedef struct {
-    const uint32_t* planes;  /* device, [N][M][K/32] */
+    const uint32_t* planes;  /* device, rb_planes_words words in the call's order */
     const void* alpha;       /* device, [N][M][K/G] */
     const void* x;           /* device, fp16 [T][K], 16-byte aligned */
     void* y;                 /* device, [T][M] */
@@ -156,8 +156,11 @@ typedef struct {
 
 /*
  * rb_gemv_grouped -- the same operation over n independent matrices in one
- * persistent launch (a decode step through a stack of layers). Work is
- * handed out to CTAs from a counter in the workspace.
+ * persistent launch (a decode step through a stack of layers). The work
+ * units (row block, K chunk, token) of all matrices are dealt to the CTAs
+ * round robin, in descriptor order; a CTA moves from one unit to the next
+ * without draining its load pipeline, so listing the longest matrices
+ * first and keeping related matrices adjacent helps.
  *
  * descs_host  host, n descriptors, read for validation and sizing only.
  * descs_dev   device, the same n descriptors (the caller uploads them once).
@@ -207,7 +210,7 @@ RB_API rb_status rb_gemm_check(void* stream);
  * implicit device synchronisation of an allocation, a plug-in inside a host
  * framework that owns every device buffer, or a fixed-budget deployment that
  * forbids allocations after start-up. For them the scratch rb_gemv keeps in
- * the workspace (work counters and K-split partial sums) lives in one static
+ * the workspace (error word, arrival counters and K-split partial sums) lives in one static
  * 1 MiB device array per GPU, held by every GPU that loads the library until
  * the process exits. The caller still passes planes, scales, x and y, with
  * the same meaning, layout and checks as rb_gemv.

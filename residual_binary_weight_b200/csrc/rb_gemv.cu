@@ -7,14 +7,15 @@
 //     T[b][c] = sum_e (bit e of b ? +x[8c+e] : -x[8c+e])
 // (2 * masked sum - block sum, built from two 16-entry nibble tables), so a
 // plane byte b costs one PRMT (which forms the table address from the byte
-// and a per-lane base), one LDS and one FADD: 3 instructions per 8 weight
-// bits instead of >= 1 per bit for a select-and-add.
+// and a per-lane base), one LDS and half of a packed fp32x2 add: about 2.5
+// instructions per 8 weight bits instead of >= 1 per bit for a select-and-add.
 //
 // Table layout: 256 rows of 64 fp32 entries (one 512-column slice of x),
 // 64 KB, at shared-window address 0x10000 (a second one, for double
 // buffering, at 0x20000). With the table 64 KB aligned the address of entry
-// (b, c) is 0x10000 | b << 8 | 4c: PRMT takes byte 0 (4c) and bytes 2-3 from
-// the lane's base register and byte 1 from the plane word.
+// (b, c) is 0x10000 | b << 8 | 4c: PRMT takes byte 1 from the plane word,
+// byte 0 (4c) from byte 0 or 1 of a base register that holds the columns of
+// two lookup steps, and bytes 2-3 (the table page) from the same register.
 //
 // Work split. A CTA (32 warps) owns R rows of one matrix for a K chunk and
 // walks its 512-column slices. An item (row, path) of a slice is 16 plane
@@ -27,6 +28,12 @@
 // of every LDS on 32 distinct banks. Partial sums stay in registers across
 // the slices of the chunk and are reduced over the 8 lanes of each item at
 // the end.
+//
+// Scheduling. Units (row block, K chunk, token) are dealt to CTAs round robin
+// and decoded once into shared memory, so each CTA knows its whole sequence
+// of (unit, slice) steps: the last step of a unit already loads the next
+// unit's first plane words, builds its first table and stages its x, and the
+// unit's epilogue overlaps those loads.
 //
 // Per-row scales are applied once per row at the end; per-128-column scales
 // (the QBB layout) multiply each word's partial sum as it is accumulated.
