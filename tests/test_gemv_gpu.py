@@ -139,7 +139,7 @@ def _grouped_case(wl_name, layer, scale_rows, T, n_paths, group, alpha_f16, orde
 def test_grouped_llama2_layer(T, order):
     items, refs = _grouped_case("llama2_7b_decode", 2, 8, T, 2, 0, False, order)
     g = rb.GroupedGemv(items, n_paths=2, group=0, T=T)
-    for _ in range(2):              # the work counter is cleared on every call
+    for _ in range(2):              # the arrival counters are cleared on every call
         for it in items:
             it[3].fill_(float("nan"))
         g.run()
@@ -154,6 +154,35 @@ def test_grouped_llama2_layer(T, order):
 def test_grouped_qbb_g128(order):
     items, refs = _grouped_case("qbb_g128", 0, 16, 1, 4, 128, True, order)
     g = rb.GroupedGemv(items, n_paths=4, group=128, T=1)
+    g.run()
+    torch.cuda.synchronize()
+    g.check_device_flag()
+    for (_, _, _, y), (y_ref, den) in zip(items, refs):
+        nbad, worst = oracle.compare_outputs(y.float().cpu().numpy(), y_ref, den)
+        assert nbad == 0, worst
+
+
+@pytest.mark.parametrize("order", ORDERS)
+def test_grouped_many_units_per_cta(order):
+    """1400 small matrices at T = 16 give ~150 units to each CTA, more than the
+    128 unit records a CTA holds at once, so the records are refilled while
+    the CTA runs (and some units are K-split)."""
+    rng = np.random.default_rng(23)
+    items, refs = [], []
+    T = 16
+    for i in range(1400):
+        M = int(rng.integers(1, 70))
+        K = int(rng.choice([128, 256, 640, 6656]) if i % 50 == 0 else rng.choice([128, 256, 640]))
+        W = (rng.standard_normal((M, K)) * 0.02).astype(np.float16)
+        x = rng.standard_normal((T, K)).astype(np.float16)
+        ref_p, ref_a, _ = oracle.pack(W, 2, 0)
+        a32 = ref_a.astype(np.float32)
+        y_ref, den = oracle.matvec(ref_p, a32.astype(np.float64), x.astype(np.float64))
+        y = torch.full((T, M), float("nan"), dtype=torch.float16, device="cuda")
+        items.append((to_dev_planes(ref_p, order=order), torch.from_numpy(a32).cuda(),
+                      torch.from_numpy(x).cuda(), y))
+        refs.append((y_ref, den))
+    g = rb.GroupedGemv(items, n_paths=2, group=0, T=T)
     g.run()
     torch.cuda.synchronize()
     g.check_device_flag()
