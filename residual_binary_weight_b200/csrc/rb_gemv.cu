@@ -139,12 +139,6 @@ __device__ __forceinline__ uint2 ldg_words2(const void* p) {
     return v;
 }
 
-__device__ __forceinline__ uint32_t ldg_word(const void* p) {
-    uint32_t v;
-    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
-    return v;
-}
-
 template <bool B>
 struct BoolC { static constexpr bool value = B; };
 

@@ -59,9 +59,11 @@ def test_path_counts(n_paths, group):
 
 
 @pytest.mark.parametrize("order", ["rows", "sliced"])
-@pytest.mark.parametrize("K", [128, 384, 1152])
+@pytest.mark.parametrize("K", [128, 384, 1152, 33280])
 @pytest.mark.parametrize("group", [0, 128])
 def test_ragged_and_minimum_shapes(K, group, order):
+    """Small and ragged K, and K = 33280 (> 32768), which takes the
+    one-CTA-per-row kernel instead of the word-per-thread one."""
     rng = np.random.default_rng(K)
     W = (rng.standard_normal((3, K)) * 0.05).astype(np.float32)
     _ok(check_pack(W, 2, group, order=order), (K, group))
