@@ -113,6 +113,27 @@ __device__ __forceinline__ void umma_commit(uint32_t bar) {
                  : "memory");
 }
 
+// D (+)= A x B with the A operand (128 rows x 16 fp16 columns) read from
+// tensor memory at a_tmem instead of shared memory
+__device__ __forceinline__ void umma_f16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+// 32 lanes x 16 columns of 32 bits into tensor memory (this warp's lane quarter)
+__device__ __forceinline__ void tmem_store16(uint32_t taddr, const uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};"
+        ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+          "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+        : "memory");
+}
+
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
@@ -197,26 +218,35 @@ struct GemmArgs {
     bool y_f16;
 };
 
-template <int NP, int BN, int STAGES, bool G128>
+// ATM: the expanded A operand goes to tensor memory (tcgen05.st) instead of
+// shared memory, so shared memory only carries the X tiles; used for token
+// tiles of at most 128, where the accumulators leave room for A stages.
+template <int NP, int BN, int STAGES, bool G128, bool ATM>
 struct GemmCfg {
     static constexpr int NACC = G128 ? 1 : NP;                         // accumulators
     // tensor-memory columns between accumulators: BN rounded up to a power of two
     static constexpr int ACC_STRIDE = BN <= 16 ? 16 : BN <= 32 ? 32 : BN <= 64 ? 64 : BN <= 128 ? 128 : 256;
     static constexpr uint32_t B_TILE_BYTES = BN * BK * 2;
-    static constexpr uint32_t STAGE_BYTES = NP * A_TILE_BYTES + B_TILE_BYTES;
+    static constexpr uint32_t STAGE_BYTES = (ATM ? 0 : NP * A_TILE_BYTES) + B_TILE_BYTES;
     static constexpr int ACC_COLS = NACC * ACC_STRIDE;
-    static constexpr uint32_t TMEM_COLS = (ACC_COLS <= 32) ? 32 : (ACC_COLS <= 64) ? 64 :
+    static constexpr int A_BASE = ACC_COLS;               // first tensor-memory column of the A stages
+    static constexpr int A_STAGE_COLS = NP * BK / 2;      // fp16 pairs of all paths of one stage
+    static constexpr uint32_t TMEM_COLS = ATM ? 512 : (ACC_COLS <= 32) ? 32 : (ACC_COLS <= 64) ? 64 :
                                           (ACC_COLS <= 128) ? 128 : (ACC_COLS <= 256) ? 256 : 512;
-    static constexpr uint32_t SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+    // with A in tensor memory the shared memory is small; ask for enough that
+    // two CTAs never share an SM (the second would wait for tensor memory)
+    static constexpr uint32_t SMEM_USED = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+    static constexpr uint32_t SMEM_BYTES = ATM && SMEM_USED < 120u * 1024u ? 120u * 1024u : SMEM_USED;
+    static_assert(!ATM || A_BASE + STAGES * A_STAGE_COLS <= 512, "A stages exceed tensor memory");
     static_assert(ACC_COLS <= 512, "accumulators exceed tensor memory");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M = 128");
     static_assert(B_TILE_BYTES % 1024 == 0, "B tile must keep the 1024-byte swizzle alignment");
 };
 
-template <int NP, int BN, int STAGES, bool G128>
+template <int NP, int BN, int STAGES, bool G128, bool ATM>
 __global__ void __launch_bounds__(THREADS, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, GemmArgs a) {
-    using C = GemmCfg<NP, BN, STAGES, G128>;
+    using C = GemmCfg<NP, BN, STAGES, G128, ATM>;
     extern __shared__ __align__(1024) unsigned char dsm[];
     // 1024-byte aligned tile area (the 128-byte swizzle repeats every 1024 B)
     const uint32_t raw = smem_addr(dsm);
@@ -229,7 +259,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, GemmArgs a) {
     const uint32_t abort_slot = tmem_slot + 4u;
     volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(dsm + (abort_slot - raw));
     auto a_tile = [&](int s, int p) { return tiles + s * C::STAGE_BYTES + p * A_TILE_BYTES; };
-    auto b_tile = [&](int s) { return tiles + s * C::STAGE_BYTES + NP * A_TILE_BYTES; };
+    auto b_tile = [&](int s) { return tiles + s * C::STAGE_BYTES + (ATM ? 0u : NP * A_TILE_BYTES); };
+    // tensor-memory column of stage s, path p of the A operand (ATM)
+    auto a_col = [&](int s, int p) { return static_cast<uint32_t>(C::A_BASE + (s * NP + p) * (BK / 2)); };
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int row_tile = blockIdx.x, tok_tile = blockIdx.y;
@@ -282,10 +314,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, GemmArgs a) {
                     const uint32_t d = tmem_base + static_cast<uint32_t>(G128 ? 0 : p * C::ACC_STRIDE);
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk) {
-                        const uint64_t ad = smem_desc(a_tile(s, p) + 32u * kk);
                         const uint64_t bd = smem_desc(b_tile(s) + 32u * kk);
                         const uint32_t acc = (kb > 0 || kk > 0 || (G128 && p > 0)) ? 1u : 0u;
-                        umma_f16(d, ad, bd, idesc, acc);
+                        if (ATM) {
+                            umma_f16_ta(d, tmem_base + a_col(s, p) + 8u * kk, bd, idesc, acc);
+                        } else {
+                            const uint64_t ad = smem_desc(a_tile(s, p) + 32u * kk);
+                            umma_f16(d, ad, bd, idesc, acc);
+                        }
                     }
                 }
                 umma_commit(empty_bar(s));      // stage s is free once these MMAs completed
@@ -317,36 +353,77 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, GemmArgs a) {
         };
         const uint32_t rsw = static_cast<uint32_t>(r & 7);
         const uint32_t row_off = static_cast<uint32_t>(r >> 3) * 1024u + rsw * 128u;
-        uint2 nxt[NP];
+        const uint32_t lane_addr_q = static_cast<uint32_t>((warp - EXP_WARP0) * 32) << 16;   // this warp's lanes
+        // The words (and group scales) of stage kb are loaded PD stages ahead
+        // into a register ring, so a stage never waits for global memory even
+        // when the tensor-core work per stage is short (few tokens).
+        constexpr int PD = 16 / NP;
+        uint2 ring[PD][NP];
+        uint32_t aring[PD][NP];
 #pragma unroll
-        for (int p = 0; p < NP; ++p) nxt[p] = words_at(p, 0);
-        for (int kb = 0; kb < nk; ++kb) {
-            const int s = kb % STAGES;
-            const uint32_t ph = static_cast<uint32_t>(kb / STAGES) & 1u;
-            uint2 cur[NP];
+        for (int i = 0; i < PD; ++i)
 #pragma unroll
             for (int p = 0; p < NP; ++p) {
-                cur[p] = nxt[p];
-                if (kb + 1 < nk) nxt[p] = words_at(p, kb + 1);
+                if (i < nk) {
+                    ring[i][p] = words_at(p, i);
+                    aring[i][p] = alpha_h2(p, i);
+                } else {
+                    ring[i][p] = make_uint2(0u, 0u);
+                    aring[i][p] = 0u;
+                }
             }
-            if (!mbar_wait(empty_bar(s), ph ^ 1u, abort_flag, 4u)) break;
+        bool go = true;
+        for (int kb0 = 0; kb0 < nk && go; kb0 += PD) {
 #pragma unroll
-            for (int p = 0; p < NP; ++p) {
-                const uint32_t v2 = alpha_h2(p, kb);
-                const uint32_t base = a_tile(s, p) + row_off;
+            for (int i = 0; i < PD; ++i) {
+                const int kb = kb0 + i;
+                if (kb < nk && go) {
+                    const int s = kb % STAGES;
+                    const uint32_t ph = static_cast<uint32_t>(kb / STAGES) & 1u;
+                    uint2 cur[NP];
+                    uint32_t v2[NP];
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t h[16];
-                    expand_word(half ? cur[p].y : cur[p].x, v2, h);
+                    for (int p = 0; p < NP; ++p) {
+                        cur[p] = ring[i][p];
+                        v2[p] = aring[i][p];
+                        if (kb + PD < nk) {
+                            ring[i][p] = words_at(p, kb + PD);
+                            aring[i][p] = alpha_h2(p, kb + PD);
+                        }
+                    }
+                    if (!mbar_wait(empty_bar(s), ph ^ 1u, abort_flag, 4u)) {
+                        go = false;
+                    } else {
 #pragma unroll
-                    for (int c4 = 0; c4 < 4; ++c4) {
-                        const uint32_t chunk = static_cast<uint32_t>(4 * half + c4);   // 16-byte chunk 0..7
-                        sts128(base + ((chunk ^ rsw) << 4), h[4 * c4], h[4 * c4 + 1], h[4 * c4 + 2], h[4 * c4 + 3]);
+                        for (int p = 0; p < NP; ++p) {
+                            const uint32_t base = a_tile(s, p) + row_off;
+#pragma unroll
+                            for (int half = 0; half < 2; ++half) {
+                                uint32_t h[16];
+                                expand_word(half ? cur[p].y : cur[p].x, v2[p], h);
+                                if (ATM) {
+                                    // row r is tensor-memory lane r; column j holds K-columns 2j, 2j+1
+                                    tmem_store16(tmem_base + lane_addr_q + a_col(s, p) + 16u * half, h);
+                                } else {
+#pragma unroll
+                                    for (int c4 = 0; c4 < 4; ++c4) {
+                                        const uint32_t chunk = static_cast<uint32_t>(4 * half + c4);   // 16-byte chunk
+                                        sts128(base + ((chunk ^ rsw) << 4), h[4 * c4], h[4 * c4 + 1], h[4 * c4 + 2],
+                                               h[4 * c4 + 3]);
+                                    }
+                                }
+                            }
+                        }
+                        if (ATM) {
+                            asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");   // stores done first
+                            tc_fence_before();
+                        } else {
+                            fence_proxy_async_smem();   // make the generic-proxy stores visible to the tensor core
+                        }
+                        mbar_arrive(full_bar(s));
                     }
                 }
             }
-            fence_proxy_async_smem();          // make the generic-proxy stores visible to the tensor core
-            mbar_arrive(full_bar(s));
         }
 
         // ------------------------------------------------------------ epilogue
@@ -419,9 +496,9 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-template <int NP, int BN, int STAGES, bool G128>
+template <int NP, int BN, int STAGES, bool G128, bool ATM = false>
 cudaError_t launch_cfg(const GemmArgs& a, const void* X, int64_t ldx, cudaStream_t s) {
-    using C = GemmCfg<NP, BN, STAGES, G128>;
+    using C = GemmCfg<NP, BN, STAGES, G128, ATM>;
     EncodeTiledFn enc = encode_fn();
     if (!enc) return cudaErrorNotSupported;
     CUtensorMap map;
@@ -433,7 +510,7 @@ cudaError_t launch_cfg(const GemmArgs& a, const void* X, int64_t ldx, cudaStream
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
-    auto kern = gemm_tc_kernel<NP, BN, STAGES, G128>;
+    auto kern = gemm_tc_kernel<NP, BN, STAGES, G128, ATM>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     dim3 grid(static_cast<unsigned>((a.M + BM - 1) / BM), static_cast<unsigned>((a.T + BN - 1) / BN));
@@ -452,6 +529,23 @@ constexpr int stages_for(int np, int bn) {
                : 8;
 }
 
+// stages of the A operand that fit in tensor memory beside the accumulators
+// of a token tile (0: fewer than two, use shared memory for A)
+constexpr int atm_stages(int np, int bn, bool g128) {
+    const int nacc = g128 ? 1 : np;
+    const int stride = bn <= 16 ? 16 : bn <= 32 ? 32 : bn <= 64 ? 64 : bn <= 128 ? 128 : 256;
+    const int st = (512 - nacc * stride) / (np * BK / 2);
+    return st >= 2 ? (st < 8 ? st : 8) : 0;
+}
+
+// token tiles up to 128: A in tensor memory when it fits
+template <int NP, int BN, bool G128>
+cudaError_t launch_narrow(const GemmArgs& a, const void* X, int64_t ldx, cudaStream_t s) {
+    constexpr int SA = atm_stages(NP, BN, G128);
+    if constexpr (SA >= 2) return launch_cfg<NP, BN, SA, G128, true>(a, X, ldx, s);
+    else return launch_cfg<NP, BN, stages_for(NP, BN), G128>(a, X, ldx, s);
+}
+
 template <int NP, bool G128>
 cudaError_t launch_np(const GemmArgs& a, const void* X, int64_t ldx, cudaStream_t s) {
     // token tile: the narrowest of 16..256 that covers T (MMA N), so small
@@ -459,13 +553,13 @@ cudaError_t launch_np(const GemmArgs& a, const void* X, int64_t ldx, cudaStream_
     // 512 tensor-memory columns
     constexpr int BN_MAX = G128 ? 256 : (NP <= 2 ? 256 : 128);
     const int T = a.T;
-    if (T <= 16) return launch_cfg<NP, 16, stages_for(NP, 16), G128>(a, X, ldx, s);
-    if (T <= 32) return launch_cfg<NP, 32, stages_for(NP, 32), G128>(a, X, ldx, s);
-    if (T <= 64) return launch_cfg<NP, 64, stages_for(NP, 64), G128>(a, X, ldx, s);
+    if (T <= 16) return launch_narrow<NP, 16, G128>(a, X, ldx, s);
+    if (T <= 32) return launch_narrow<NP, 32, G128>(a, X, ldx, s);
+    if (T <= 64) return launch_narrow<NP, 64, G128>(a, X, ldx, s);
     if constexpr (BN_MAX == 128) {
-        return launch_cfg<NP, 128, stages_for(NP, 128), G128>(a, X, ldx, s);
+        return launch_narrow<NP, 128, G128>(a, X, ldx, s);
     } else {
-    if (T <= 128) return launch_cfg<NP, 128, stages_for(NP, 128), G128>(a, X, ldx, s);
+    if (T <= 128) return launch_narrow<NP, 128, G128>(a, X, ldx, s);
     // Wide token tiles: 240 instead of 256 when the last wave of 256-wide
     // tiles would leave most SMs idle and 240 needs no extra wave: e.g. 112
     // row tiles x 2048 tokens are 896 tiles of 256 (6 full waves on 148 SMs
