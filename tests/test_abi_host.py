@@ -142,3 +142,11 @@ def test_workspace_sizes_follow_the_split():
     assert small > 256 + 4 * 512
     # a layout that is rejected needs nothing
     assert lib.rb_gemv_workspace_bytes(Layout(512, 8000, 2, 0, 0, 0), 1) == 0
+
+
+def test_missing_library_fails_loudly(monkeypatch):
+    """Without librb.so the binding raises; there is no fallback path."""
+    monkeypatch.setattr(_lib, "_lib", None)
+    monkeypatch.setattr(_lib, "LIB_PATH", "/nonexistent/librb.so")
+    with pytest.raises(ImportError):
+        _lib.load()
