@@ -149,7 +149,9 @@ struct Log2 { static constexpr int v = J == 16 ? 4 : J == 8 ? 3 : J == 4 ? 2 : J
 // lanes per item, 2 words per lane); J such loads per lane and slice.
 template <int NP, bool G128>
 struct Cfg {
-    static constexpr int J = G128 && NP <= 4 ? 4 : 8;  // item loads per lane per slice (>= NP)
+    // item loads per lane per slice (>= NP); 8 for every layout (with group
+    // scales 4 loads per lane halved the rows per table and was ~20 % slower)
+    static constexpr int J = 8;
     static constexpr int HR = J / NP > 0 ? J / NP : 1; // row quads per path per warp
     static constexpr int RW = 4 * HR;                 // rows per warp
     static constexpr int JV = NP * HR <= J ? NP * HR : J;   // loads in use
@@ -711,8 +713,8 @@ cudaError_t launch_order(const GvArgs& a, const GvPlan& plan, cudaStream_t s) {
 
 int gemv_max_jobs() { return MAX_JOBS; }
 
-int gemv_rows_per_cta(int n_paths, int group) {
-    const int J = group && n_paths <= 4 ? 4 : 8;
+int gemv_rows_per_cta(int n_paths, int /*group*/) {
+    const int J = 8;   // Cfg::J
     const int hr = J / n_paths > 0 ? J / n_paths : 1;
     return WARPS * 4 * hr;
 }
