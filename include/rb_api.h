@@ -149,7 +149,9 @@ typedef struct {
     const uint32_t* planes;  /* device, rb_planes_words words in the call's order */
     const void* alpha;       /* device, [N][M][K/G] */
     const void* x;           /* device, fp16 [T][K], 16-byte aligned */
-    void* y;                 /* device, [T][M] */
+    void* y;                 /* device, [T][M]; or pinned host memory mapped for
+                                the device (its device address), which the
+                                kernel then writes over the bus */
     int64_t M;
     int64_t K;
 } rb_gemv_desc;

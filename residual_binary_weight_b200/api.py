@@ -64,6 +64,24 @@ def _require_cuda(*ts: torch.Tensor) -> torch.device:
     return dev
 
 
+def _mapped_host_ptr(t: torch.Tensor) -> int:
+    """Device address of a pinned host tensor (the kernel writes it over the
+    bus). Page-locked host memory is mapped into the device address space
+    under unified addressing; the runtime is asked for the address rather
+    than assuming it."""
+    if t.is_cuda or not t.is_pinned():
+        raise ValueError("expected a pinned host tensor")
+    try:
+        from cuda.bindings import runtime as rt
+    except ImportError as e:   # pragma: no cover - cuda-python is part of the image
+        raise ValueError("a pinned host output needs cuda-python (cuda.bindings)") from e
+    base = t.untyped_storage().data_ptr()          # the allocation the runtime knows
+    err, dptr = rt.cudaHostGetDevicePointer(base, 0)
+    if int(err) != 0 or not dptr:
+        raise ValueError(f"pinned host tensor is not mapped for the device (cudaHostGetDevicePointer: {err})")
+    return int(dptr) + (t.data_ptr() - base)
+
+
 def pack(W: torch.Tensor, n_paths: int = 2, group: int = 0, alpha_f16: bool = False, order: str = "rows"):
     """Derive N residual sign planes and scales from the shared weight W (M x K).
 
@@ -128,6 +146,9 @@ class GroupedGemv:
 
     The descriptor table is uploaded once at construction; call ``run()`` for
     every step (the x tensors are read and the y tensors written in place).
+    A y tensor may also be a pinned host tensor: the kernel then writes its
+    rows straight into host memory over the bus, so the result needs no
+    separate device-to-host copy.
     """
 
     def __init__(self, items: Sequence[tuple], n_paths: int, group: int = 0, T: int = 1):
@@ -139,7 +160,7 @@ class GroupedGemv:
         adt = ydt = order = None
         dev = None
         for i, (planes, alpha, x, y) in enumerate(self.items):
-            dev = _require_cuda(planes, alpha, x, y)
+            dev = _require_cuda(planes, alpha, x, None if (not y.is_cuda and y.is_pinned()) else y)
             K = x.shape[-1]
             N, M, o = _planes_geometry(planes, K)
             order = o if order is None else order
@@ -151,7 +172,8 @@ class GroupedGemv:
             ydt = y.dtype if ydt is None else ydt
             if alpha.dtype != adt or y.dtype != ydt:
                 raise ValueError("all items must share the scale and output dtypes")
-            self.host[i] = GemvDesc(planes.data_ptr(), alpha.data_ptr(), x.data_ptr(), y.data_ptr(), M, K)
+            y_ptr = y.data_ptr() if y.is_cuda else _mapped_host_ptr(y)
+            self.host[i] = GemvDesc(planes.data_ptr(), alpha.data_ptr(), x.data_ptr(), y_ptr, M, K)
         self.device = dev
         raw = bytes(self.host)
         self.dev_descs = torch.frombuffer(bytearray(raw), dtype=torch.uint8).to(dev)

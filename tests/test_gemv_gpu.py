@@ -162,6 +162,25 @@ def test_grouped_qbb_g128(order):
         assert nbad == 0, worst
 
 
+def test_grouped_output_in_pinned_host_memory():
+    """y given as pinned host tensors: the launch writes the rows over the bus
+    and they equal the oracle's (and the device-y run's)."""
+    items, refs = _grouped_case("llama2_7b_decode", 1, 16, 1, 2, 0, False, "sliced")
+    host_items = [(p, a, x, torch.empty(y.shape, dtype=y.dtype, pin_memory=True).fill_(float("nan")))
+                  for p, a, x, y in items]
+    g = rb.GroupedGemv(host_items, n_paths=2, group=0, T=1)
+    g.run()
+    torch.cuda.synchronize()
+    g.check_device_flag()
+    gd = rb.GroupedGemv(items, n_paths=2, group=0, T=1)
+    gd.run()
+    torch.cuda.synchronize()
+    for (_, _, _, yh), (_, _, _, yd), (y_ref, den) in zip(host_items, items, refs):
+        assert torch.equal(yh, yd.cpu())
+        nbad, worst = oracle.compare_outputs(yh.float().numpy(), y_ref, den)
+        assert nbad == 0, worst
+
+
 @pytest.mark.parametrize("order", ORDERS)
 def test_grouped_many_units_per_cta(order):
     """1400 small matrices at T = 16 give ~150 units to each CTA, more than the
