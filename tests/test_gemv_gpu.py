@@ -183,13 +183,14 @@ def test_grouped_output_in_pinned_host_memory():
 
 @pytest.mark.parametrize("order", ORDERS)
 def test_grouped_many_units_per_cta(order):
-    """1400 small matrices at T = 16 give ~150 units to each CTA, more than the
-    128 unit records a CTA holds at once, so the records are refilled while
-    the CTA runs (and some units are K-split)."""
+    """The largest grouped launch (2047 descriptors) of small matrices at
+    T = 16: ~220 units per CTA, more than the 128 unit records a CTA holds at
+    once, so the records are refilled while the CTA runs (and some units are
+    K-split)."""
     rng = np.random.default_rng(23)
     items, refs = [], []
     T = 16
-    for i in range(1400):
+    for i in range(2047):
         M = int(rng.integers(1, 70))
         K = int(rng.choice([128, 256, 640, 6656]) if i % 50 == 0 else rng.choice([128, 256, 640]))
         W = (rng.standard_normal((M, K)) * 0.02).astype(np.float16)
