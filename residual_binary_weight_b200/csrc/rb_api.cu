@@ -291,7 +291,10 @@ rb_status rb_gemv_check(const void* workspace, void* stream) {
                                     cudaMemcpyDeviceToHost, s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) return cuda_fail(e, "rb_gemv_check");
-    if (flag) return fail(RB_ERR_DEVICE, "matvec kernel flag 0x%x", flag);
+    if (flag)
+        return fail(RB_ERR_DEVICE, "matvec kernel flag 0x%x (%s%s)", flag,
+                    (flag & GV_ERR_SMEM_LAYOUT) ? "shared-memory window not where the tables need it " : "",
+                    (flag & GV_ERR_TOO_MANY_JOBS) ? "more descriptors than a launch takes" : "");
     return RB_OK;
 }
 
