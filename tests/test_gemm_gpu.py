@@ -79,6 +79,9 @@ def test_dtypes_and_pitches():
     X = rng.standard_normal((96, 768)).astype(np.float16)
     _ok(_run(W, X, 2, 0, False, y_dtype=torch.float32, ldx_pad=8, ldy_pad=3), "f32 out, pitches")
     _ok(_run(W, X, 4, 128, True, "sliced", ldx_pad=16, ldy_pad=1), "g128 pitches")
+    # 300 tokens: 240-wide token tiles (A in shared memory), partial last tile
+    X3 = rng.standard_normal((300, 768)).astype(np.float16)
+    _ok(_run(W, X3, 2, 0, False, "sliced", ldx_pad=8, ldy_pad=5), "240-wide tiles, pitches")
 
 
 def test_qbb_batch16():

@@ -77,6 +77,10 @@ def test_row_pitch_and_fp32_groups():
     _ok(check_pack(W, 2, 128, ldw_pad=4), "fp32 g128 padded")
     W16 = W.astype(np.float16)
     _ok(check_pack(W16, 2, 0, ldw_pad=8), "fp16 row padded")
+    # several rows per CTA in the word-per-thread kernel, with a row pitch
+    Wl = (rng.standard_normal((37, 4096)) * 0.02).astype(np.float32)
+    _ok(check_pack(Wl.astype(np.float16), 2, 0, ldw_pad=24, order="sliced"), "fp16 4096 padded")
+    _ok(check_pack(Wl, 3, 0, ldw_pad=4), "fp32 4096 padded")
 
 
 def test_zeros_negative_zeros_and_ties():
