@@ -316,3 +316,138 @@ def test_compare_helpers_catch_plausible_mistakes():
     y_flip, _ = oracle.matvec(planes[::-1].copy(), alpha, x)
     assert oracle.compare_outputs(y_flip, y, den)[0] > 0
     assert oracle.compare_scales_f16(oracle.alpha_to_f16(alpha), alpha) == 0
+
+
+def _runs_row(vals):
+    """A 32-column row of four runs of 8 equal values."""
+    return np.repeat(np.array(vals, dtype=np.float64), 8)
+
+
+def test_rabs_is_the_magnitude_each_sign_was_taken_on():
+    """rabs[k] = |R_{k-1}|, against hand values for rows C and D
+    (tests/golden/residual_magnitudes.txt): recording it after the update
+    (|R_k|) or only for the first path fails here."""
+    rows = {name: vals for name, vals, *_ in _golden_lines("worked_examples.txt")}
+    expected = {}
+    for name, k, runs in _golden_lines("residual_magnitudes.txt"):
+        expected.setdefault(name, {})[int(k)] = _runs_row([float(v) for v in runs.split(",")])
+    assert set(expected) == {"C", "D"}
+    for name, per_path in expected.items():
+        w = np.array([float(v) for v in rows[name].split(",")])
+        planes, alpha, rabs = oracle.pack(w[None, :], 3, 0, want_rabs=True)
+        for k, want in per_path.items():
+            assert np.array_equal(rabs[k - 1, 0], want), (name, k, rabs[k - 1, 0])
+
+
+def _allowance_case():
+    """1024 x 1024 weights (1,048,576 entries, so the count bound admits one
+    flipped entry and not two), 3 paths, scale groups of 32 columns. Row 0
+    group 0 is worked example D (exact ties at path 2), row 1 group 0 is
+    example C (exact ties at path 3), row 2 group 0 holds 31 ones and one
+    entry of 5e-7 (below 1e-6 * alpha1 = 9.7e-7), row 3 group 0 the same
+    with 2e-6 (above it)."""
+    rng = np.random.default_rng(31)
+    W = rng.standard_normal((1024, 1024))
+    rows = {name: vals for name, vals, *_ in _golden_lines("worked_examples.txt")}
+    W[0, :32] = [float(v) for v in rows["D"].split(",")]
+    W[1, :32] = [float(v) for v in rows["C"].split(",")]
+    W[2, :32] = 1.0
+    W[2, 5] = 5e-7
+    W[3, :32] = 1.0
+    W[3, 5] = 2e-6
+    planes, alpha, rabs = oracle.pack(W, 3, 32, want_rabs=True)
+    return planes, alpha, rabs
+
+
+def _flip(p, k, i, j):
+    p[k, i, j // 32] ^= np.uint32(1 << (j % 32))
+
+
+def test_compare_planes_allowance_cascade_and_count_bound():
+    """The lenient branches of the plane comparison, each with a case a
+    plausible mistake would get wrong: an allowed flip is counted once even
+    when later planes of the entry follow it (taking the last differing path
+    instead of the first rejects it); a later-plane difference with no allowed
+    flip before it fails; the threshold |R| <= 1e-6 * alpha is applied in the
+    right direction; two flipped entries exceed the count bound."""
+    ref, alpha, rabs = _allowance_case()
+    assert alpha[1, 0, 0] == 0.5 and rabs[1, 0, 0] == 0.0 and rabs[2, 0, 0] == 0.5
+    rep = oracle.compare_planes(ref.copy(), ref, rabs, alpha)
+    assert (rep.flipped, rep.bad, rep.ok) == (0, 0, True)
+
+    # D: the tie at path 2 flips, and path 3 follows it (the cascade)
+    c = ref.copy()
+    _flip(c, 1, 0, 3)
+    _flip(c, 2, 0, 3)
+    rep = oracle.compare_planes(c, ref, rabs, alpha)
+    assert (rep.flipped, rep.bad, rep.ok) == (1, 0, True), rep
+
+    # path 3 alone differs where |R_2| = 0.5: no earlier allowed flip, so it fails
+    c = ref.copy()
+    _flip(c, 2, 0, 3)
+    rep = oracle.compare_planes(c, ref, rabs, alpha)
+    assert (rep.flipped, rep.bad, rep.ok) == (0, 1, False), rep
+
+    # the threshold: 5e-7 <= 1e-6 * alpha1 is allowed, 2e-6 is not
+    a1 = alpha[0, 2, 0]
+    assert 5e-7 <= 1e-6 * a1 < 2e-6
+    c = ref.copy()
+    _flip(c, 0, 2, 5)
+    rep = oracle.compare_planes(c, ref, rabs, alpha)
+    assert (rep.flipped, rep.bad, rep.ok) == (1, 0, True), rep
+    c = ref.copy()
+    _flip(c, 0, 3, 5)
+    rep = oracle.compare_planes(c, ref, rabs, alpha)
+    assert (rep.flipped, rep.bad, rep.ok) == (0, 1, False), rep
+
+    # two allowed entries (D at path 2, C's exact tie at path 3 col 10):
+    # 2 >= 1e-6 * 1,048,576, so the count bound fails
+    c = ref.copy()
+    _flip(c, 1, 0, 3)
+    _flip(c, 2, 1, 10)
+    rep = oracle.compare_planes(c, ref, rabs, alpha)
+    assert (rep.flipped, rep.bad, rep.ok) == (2, 0, False), rep
+
+    # a flip at an entry far from zero (D col 8 at path 1: |R_0| = 1)
+    c = ref.copy()
+    _flip(c, 0, 0, 8)
+    rep = oracle.compare_planes(c, ref, rabs, alpha)
+    assert rep.bad == 1 and not rep.ok
+
+
+def test_compare_scales_f16_midpoint_branch():
+    """Near an fp16 rounding midpoint either neighbour is accepted, elsewhere
+    only the round-to-nearest-even value: 1 + 2^-11 lies half way between
+    0x3C00 and 0x3C01."""
+    def f16(bits):
+        return np.array([bits], dtype=np.uint16).view(np.float16)
+
+    mid = np.array([1.0 + 2.0 ** -11])
+    assert oracle.compare_scales_f16(f16(0x3C00), mid) == 0
+    assert oracle.compare_scales_f16(f16(0x3C01), mid) == 0
+    for bad in (0x3C02, 0x3BFF, 0x0000):
+        assert oracle.compare_scales_f16(f16(bad), mid) == 1, hex(bad)
+    # within 1e-6 relative of the midpoint: still either neighbour
+    near = mid * (1 + 5e-7)
+    assert oracle.compare_scales_f16(f16(0x3C00), near) == 0
+    assert oracle.compare_scales_f16(f16(0x3C01), near) == 0
+    # 3e-6 above it: only the nearest value, 0x3C01
+    above = mid * (1 + 3e-6)
+    assert oracle.compare_scales_f16(f16(0x3C01), above) == 0
+    assert oracle.compare_scales_f16(f16(0x3C00), above) == 1
+    below = mid * (1 - 3e-6)
+    assert oracle.compare_scales_f16(f16(0x3C00), below) == 0
+    assert oracle.compare_scales_f16(f16(0x3C01), below) == 1
+
+
+def test_alpha_to_f16_bit_patterns():
+    """The stored fp16 scale copy, against hand-written IEEE half patterns:
+    1/3 -> 0x3555, 0.1 -> 0x2E66, the largest finite half 0x7BFF, the
+    smallest subnormal 0x0001, ties to even at 1 + 2^-11 (-> 0x3C00) and
+    1 + 3 * 2^-11 (-> 0x3C02), and 1 + 2^-11 + 2^-40, just above the
+    midpoint (-> 0x3C01; rounding through fp32 first would give 0x3C00)."""
+    vals = np.array([1 / 3, 0.1, 65504.0, 2.0 ** -24, 1 + 2.0 ** -11, 1 + 3 * 2.0 ** -11,
+                     1 + 2.0 ** -11 + 2.0 ** -40])
+    want = [0x3555, 0x2E66, 0x7BFF, 0x0001, 0x3C00, 0x3C02, 0x3C01]
+    got = oracle.alpha_to_f16(vals).view(np.uint16).tolist()
+    assert got == want, [hex(g) for g in got]
