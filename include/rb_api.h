@@ -164,8 +164,13 @@ typedef struct {
  * without draining its load pipeline, so listing the longest matrices
  * first and keeping related matrices adjacent helps.
  *
- * descs_host  host, n descriptors, read for validation and sizing only.
+ * descs_host  host, n descriptors, read for validation and sizing only:
+ *             every descriptor's planes and x must be 16-byte aligned, its
+ *             alpha and y aligned for their dtypes.
  * descs_dev   device, the same n descriptors (the caller uploads them once).
+ *             A device copy that gives another work plan than the host copy
+ *             is detected by the kernel, which then does nothing and records
+ *             a flag for rb_gemv_check().
  * n           1..2047.  n_paths, group, order (an rb_order), alpha_dtype,
  *             y_dtype: shared by all.
  * T           tokens, 1..64.
@@ -180,29 +185,46 @@ RB_API size_t rb_gemv_grouped_workspace_bytes(const rb_gemv_desc* descs_host, in
                                        int32_t n_paths, int32_t T);
 
 /*
- * rb_gemm -- Y_t = sum_k alpha_k (.) (B_k X_t) for a prefill block of T
- * tokens on the tcgen05 tensor cores. The plane bits are expanded exactly to
- * fp16 +-1 (one scale per row: one fp32 accumulator per path in tensor
- * memory, scaled by alpha_k in the epilogue) or to +-alpha_k in fp16 (one
- * scale per 128 columns; alpha is then read as fp16, exact when alpha_dtype
- * is RB_F16), multiplied with fp16 X and accumulated in fp32.
+ * rb_gemm -- Y_t = sum_k alpha_k (.) (B_k X_t) for a block of T tokens on the
+ * tcgen05 tensor cores (RaBiT section 4.1: binary cores with per-channel
+ * scales; QBB W(4x1)A16g128 for one scale per 128 columns). The plane bits
+ * are expanded exactly to fp16 +-1 (one scale per row: one fp32 accumulator
+ * per path in tensor memory, scaled by alpha_k at the end) or to +-alpha_k in
+ * fp16 (one scale per 128 columns), multiplied with fp16 X, accumulated in
+ * fp32. Two kernels: decode batches (T <= 64) run on a persistent grid that
+ * splits the rows x K work evenly over the SMs; prefill blocks (T > 64) run
+ * one 128-row x up-to-256-token tile per CTA.
  *
  * planes    device, rb_planes_words(L) words in L.order; 16-byte aligned.
- * alpha     device, rb_scales_count(L) scales of type alpha_dtype.
+ * alpha     device, rb_scales_count(L) scales of type alpha_dtype. With
+ *           group = 128 the scales must be RB_F16 (they become operand
+ *           values, which is exact only for fp16); RB_F32 group scales are
+ *           refused with RB_ERR_UNSUPPORTED.
  * X         device, fp16 [T][ldx], ldx >= K, base and row pitch 16-byte aligned.
  * Y         device, out, [T][ldy] of type y_dtype, ldy >= M.
- * L         1..4 paths.  T >= 1.
- * Errors: validation as rb_gemv; RB_ERR_CUDA if the tensor-map encoder or the
- *         launch fails. A kernel whose pipeline waits ran out records a code
- *         that rb_gemm_check() reports.
+ * L         1..4 paths.  T in 1..2^22.
+ * workspace device scratch of at least rb_gemm_workspace_bytes(L, T) bytes,
+ *           16-byte aligned, owned by the caller: a 256-byte header (word 1
+ *           is the call's device error word) and, for T <= 64, arrival
+ *           counters, fp32 partial sums and a column-permuted copy of X.
+ *           The call clears what must start at zero (a memset on `stream`);
+ *           calls that may overlap on the GPU need separate workspaces.
+ * Errors: validation as rb_gemv (RB_ERR_WORKSPACE if the workspace is too
+ *         small); RB_ERR_CUDA if the tensor-map encoder or a launch fails. A
+ *         kernel whose bounded pipeline waits ran out records a code in the
+ *         workspace header; rb_gemm_check() reports it.
  */
 RB_API rb_status rb_gemm(const uint32_t* planes, const void* alpha, rb_dtype alpha_dtype, rb_layout L,
                          const void* X, int64_t ldx, int32_t T, void* Y, rb_dtype y_dtype, int64_t ldy,
-                         void* stream);
+                         void* workspace, size_t ws_bytes, void* stream);
 
-/* rb_gemm_check -- wait for `stream`, then report RB_ERR_DEVICE (and clear
- * the record) if an rb_gemm kernel recorded a failure, else RB_OK. */
-RB_API rb_status rb_gemm_check(void* stream);
+/* Workspace bytes rb_gemm needs for layout L and T tokens on the current
+ * device (0 for an invalid layout or T < 1). */
+RB_API size_t rb_gemm_workspace_bytes(rb_layout L, int32_t T);
+
+/* rb_gemm_check -- wait for `stream`, then report RB_ERR_DEVICE if the
+ * rb_gemm call that used `workspace` recorded a failure, else RB_OK. */
+RB_API rb_status rb_gemm_check(const void* workspace, void* stream);
 
 /*
  * rb_gemv_noalloc -- rb_gemv for callers that cannot allocate device memory.
@@ -227,6 +249,8 @@ RB_API rb_status rb_gemm_check(void* stream);
  *   on the GPU -- on different streams of one device -- race on the array and
  *   must be ordered by the caller.
  * - Nothing here calls cudaMalloc, cudaFree or any allocating routine.
+ * - A kernel-side failure is recorded in the array's header like rb_gemv's;
+ *   rb_gemv_check(NULL, stream) reports it.
  */
 RB_API rb_status rb_gemv_noalloc(const uint32_t* planes, const void* alpha, rb_dtype alpha_dtype,
                                  rb_layout L, const void* x, int64_t ldx, int32_t T,
@@ -234,7 +258,9 @@ RB_API rb_status rb_gemv_noalloc(const uint32_t* planes, const void* alpha, rb_d
 
 /*
  * rb_gemv_check -- wait for `stream`, then report RB_ERR_DEVICE if a matvec
- * kernel that used `workspace` recorded a failure, else RB_OK.
+ * kernel that used `workspace` recorded a failure, else RB_OK. With
+ * workspace = NULL it reads the error word of rb_gemv_noalloc's static
+ * scratch on the current device (the last noalloc call there).
  */
 RB_API rb_status rb_gemv_check(const void* workspace, void* stream);
 

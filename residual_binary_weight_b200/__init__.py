@@ -9,12 +9,13 @@ library's CUDA kernels.
 
     planes, alpha, alpha16 = pack(W, n_paths=2, group=0)
     y = gemv(planes, alpha, x, group=0)               # decode, T <= 64 tokens
-    Y = gemm(planes, alpha, X, group=0)               # prefill, tcgen05 tensor cores
+    Y = gemm(planes, alpha, X, group=0)               # any batch, tcgen05 tensor cores
 """
 from ._lib import RbError, load  # noqa: F401
 from .api import (  # noqa: F401
     GroupedGemv,
     gemm,
+    gemm_workspace_bytes,
     gemv,
     gemv_workspace_bytes,
     layout,
@@ -24,4 +25,4 @@ from .api import (  # noqa: F401
 )
 
 __all__ = ["pack", "gemv", "gemm", "GroupedGemv", "layout", "planes_words", "scales_count",
-           "gemv_workspace_bytes", "RbError", "load"]
+           "gemv_workspace_bytes", "gemm_workspace_bytes", "RbError", "load"]

@@ -23,7 +23,7 @@ RB_ROWS, RB_SLICED = 0, 1
 EXPORTED = ("rb_planes_words", "rb_scales_count", "rb_status_string", "rb_last_error",
             "rb_pack", "rb_gemv", "rb_gemv_workspace_bytes", "rb_gemv_grouped",
             "rb_gemv_grouped_workspace_bytes", "rb_gemv_check", "rb_gemv_noalloc",
-            "rb_gemm", "rb_gemm_check")
+            "rb_gemm", "rb_gemm_workspace_bytes", "rb_gemm_check")
 
 
 class RbError(RuntimeError):
@@ -81,9 +81,11 @@ def load() -> ctypes.CDLL:
         lib.rb_gemv_check.restype = st
         lib.rb_gemv_noalloc.argtypes = [vp, vp, st, Layout, vp, i64, i32, vp, st, i64, vp]
         lib.rb_gemv_noalloc.restype = st
-        lib.rb_gemm.argtypes = [vp, vp, st, Layout, vp, i64, i32, vp, st, i64, vp]
+        lib.rb_gemm.argtypes = [vp, vp, st, Layout, vp, i64, i32, vp, st, i64, vp, sz, vp]
         lib.rb_gemm.restype = st
-        lib.rb_gemm_check.argtypes = [vp]
+        lib.rb_gemm_workspace_bytes.argtypes = [Layout, i32]
+        lib.rb_gemm_workspace_bytes.restype = sz
+        lib.rb_gemm_check.argtypes = [vp, vp]
         lib.rb_gemm_check.restype = st
         _lib = lib
         return lib

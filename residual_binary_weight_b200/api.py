@@ -82,24 +82,34 @@ def _mapped_host_ptr(t: torch.Tensor) -> int:
     return int(dptr) + (t.data_ptr() - base)
 
 
-def pack(W: torch.Tensor, n_paths: int = 2, group: int = 0, alpha_f16: bool = False, order: str = "rows"):
+def pack(W: torch.Tensor, n_paths: int = 2, group: int = 0, alpha_f16: bool = False, order: str = "rows",
+         planes: Optional[torch.Tensor] = None, alpha: Optional[torch.Tensor] = None,
+         alpha16: Optional[torch.Tensor] = None):
     """Derive N residual sign planes and scales from the shared weight W (M x K).
 
     Returns (planes, alpha fp32 [N, M, K/G], alpha16 fp16 [N, M, K/G] or None).
     planes holds uint32 words in an int32 tensor: [N, M, K/32] for
     order="rows", [N, ceil(K/512), M, 16] for order="sliced" (the order the
-    matvec kernel streams fastest).
+    matvec kernel streams fastest). Output tensors of those shapes may be
+    passed in to be filled instead of allocated.
     """
     lib = _lib.load()
-    dev = _require_cuda(W)
+    dev = _require_cuda(W, planes, alpha, alpha16)
     if W.dim() != 2 or W.stride(1) != 1 or W.dtype not in _DT:
         raise ValueError("W must be a 2-D fp16/fp32 tensor with unit column stride")
     M, K = W.shape
     G = K if group == 0 else group
     shape = (n_paths, M, K // 32) if order == "rows" else (n_paths, (K + 511) // 512, M, 16)
-    planes = torch.empty(shape, dtype=torch.int32, device=dev)
-    alpha = torch.empty((n_paths, M, K // G), dtype=torch.float32, device=dev)
-    a16 = torch.empty((n_paths, M, K // G), dtype=torch.float16, device=dev) if alpha_f16 else None
+
+    def out(t, shp, dt):
+        if t is None:
+            return torch.empty(shp, dtype=dt, device=dev)
+        if tuple(t.shape) != tuple(shp) or t.dtype != dt or not t.is_contiguous():
+            raise ValueError(f"output tensor must be contiguous {dt} of shape {shp}")
+        return t
+    planes = out(planes, shape, torch.int32)
+    alpha = out(alpha, (n_paths, M, K // G), torch.float32)
+    a16 = out(alpha16, (n_paths, M, K // G), torch.float16) if alpha_f16 else None
     with torch.cuda.device(dev):
         check(lib.rb_pack(_p(W), _DT[W.dtype], W.stride(0), layout(M, K, n_paths, group, order),
                           _p(planes), _p(alpha), _p(a16), _stream(dev)))
@@ -120,8 +130,12 @@ def _x2d(x: torch.Tensor) -> torch.Tensor:
 
 def gemv(planes: torch.Tensor, alpha: torch.Tensor, x: torch.Tensor, group: int = 0,
          y: Optional[torch.Tensor] = None, y_dtype: torch.dtype = torch.float16,
-         workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """y[t] = sum_k alpha_k (.) (B_k x[t]) for T <= 64 tokens (CUDA-core table kernel)."""
+         workspace: Optional[torch.Tensor] = None, check_device: bool = False) -> torch.Tensor:
+    """y[t] = sum_k alpha_k (.) (B_k x[t]) for T <= 64 tokens (CUDA-core table kernel).
+
+    With check_device=True the call waits for the stream and raises if the
+    kernel recorded a failure in its workspace (rb_gemv_check).
+    """
     lib = _lib.load()
     x = _x2d(x)
     dev = _require_cuda(planes, alpha, x, y, workspace)
@@ -138,6 +152,8 @@ def gemv(planes: torch.Tensor, alpha: torch.Tensor, x: torch.Tensor, group: int 
         check(lib.rb_gemv(_p(planes), _p(alpha), _DT[alpha.dtype], L, _p(x), x.stride(0), T,
                           _p(y), _DT[y.dtype], y.stride(0), _p(workspace),
                           workspace.numel() * workspace.element_size(), _stream(dev)))
+        if check_device:
+            check(lib.rb_gemv_check(_p(workspace), _stream(dev)))
     return y
 
 
@@ -168,6 +184,9 @@ class GroupedGemv:
                 raise ValueError(f"item {i}: inconsistent shapes or plane orders")
             if not (x.is_contiguous() and y.is_contiguous()):
                 raise ValueError(f"item {i}: x and y must be contiguous [T, K] / [T, M]")
+            # the descriptors are dense [T][K] / [T][M]: exactly T rows each
+            if x.numel() != T * K or y.numel() != T * M:
+                raise ValueError(f"item {i}: x must hold {T} x {K} and y {T} x {M} values")
             adt = alpha.dtype if adt is None else adt
             ydt = y.dtype if ydt is None else ydt
             if alpha.dtype != adt or y.dtype != ydt:
@@ -194,20 +213,34 @@ class GroupedGemv:
         check(_lib.load().rb_gemv_check(_p(self.workspace), _stream(self.device)))
 
 
+def gemm_workspace_bytes(M: int, K: int, n_paths: int, group: int, T: int) -> int:
+    return _lib.load().rb_gemm_workspace_bytes(layout(M, K, n_paths, group), T)
+
+
 def gemm(planes: torch.Tensor, alpha: torch.Tensor, X: torch.Tensor, group: int = 0,
-         Y: Optional[torch.Tensor] = None, y_dtype: torch.dtype = torch.float16) -> torch.Tensor:
-    """Y[t] = sum_k alpha_k (.) (B_k X[t]) for a prefill block (tcgen05 tensor-core kernel)."""
+         Y: Optional[torch.Tensor] = None, y_dtype: torch.dtype = torch.float16,
+         workspace: Optional[torch.Tensor] = None, check_device: bool = False) -> torch.Tensor:
+    """Y[t] = sum_k alpha_k (.) (B_k X[t]) on the tcgen05 tensor cores (any T).
+
+    With check_device=True the call waits for the stream and raises if a
+    kernel recorded a failure in its workspace (rb_gemm_check).
+    """
     lib = _lib.load()
-    if not hasattr(lib, "rb_gemm"):
-        raise _lib.RbError(2, "this build has no rb_gemm")
     X = _x2d(X)
-    dev = _require_cuda(planes, alpha, X, Y)
+    dev = _require_cuda(planes, alpha, X, Y, workspace)
     K = X.shape[1]
     N, M, order = _planes_geometry(planes, K)
     T = X.shape[0]
     if Y is None:
         Y = torch.empty((T, M), dtype=y_dtype, device=dev)
+    L = layout(M, K, N, group, order)
+    need = lib.rb_gemm_workspace_bytes(L, T)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
     with torch.cuda.device(dev):
-        check(lib.rb_gemm(_p(planes), _p(alpha), _DT[alpha.dtype], layout(M, K, N, group, order), _p(X), X.stride(0), T,
-                          _p(Y), _DT[Y.dtype], Y.stride(0), _stream(dev)))
+        check(lib.rb_gemm(_p(planes), _p(alpha), _DT[alpha.dtype], L, _p(X), X.stride(0), T,
+                          _p(Y), _DT[Y.dtype], Y.stride(0), _p(workspace),
+                          workspace.numel() * workspace.element_size(), _stream(dev)))
+        if check_device:
+            check(lib.rb_gemm_check(_p(workspace), _stream(dev)))
     return Y

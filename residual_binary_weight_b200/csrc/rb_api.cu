@@ -1,6 +1,7 @@
 // Host side of the C ABI declared in include/rb_api.h: argument validation,
 // launch planning and error reporting. Every check runs before anything is
-// enqueued; the kernels live in rb_pack.cu, rb_gemv.cu and rb_gemm.cu.
+// enqueued; the kernels live in rb_pack.cu, rb_gemv.cu, rb_gemm.cu (prefill
+// blocks) and rb_gemm_dec.cu (decode batches).
 #include "../../include/rb_api.h"
 #include "rb_internal.cuh"
 
@@ -177,14 +178,19 @@ rb_status rb_gemv(const uint32_t* planes, const void* alpha, rb_dtype alpha_dtyp
     a.chunk_slices = pl.chunk_slices;
     a.workspace = workspace;
     a.ws_bytes = ws_bytes;
+    a.expect_units = static_cast<uint32_t>(pl.units);
+    a.expect_ctrs = static_cast<uint32_t>(pl.counters);
+    a.expect_parts = static_cast<uint32_t>(pl.partials);
     e = launch_gemv(a, pl, s);
     if (e != cudaSuccess) return cuda_fail(e, "rb_gemv launch");
     return RB_OK;
 }
 
-static rb_status check_descs(const rb_gemv_desc* d, int32_t n, int32_t n_paths, int32_t group, int32_t order) {
+static rb_status check_descs(const rb_gemv_desc* d, int32_t n, int32_t n_paths, int32_t group, int32_t order,
+                             rb_dtype alpha_dtype, rb_dtype y_dtype) {
     if (!d) return fail(RB_ERR_INVALID_ARG, "null descriptors");
     if (n < 1 || n > gemv_max_jobs()) return fail(RB_ERR_UNSUPPORTED, "n=%d outside 1..%d", n, gemv_max_jobs());
+    if (!valid_dtype(alpha_dtype) || !valid_dtype(y_dtype)) return fail(RB_ERR_INVALID_ARG, "bad dtype");
     for (int32_t i = 0; i < n; ++i) {
         rb_layout L{d[i].M, d[i].K, n_paths, group, order, 0};
         rb_status st = check_layout(L);
@@ -193,6 +199,10 @@ static rb_status check_descs(const rb_gemv_desc* d, int32_t n, int32_t n_paths, 
             return fail(RB_ERR_INVALID_ARG, "descriptor %d has a null pointer", i);
         if (!aligned16(d[i].planes) || !aligned16(d[i].x))
             return fail(RB_ERR_ALIGNMENT, "descriptor %d: planes and x must be 16-byte aligned", i);
+        if (reinterpret_cast<uintptr_t>(d[i].alpha) & (dtype_size(alpha_dtype) - 1))
+            return fail(RB_ERR_ALIGNMENT, "descriptor %d: alpha misaligned for its dtype", i);
+        if (reinterpret_cast<uintptr_t>(d[i].y) & (dtype_size(y_dtype) - 1))
+            return fail(RB_ERR_ALIGNMENT, "descriptor %d: y misaligned for its dtype", i);
     }
     return RB_OK;
 }
@@ -216,7 +226,7 @@ rb_status rb_gemv_grouped(const rb_gemv_desc* descs_host, const rb_gemv_desc* de
                           void* workspace, size_t ws_bytes, void* stream) {
     g_last_error.clear();
     static_assert(sizeof(rb_gemv_desc) == sizeof(GvJob), "descriptor layout");
-    rb_status st = check_descs(descs_host, n, n_paths, group, order);
+    rb_status st = check_descs(descs_host, n, n_paths, group, order, alpha_dtype, y_dtype);
     if (st != RB_OK) return st;
     if (!descs_dev || (reinterpret_cast<uintptr_t>(descs_dev) & 7u))
         return fail(RB_ERR_INVALID_ARG, "descs_dev must be a non-null, 8-byte aligned device pointer");
@@ -244,56 +254,106 @@ rb_status rb_gemv_grouped(const rb_gemv_desc* descs_host, const rb_gemv_desc* de
     a.chunk_slices = pl.chunk_slices;
     a.workspace = workspace;
     a.ws_bytes = ws_bytes;
+    a.expect_units = static_cast<uint32_t>(pl.units);
+    a.expect_ctrs = static_cast<uint32_t>(pl.counters);
+    a.expect_parts = static_cast<uint32_t>(pl.partials);
     e = launch_gemv(a, pl, s);
     if (e != cudaSuccess) return cuda_fail(e, "rb_gemv_grouped launch");
     return RB_OK;
 }
 
+size_t rb_gemm_workspace_bytes(rb_layout L, int32_t T) {
+    if (check_layout(L) != RB_OK || T < 1) return 0;
+    if (T > GEMM_DEC_MAX_T) return GEMM_HEADER_BYTES;
+    const GemmDecPlan pl = gemm_dec_plan(L.M, L.K, L.n_paths, T, device_sm_count());
+    return GEMM_HEADER_BYTES + pl.counters_bytes + pl.partials_bytes + pl.xp_bytes;
+}
+
 rb_status rb_gemm(const uint32_t* planes, const void* alpha, rb_dtype alpha_dtype, rb_layout L,
-                  const void* X, int64_t ldx, int32_t T, void* Y, rb_dtype y_dtype, int64_t ldy, void* stream) {
+                  const void* X, int64_t ldx, int32_t T, void* Y, rb_dtype y_dtype, int64_t ldy,
+                  void* workspace, size_t ws_bytes, void* stream) {
     g_last_error.clear();
     rb_status st = check_layout(L);
     if (st != RB_OK) return st;
     if (!planes || !alpha || !X || !Y) return fail(RB_ERR_INVALID_ARG, "null planes, alpha, X or Y");
     if (!valid_dtype(alpha_dtype) || !valid_dtype(y_dtype)) return fail(RB_ERR_INVALID_ARG, "bad dtype");
-    if (!gemm_supported(L.n_paths, L.group)) return fail(RB_ERR_UNSUPPORTED, "rb_gemm supports 1..4 paths");
-    if (T < 1 || T > (1 << 24)) return fail(RB_ERR_UNSUPPORTED, "T=%d outside 1..2^24", T);
+    if (L.n_paths > 4) return fail(RB_ERR_UNSUPPORTED, "rb_gemm supports 1..4 paths");
+    if (L.group == 128 && alpha_dtype != RB_F16)
+        return fail(RB_ERR_UNSUPPORTED, "rb_gemm with one scale per 128 columns takes fp16 scales "
+                                        "(they are folded exactly into the fp16 operand)");
+    if (T < 1 || T > (1 << 22)) return fail(RB_ERR_UNSUPPORTED, "T=%d outside 1..2^22", T);
     if (ldx < L.K || ldy < L.M) return fail(RB_ERR_INVALID_ARG, "ldx < K or ldy < M");
     if (!aligned16(planes) || !aligned16(X) || (ldx * 2) % 16 != 0)
         return fail(RB_ERR_ALIGNMENT, "planes, X and the row pitch of X must be 16-byte aligned");
     if (reinterpret_cast<uintptr_t>(alpha) & (dtype_size(alpha_dtype) - 1))
         return fail(RB_ERR_ALIGNMENT, "alpha misaligned for its dtype");
     if (reinterpret_cast<uintptr_t>(Y) & (dtype_size(y_dtype) - 1)) return fail(RB_ERR_ALIGNMENT, "Y misaligned");
-    cudaError_t e = launch_gemm(planes, alpha, alpha_dtype == RB_F16, L.M, L.K, L.n_paths, L.group,
+    const bool dec = T <= GEMM_DEC_MAX_T;
+    GemmDecPlan pl{};
+    size_t need = GEMM_HEADER_BYTES, clear = GEMM_HEADER_BYTES;
+    if (dec) {
+        pl = gemm_dec_plan(L.M, L.K, L.n_paths, T, device_sm_count());
+        need += pl.counters_bytes + pl.partials_bytes + pl.xp_bytes;
+        clear += pl.counters_bytes;
+    }
+    if (!workspace || ws_bytes < need || !aligned16(workspace))
+        return fail(RB_ERR_WORKSPACE, "workspace needs %zu bytes (16-byte aligned), got %zu", need, ws_bytes);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(workspace, 0, clear, s);
+    if (e != cudaSuccess) return cuda_fail(e, "rb_gemm workspace clear");
+    if (dec)
+        e = launch_gemm_dec(planes, alpha, alpha_dtype == RB_F16, L.M, L.K, L.n_paths, L.group, L.order == RB_SLICED,
+                            X, ldx, T, Y, y_dtype == RB_F16, ldy, workspace, pl, s);
+    else
+        e = launch_gemm_prefill(planes, alpha, alpha_dtype == RB_F16, L.M, L.K, L.n_paths, L.group,
                                 L.order == RB_SLICED, X, ldx, T, Y, y_dtype == RB_F16, ldy,
-                                static_cast<cudaStream_t>(stream));
+                                static_cast<uint32_t*>(workspace) + 1, s);
     if (e == cudaErrorNotSupported) return fail(RB_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
     if (e != cudaSuccess) return cuda_fail(e, "rb_gemm launch");
     return RB_OK;
 }
 
-rb_status rb_gemm_check(void* stream) {
+// Wait for `stream`, then read word 1 (the error flags) of a workspace header.
+static rb_status read_flags(const void* header, void* stream, const char* who, uint32_t* flags) {
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(flags, static_cast<const uint32_t*>(header) + 1, sizeof(uint32_t),
+                                    cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, who);
+    return RB_OK;
+}
+
+rb_status rb_gemm_check(const void* workspace, void* stream) {
     g_last_error.clear();
-    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
-    unsigned int code = 0;
-    if (e == cudaSuccess) e = gemm_read_error(&code);
-    if (e != cudaSuccess) return cuda_fail(e, "rb_gemm_check");
-    if (code) return fail(RB_ERR_DEVICE, "rb_gemm kernel wait ran out (code 0x%x)", code);
+    if (!workspace) return fail(RB_ERR_INVALID_ARG, "null workspace");
+    uint32_t flag = 0;
+    rb_status st = read_flags(workspace, stream, "rb_gemm_check", &flag);
+    if (st != RB_OK) return st;
+    if (flag)
+        return fail(RB_ERR_DEVICE, "rb_gemm kernel flag 0x%x: a pipeline wait ran out in (%s%s%s%s)", flag,
+                    (flag & 1u) ? "X-tile producer " : "", (flag & 2u) ? "MMA issuer " : "",
+                    (flag & 4u) ? "operand expansion " : "", (flag & 8u) ? "epilogue" : "");
     return RB_OK;
 }
 
 rb_status rb_gemv_check(const void* workspace, void* stream) {
     g_last_error.clear();
-    if (!workspace) return fail(RB_ERR_INVALID_ARG, "null workspace");
+    const void* header = workspace;
+    if (!header) {
+        // the static scratch of rb_gemv_noalloc on the current device
+        void* p = nullptr;
+        cudaError_t e = noalloc_scratch(&p);
+        if (e != cudaSuccess) return cuda_fail(e, "rb_gemv_check (static scratch)");
+        header = p;
+    }
     uint32_t flag = 0;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = cudaMemcpyAsync(&flag, static_cast<const uint32_t*>(workspace) + 1, sizeof(flag),
-                                    cudaMemcpyDeviceToHost, s);
-    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
-    if (e != cudaSuccess) return cuda_fail(e, "rb_gemv_check");
+    rb_status st = read_flags(header, stream, "rb_gemv_check", &flag);
+    if (st != RB_OK) return st;
     if (flag)
-        return fail(RB_ERR_DEVICE, "matvec kernel flag 0x%x (%s%s)", flag,
-                    (flag & GV_ERR_SMEM_LAYOUT) ? "shared-memory window not where the tables need it " : "",
+        return fail(RB_ERR_DEVICE, "matvec kernel flag 0x%x (%s%s%s)", flag,
+                    (flag & GV_ERR_SMEM_LAYOUT) ? "shared-memory window not where the tables need it; " : "",
+                    (flag & GV_ERR_BAD_JOB) ? "device descriptors differ from the host copy the launch was "
+                                              "planned on; " : "",
                     (flag & GV_ERR_TOO_MANY_JOBS) ? "more descriptors than a launch takes" : "");
     return RB_OK;
 }

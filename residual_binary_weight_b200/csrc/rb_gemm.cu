@@ -1,5 +1,6 @@
-// rb_gemm: Y = sum_k alpha_k (.) (B_k X^T) for a block of T tokens on the
-// tcgen05 tensor cores (sm_100a).
+// rb_gemm, prefill blocks: Y = sum_k alpha_k (.) (B_k X^T) for a block of
+// T > 64 tokens on the tcgen05 tensor cores (sm_100a). Decode batches of at
+// most 64 tokens go to the persistent kernel of rb_gemm_dec.cu.
 //
 // The per-path contraction B_k X^T is a dense GEMM with a +-1 operand: the
 // plane bits are expanded exactly to fp16 +-1.0 (or, with one scale per 128
@@ -18,128 +19,23 @@
 //              K-major 128-byte-swizzled fp16 A tile of every path, then run
 //              the epilogue: tcgen05.ld of the accumulators, scale, fp16/fp32
 //              store.
-// Stages are handed over with mbarriers: full[s] (TMA bytes + 128 expansion
-// arrivals) and empty[s] (tcgen05.commit after the MMAs that read stage s).
-// Every wait is bounded; a wait that runs out records an error code, raises
-// a CTA-wide abort flag and the kernel winds down instead of hanging.
-#include "rb_internal.cuh"
-
-#include <cuda.h>
+// Stages are handed over with mbarriers: full_x[s] (TMA bytes), full_a[s]
+// (128 expansion arrivals) and empty[s] (tcgen05.commit after the MMAs that
+// read stage s). Every wait is bounded; a wait that runs out records an error
+// code in the call's error word, raises a CTA-wide abort flag and the kernel
+// winds down instead of hanging (after draining its issued MMAs and loads).
+#include "rb_tc.cuh"
 
 namespace rb {
 namespace {
 
-constexpr int BM = 128;          // rows per tile (UMMA M)
-constexpr int BK = 64;           // columns per stage (one 128-byte swizzle row of fp16)
+using namespace tc;
+
 constexpr int THREADS = 256;
 constexpr int EXP_WARP0 = 4;     // first expansion/epilogue warp
 constexpr uint32_t A_TILE_BYTES = BM * BK * 2;   // 16 KB
-constexpr uint32_t WAIT_LIMIT = 1u << 26;
-
-__device__ unsigned int g_gemm_error;   // first failure code of any rb_gemm launch
 
 __device__ __forceinline__ uint32_t elect_lane0() { return (threadIdx.x & 31) == 0; }
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-// Bounded wait for phase `parity` of barrier `bar`. Returns false (after
-// recording `code` and raising the CTA abort flag) if it runs out, or at once
-// if another thread already aborted.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile uint32_t* abort_flag,
-                                          uint32_t code) {
-    for (uint32_t i = 0; i < WAIT_LIMIT; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if (*abort_flag) return false;
-    }
-    atomicOr(&g_gemm_error, code);
-    *abort_flag = 1u;
-    return false;
-}
-
-__device__ __forceinline__ void fence_proxy_async_smem() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-// UMMA shared-memory descriptor of a K-major tile in the 128-byte swizzle
-// layout: 8-row atoms of 1024 bytes (leading offset 16 B, stride 1024 B).
-__device__ __forceinline__ uint64_t smem_desc(uint32_t addr) {
-    return static_cast<uint64_t>((addr >> 4) & 0x3FFFu) | (static_cast<uint64_t>(1) << 16) |
-           (static_cast<uint64_t>(1024 >> 4) << 32) | (static_cast<uint64_t>(1) << 46) |
-           (static_cast<uint64_t>(2) << 61);
-}
-
-// kind::f16 instruction descriptor: fp32 accumulator, fp16 A and B, both
-// K-major, M = 128, N = BN.
-__host__ __device__ constexpr uint32_t instr_desc(int bn) {
-    return (1u << 4) | (static_cast<uint32_t>(bn >> 3) << 17) | (static_cast<uint32_t>(BM >> 4) << 24);
-}
-
-__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                         uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-__device__ __forceinline__ void umma_commit(uint32_t bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-                 : "memory");
-}
-
-// D (+)= A x B with the A operand (128 rows x 16 fp16 columns) read from
-// tensor memory at a_tmem instead of shared memory
-__device__ __forceinline__ void umma_f16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
-                                            uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
-        ::"r"(d_tmem), "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate));
-}
-
-// 32 lanes x 16 columns of 32 bits into tensor memory (this warp's lane quarter)
-__device__ __forceinline__ void tmem_store16(uint32_t taddr, const uint32_t (&v)[16]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};"
-        ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
-          "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
-        : "memory");
-}
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
-        ::"r"(dst), "l"(map), "r"(x), "r"(y), "r"(bar)
-        : "memory");
-}
 
 __device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
@@ -174,38 +70,8 @@ __device__ __forceinline__ void expand_word(uint32_t w, uint32_t val2, uint32_t 
     }
 }
 
-// 32 lanes x CW columns of fp32 from tensor memory (this warp's lane quarter)
-template <int CW>
-__device__ __forceinline__ void tmem_load(uint32_t taddr, uint32_t (&v)[CW]);
-
-template <>
-__device__ __forceinline__ void tmem_load<32>(uint32_t taddr, uint32_t (&v)[32]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
-          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
-          "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]),
-          "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]),
-          "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
-template <>
-__device__ __forceinline__ void tmem_load<16>(uint32_t taddr, uint32_t (&v)[16]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
-        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
-          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
-          "=r"(v[14]), "=r"(v[15])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
 struct GemmArgs {
+    uint32_t* err;          // device error word of the call (workspace header word 1)
     const uint32_t* planes;
     const void* alpha;
     void* y;
@@ -251,10 +117,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, GemmArgs a) {
     // 1024-byte aligned tile area (the 128-byte swizzle repeats every 1024 B)
     const uint32_t raw = smem_addr(dsm);
     const uint32_t tiles = (raw + 1023u) & ~1023u;
-    const uint32_t bars = tiles + STAGES * C::STAGE_BYTES;     // full[STAGES], empty[STAGES], accf
-    auto full_bar = [&](int s) { return bars + 8u * s; };
-    auto empty_bar = [&](int s) { return bars + 8u * (STAGES + s); };
-    const uint32_t acc_bar = bars + 8u * (2 * STAGES);
+    // barriers: full_x[STAGES] (X tile landed), full_a[STAGES] (A expanded),
+    // empty[STAGES] (MMAs of the stage done), acc (all MMAs done)
+    const uint32_t bars = tiles + STAGES * C::STAGE_BYTES;
+    auto full_x = [&](int s) { return bars + 8u * s; };
+    auto full_a = [&](int s) { return bars + 8u * (STAGES + s); };
+    auto empty_bar = [&](int s) { return bars + 8u * (2 * STAGES + s); };
+    const uint32_t acc_bar = bars + 8u * (3 * STAGES);
     const uint32_t tmem_slot = acc_bar + 8u;
     const uint32_t abort_slot = tmem_slot + 4u;
     volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(dsm + (abort_slot - raw));
@@ -270,34 +139,38 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, GemmArgs a) {
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(full_bar(s), 1 + 128);
+            mbar_init(full_x(s), 1);
+            mbar_init(full_a(s), 128);
             mbar_init(empty_bar(s), 1);
         }
         mbar_init(acc_bar, 1);
         *abort_flag = 0u;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(tmem_slot),
-                     "r"(C::TMEM_COLS)
-                     : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-    }
-    tc_fence_before();
+    if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
+    fence_before();
     __syncthreads();
-    tc_fence_after();
+    fence_after();
+    uint32_t* err = a.err;
     const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(dsm + (tmem_slot - raw));
 
     if (warp == 0) {
         // ---------------------------------------------------------- TMA producer
         if (elect_lane0()) {
+            int issued = 0;
             for (int kb = 0; kb < nk; ++kb) {
                 const int s = kb % STAGES;
                 const uint32_t ph = static_cast<uint32_t>(kb / STAGES) & 1u;
-                if (!mbar_wait(empty_bar(s), ph ^ 1u, abort_flag, 1u)) break;
-                mbar_arrive_expect_tx(full_bar(s), C::B_TILE_BYTES);
-                tma_load_2d(b_tile(s), &xmap, kb * BK, tok_tile * BN, full_bar(s));
+                if (!mbar_wait(empty_bar(s), ph ^ 1u, abort_flag, err, 1u)) break;
+                mbar_arrive_expect_tx(full_x(s), C::B_TILE_BYTES);
+                tma_load_2d(b_tile(s), &xmap, kb * BK, tok_tile * BN, full_x(s));
+                issued = kb + 1;
             }
+            // after an abort, the loads still in flight land before the CTA
+            // releases its shared memory: wait for the last load of each stage
+            if (*abort_flag)
+                for (int kb = issued - 1; kb >= 0 && kb >= issued - STAGES; --kb)
+                    mbar_drain(full_x(kb % STAGES), static_cast<uint32_t>(kb / STAGES) & 1u);
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
@@ -307,8 +180,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, GemmArgs a) {
             for (int kb = 0; kb < nk && ok; ++kb) {
                 const int s = kb % STAGES;
                 const uint32_t ph = static_cast<uint32_t>(kb / STAGES) & 1u;
-                if (!mbar_wait(full_bar(s), ph, abort_flag, 2u)) { ok = false; break; }
-                tc_fence_after();
+                if (!mbar_wait(full_x(s), ph, abort_flag, err, 2u) || !mbar_wait(full_a(s), ph, abort_flag, err, 2u)) {
+                    ok = false;
+                    break;
+                }
+                fence_after();
 #pragma unroll
                 for (int p = 0; p < NP; ++p) {
                     const uint32_t d = tmem_base + static_cast<uint32_t>(G128 ? 0 : p * C::ACC_STRIDE);
@@ -326,7 +202,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, GemmArgs a) {
                 }
                 umma_commit(empty_bar(s));      // stage s is free once these MMAs completed
             }
-            umma_commit(acc_bar);               // accumulators complete
+            umma_commit(acc_bar);               // accumulators complete (also after an abort:
+                                                // the teardown waits on it before freeing TMEM)
         }
     } else if (warp >= EXP_WARP0) {
         // ------------------------------------------------- expansion, then epilogue
@@ -346,9 +223,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, GemmArgs a) {
         auto alpha_h2 = [&](int p, int kb) -> uint32_t {
             if (!G128) return 0x3C003C00u;                             // +1.0 in both halves
             const int64_t ai = (p * M + crow) * gpr + (static_cast<int64_t>(kb) * BK >> 7);
-            uint32_t hv;
-            if (a.alpha_f16) hv = static_cast<const unsigned short*>(a.alpha)[ai];
-            else hv = __half_as_ushort(__float2half_rn(static_cast<const float*>(a.alpha)[ai]));
+            // group scales are fp16 (the host refuses fp32 ones): +-alpha is exact
+            const uint32_t hv = static_cast<const unsigned short*>(a.alpha)[ai];
             return hv | (hv << 16);
         };
         const uint32_t rsw = static_cast<uint32_t>(r & 7);
@@ -391,7 +267,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, GemmArgs a) {
                             aring[i][p] = alpha_h2(p, kb + PD);
                         }
                     }
-                    if (!mbar_wait(empty_bar(s), ph ^ 1u, abort_flag, 4u)) {
+                    // warp-uniform: the tensor-memory stores below are .sync.aligned
+                    if (!__all_sync(FULL_MASK, mbar_wait(empty_bar(s), ph ^ 1u, abort_flag, err, 4u))) {
                         go = false;
                     } else {
 #pragma unroll
@@ -415,20 +292,20 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, GemmArgs a) {
                             }
                         }
                         if (ATM) {
-                            asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");   // stores done first
-                            tc_fence_before();
+                            tmem_store_wait();   // stores done first
+                            fence_before();
                         } else {
                             fence_proxy_async_smem();   // make the generic-proxy stores visible to the tensor core
                         }
-                        mbar_arrive(full_bar(s));
+                        mbar_arrive(full_a(s));
                     }
                 }
             }
         }
 
         // ------------------------------------------------------------ epilogue
-        const bool ok = mbar_wait(acc_bar, 0u, abort_flag, 8u);
-        tc_fence_after();
+        const bool ok = __all_sync(FULL_MASK, mbar_wait(acc_bar, 0u, abort_flag, err, 8u));
+        fence_after();
         if (ok) {
             float al[C::NACC];
 #pragma unroll
@@ -468,48 +345,25 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, GemmArgs a) {
     }
 
     __syncwarp();            // lanes 1..31 of warps 0 and 1 wait for their lane 0
-    tc_fence_before();
+    fence_before();
     __syncthreads();
     if (warp == 1) {
-        tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(C::TMEM_COLS)
-                     : "memory");
+        // after an abort, the MMAs already issued finish before their tensor
+        // memory is released (the MMA thread committed them to acc_bar)
+        if (elect_lane0() && *abort_flag) mbar_drain(acc_bar, 0u);
+        __syncwarp();
+        fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
     }
 }
 
 // ---------------------------------------------------------------- host side
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    static bool tried = false;
-    if (!tried) {
-        tried = true;
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
-    return fn;
-}
-
 template <int NP, int BN, int STAGES, bool G128, bool ATM = false>
 cudaError_t launch_cfg(const GemmArgs& a, const void* X, int64_t ldx, cudaStream_t s) {
     using C = GemmCfg<NP, BN, STAGES, G128, ATM>;
-    EncodeTiledFn enc = encode_fn();
-    if (!enc) return cudaErrorNotSupported;
     CUtensorMap map;
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.K), static_cast<cuuint64_t>(a.T)};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ldx) * 2};
-    const cuuint32_t box[2] = {BK, BN};
-    const cuuint32_t estr[2] = {1, 1};
-    if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(X), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return cudaErrorInvalidValue;
+    cudaError_t me = make_x_map(&map, X, a.K, a.T, ldx, BN);
+    if (me != cudaSuccess) return me;
     auto kern = gemm_tc_kernel<NP, BN, STAGES, G128, ATM>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
@@ -519,8 +373,6 @@ cudaError_t launch_cfg(const GemmArgs& a, const void* X, int64_t ldx, cudaStream
 }
 
 }  // namespace
-
-bool gemm_supported(int n_paths, int group) { return n_paths >= 1 && n_paths <= 4 && (group == 0 || group == 128); }
 
 // stages that fit in shared memory for a configuration (at most 8)
 constexpr int stages_for(int np, int bn) {
@@ -576,10 +428,10 @@ cudaError_t launch_np(const GemmArgs& a, const void* X, int64_t ldx, cudaStream_
     }
 }
 
-cudaError_t launch_gemm(const uint32_t* planes, const void* alpha, bool alpha_f16, int64_t M, int64_t K, int n_paths,
-                        int group, bool sliced, const void* X, int64_t ldx, int T, void* Y, bool y_f16, int64_t ldy,
-                        cudaStream_t s) {
-    GemmArgs a{planes, alpha, Y, M, K, ldy, T, n_paths, group == 128, sliced, alpha_f16, y_f16};
+cudaError_t launch_gemm_prefill(const uint32_t* planes, const void* alpha, bool alpha_f16, int64_t M, int64_t K,
+                                int n_paths, int group, bool sliced, const void* X, int64_t ldx, int T, void* Y,
+                                bool y_f16, int64_t ldy, uint32_t* err, cudaStream_t s) {
+    GemmArgs a{err, planes, alpha, Y, M, K, ldy, T, n_paths, group == 128, sliced, alpha_f16, y_f16};
     if (group == 0) {
         switch (n_paths) {
             case 1: return launch_np<1, false>(a, X, ldx, s);
@@ -598,14 +450,32 @@ cudaError_t launch_gemm(const uint32_t* planes, const void* alpha, bool alpha_f1
     return cudaErrorInvalidValue;
 }
 
-cudaError_t gemm_read_error(unsigned int* code) {
-    cudaError_t e = cudaMemcpyFromSymbol(code, g_gemm_error, sizeof(unsigned int));
-    if (e != cudaSuccess) return e;
-    if (*code) {
-        const unsigned int zero = 0;
-        e = cudaMemcpyToSymbol(g_gemm_error, &zero, sizeof(zero));
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
     }
-    return e;
+    return fn;
+}
+
+cudaError_t make_x_map(CUtensorMap* map, const void* X, int64_t cols, int64_t rows, int64_t ld, int box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return cudaErrorNotSupported;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(tc::BK), static_cast<cuuint32_t>(box_rows)};
+    const cuuint32_t estr[2] = {1, 1};
+    if (enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(X), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    return cudaSuccess;
 }
 
 }  // namespace rb

@@ -1,0 +1,512 @@
+// rb_gemm for decode batches: Y = sum_k alpha_k (.) (B_k X^T) for T <= 64
+// tokens on the tcgen05 tensor cores, one persistent CTA per SM.
+//
+// RaBiT (arXiv 2602.05367) section 4.1: y = sum_k alpha_k (.) (B_k x) with
+// B_k in {-1, +1}; QBB W(4x1)A16g128 for the per-128-column scales.
+//
+// At a few tokens the tensor core has little to do (an M=128, N=16, K=16 MMA
+// takes ~14 cycles); what bounds the contraction is turning plane bits into
+// fp16 operands, one value per weight and path, and handing stages between
+// the warps. The expansion is one shift and one LOP3 per two weights:
+//   * The columns of X are permuted once per call (a small pre-pass into the
+//     workspace) so that inside every 32-column block position 2k holds
+//     column k and position 2k + 1 holds column k + 16.
+//   * The fp16x2 operand of positions (2k, 2k + 1) then takes its two signs
+//     from bits k and k + 16 of the plane word: shifting the word left by
+//     15 - k puts them at bits 15 and 31, the two fp16 sign bits, and
+//     ((w << (15 - k)) & 0x80008000) ^ (-v, -v) is +-v in each half
+//     (v = 1.0, or alpha_k in fp16 with one scale per 128 columns: exact).
+//   * The expanded operand goes to tensor memory (tcgen05.st), so the MMA
+//     reads only the small X tile from shared memory.
+// A stage is SW = 128 columns (64 with more than two paths, for tensor-memory
+// room); the two groups of expansion warps take alternate stages, so each
+// warp synchronises once per two stages.
+//
+// Work split (stream-K): the row tiles (128 rows) x K stages are one sequence
+// of tiles * K/SW stages, cut into gridDim.x equal contiguous ranges, one per
+// CTA. A CTA's range covers whole tiles and at most two partial tiles (its
+// first and last); a partial tile's rows are written as fp32 partial sums
+// into the workspace, and the last of its CTAs to finish adds the parts in
+// CTA order (deterministic) and stores Y.
+//
+// Roles (14 warps):
+//   warps 0-7   expansion: warp w writes rows 32 (w % 4) .. + 31 (its tensor
+//               memory lane quarter) of every path, for the stages i of the
+//               CTA's range with i % 2 == w / 4;
+//   warps 8-11  epilogue: tcgen05.ld of the accumulators, per-row scales,
+//               store or partial sums;
+//   warp 12     TMA loads of the permuted X tiles;
+//   warp 13     allocates tensor memory and issues the MMAs.
+// Warps 12 and 13 run their loops converged (warp-uniform operands) and
+// issue through one elected lane. mbarriers: full[s] (TMA bytes + the 4
+// warps of the stage's group), empty[s] (MMAs of stage s done),
+// acc_full[b] / acc_empty[b] (accumulator buffer b filled / read). Every
+// wait is bounded; a wait that runs out records a code in the call's error
+// word and the CTA winds down after draining what it issued.
+#include "rb_tc.cuh"
+
+#include <type_traits>
+
+namespace rb {
+namespace {
+
+using namespace tc;
+
+constexpr int THREADS = 448;
+constexpr int EPI_WARP0 = 8;
+constexpr int TMA_WARP = 12;
+constexpr int MMA_WARP = 13;
+
+struct DecArgs {
+    uint32_t* err;          // the call's device error word
+    uint32_t* counters;     // one arrival counter per row tile (cleared by the host)
+    float* partials;        // [gridDim.x][2][BN][128] fp32 partial sums
+    const uint32_t* planes;
+    const void* alpha;
+    void* y;
+    int64_t M, K, ldy;
+    int64_t tiles;          // row tiles
+    int64_t total;          // tiles * K / SW stages
+    int T;
+    bool sliced, alpha_f16, y_f16;
+};
+
+__host__ __device__ constexpr int stage_cols(int np) { return np <= 2 ? 128 : 64; }
+
+template <int NP, int BN, bool G128>
+struct DecCfg {
+    static constexpr int SW = stage_cols(NP);             // K columns per stage
+    static constexpr int WPS = SW / 32;                    // plane words per row, path and stage
+    static constexpr int SUB = SW / BK;                    // 64-column X boxes per stage
+    static constexpr int NACC = G128 ? 1 : NP;             // accumulators per buffer
+    static constexpr int ACC_STRIDE = BN;                  // 16, 32 or 64 columns
+    static constexpr int A_STAGE_COLS = NP * SW / 2;       // fp16 pairs of all paths of one stage
+    // two accumulator buffers (the epilogue of one tile overlaps the next
+    // tile's MMAs) when that still leaves three operand stages
+    static constexpr int ACC_BUF = (512 - 2 * NACC * ACC_STRIDE) / A_STAGE_COLS >= 3 ? 2 : 1;
+    static constexpr int ACC_COLS = ACC_BUF * NACC * ACC_STRIDE;
+    static constexpr int STAGES_FIT = (512 - ACC_COLS) / A_STAGE_COLS;
+    static constexpr int STAGES = STAGES_FIT < 8 ? STAGES_FIT : 8;
+    static constexpr uint32_t SUB_BYTES = BN * BK * 2;     // one 64-column box of BN rows
+    static constexpr uint32_t B_TILE_BYTES = SUB * SUB_BYTES;
+    static constexpr uint32_t SMEM_USED = STAGES * B_TILE_BYTES + 1024 /*align*/ + 512 /*barriers*/;
+    // at least 120 KB, so that two CTAs never share an SM's tensor memory
+    static constexpr uint32_t SMEM_BYTES = SMEM_USED < 120u * 1024u ? 120u * 1024u : SMEM_USED;
+    static_assert(STAGES >= 2, "operand stages do not fit beside the accumulators");
+    static_assert(BN == 16 || BN == 32 || BN == 64, "token tile");
+    static_assert(SUB_BYTES % 1024 == 0, "X box must keep the 1024-byte swizzle alignment");
+};
+
+// first stage of CTA c's range and the CTA whose range holds stage g
+__device__ __forceinline__ int64_t range_lo(int64_t c, int64_t total, int64_t G) { return c * total / G; }
+__device__ __forceinline__ int64_t cta_of(int64_t g, int64_t total, int64_t G) { return ((g + 1) * G - 1) / total; }
+
+template <int NP, int BN, bool G128>
+__global__ void __launch_bounds__(THREADS, 1)
+gemm_dec_kernel(const __grid_constant__ CUtensorMap xmap, DecArgs a) {
+    using C = DecCfg<NP, BN, G128>;
+    constexpr int STAGES = C::STAGES, ACC_BUF = C::ACC_BUF, SW = C::SW, WPS = C::WPS;
+    extern __shared__ __align__(1024) unsigned char dsm[];
+    const uint32_t raw = smem_addr(dsm);
+    const uint32_t tiles_s = (raw + 1023u) & ~1023u;
+    const uint32_t bars = tiles_s + STAGES * C::B_TILE_BYTES;
+    auto full_bar = [&](int s) { return bars + 8u * s; };
+    auto empty_bar = [&](int s) { return bars + 8u * (STAGES + s); };
+    auto acc_full = [&](int b) { return bars + 8u * (2 * STAGES + b); };
+    auto acc_empty = [&](int b) { return bars + 8u * (2 * STAGES + 2 + b); };
+    const uint32_t fin_bar = bars + 8u * (2 * STAGES + 4);
+    const uint32_t tmem_slot = fin_bar + 8u;
+    const uint32_t abort_slot = tmem_slot + 4u;
+    const uint32_t last_slot = abort_slot + 4u;
+    volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(dsm + (abort_slot - raw));
+    volatile uint32_t* last_flag = reinterpret_cast<volatile uint32_t*>(dsm + (last_slot - raw));
+    auto b_tile = [&](int s) { return tiles_s + static_cast<uint32_t>(s) * C::B_TILE_BYTES; };
+    auto a_col = [&](int s, int p) { return static_cast<uint32_t>(C::ACC_COLS + (s * NP + p) * (SW / 2)); };
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t M = a.M, K = a.K, S = K / SW, total = a.total, G = gridDim.x, me = blockIdx.x;
+    const int64_t lo = range_lo(me, total, G), hi = range_lo(me + 1, total, G);
+    uint32_t* err = a.err;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(full_bar(s), 1 + 4);
+            mbar_init(empty_bar(s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(acc_full(b), 1);
+            mbar_init(acc_empty(b), 4);
+        }
+        mbar_init(fin_bar, 1);
+        *abort_flag = 0u;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == MMA_WARP) tmem_alloc(tmem_slot, 512);
+    fence_before();
+    __syncthreads();
+    fence_after();
+    const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(dsm + (tmem_slot - raw));
+
+    if (warp == TMA_WARP) {
+        // ------------------------------------------------------------ X tiles
+        int64_t issued = 0;
+        int s = 0, kb = static_cast<int>(lo % S);
+        uint32_t ph = 0;
+        for (int64_t i = 0; i < hi - lo; ++i) {
+            if (!__all_sync(FULL_MASK, mbar_wait(empty_bar(s), ph ^ 1u, abort_flag, err, 1u))) break;
+            if (elect_one()) {
+                mbar_arrive_expect_tx(full_bar(s), C::B_TILE_BYTES);
+#pragma unroll
+                for (int u = 0; u < C::SUB; ++u)
+                    tma_load_2d(b_tile(s) + u * C::SUB_BYTES, &xmap, kb * SW + u * BK, 0, full_bar(s));
+            }
+            __syncwarp();
+            issued = i + 1;
+            if (++kb == S) kb = 0;
+            if (++s == STAGES) {
+                s = 0;
+                ph ^= 1u;
+            }
+        }
+        if (*abort_flag)   // loads still in flight land before the CTA exits
+            for (int64_t i = issued - 1; i >= 0 && i >= issued - STAGES; --i)
+                mbar_drain(full_bar(static_cast<int>(i % STAGES)), static_cast<uint32_t>(i / STAGES) & 1u);
+    } else if (warp == MMA_WARP) {
+        // ---------------------------------------------------------------- MMA
+        constexpr uint32_t idesc = instr_desc(BN);
+        int st = 0;          // stage slot and phase of the next stage
+        uint32_t sph = 0;
+        int j = 0;           // segment counter
+        bool ok = true;
+        for (int64_t t = lo / S; ok && t * S < hi; ++t, ++j) {
+            const int64_t k0 = (lo > t * S ? lo - t * S : 0), k1 = (hi < (t + 1) * S ? hi - t * S : S);
+            const int b = j % ACC_BUF;
+            if (j >= ACC_BUF && !__all_sync(FULL_MASK, mbar_wait(acc_empty(b), static_cast<uint32_t>(j / ACC_BUF - 1) & 1u,
+                                                                  abort_flag, err, 2u))) {
+                ok = false;
+                break;
+            }
+            fence_after();
+            const uint32_t dbase = tmem_base + static_cast<uint32_t>(b * C::NACC * C::ACC_STRIDE);
+            for (int64_t kb = k0; kb < k1; ++kb) {
+                const int s = st;
+                const uint32_t ph = sph;
+                if (++st == STAGES) {
+                    st = 0;
+                    sph ^= 1u;
+                }
+                if (!__all_sync(FULL_MASK, mbar_wait(full_bar(s), ph, abort_flag, err, 2u))) {
+                    ok = false;
+                    break;
+                }
+                fence_after();
+                const uint64_t bd0 = smem_desc(b_tile(s));
+                const uint32_t acc0 = kb > k0 ? 1u : 0u;
+#pragma unroll
+                for (int p = 0; p < NP; ++p) {
+                    const uint32_t d = dbase + static_cast<uint32_t>(G128 ? 0 : p * C::ACC_STRIDE);
+#pragma unroll
+                    for (int kk = 0; kk < SW / 16; ++kk) {
+                        // 64-column box kk / 4; +32 bytes along K inside a
+                        // swizzled box is +2 in the descriptor's address field
+                        const uint64_t bd = bd0 + ((kk >> 2) * C::SUB_BYTES >> 4) + 2u * (kk & 3);
+                        const uint32_t acc = (kk > 0 || (G128 && p > 0)) ? 1u : acc0;
+                        umma_f16_ta_elect(d, tmem_base + a_col(s, p) + 8u * kk, bd, idesc, acc);
+                    }
+                }
+                umma_commit_elect(empty_bar(s));
+            }
+            if (ok) umma_commit_elect(acc_full(b));
+        }
+        umma_commit_elect(fin_bar);   // every MMA issued above has completed once this arrives
+    } else if (warp < 8) {
+        // ---------------------------------------------------------- expansion
+        // Thread = one row of the tile (its tensor-memory lane), all paths,
+        // the stages i with i % 2 == grp. The plane words of a stage (SW / 32
+        // per path) are loaded PR of the group's stages ahead.
+        const int q = warp & 3, grp = warp >> 2;
+        const int r = 32 * q + lane;
+        const uint32_t lane_q = static_cast<uint32_t>(32 * q) << 16;
+        const uint32_t uM = static_cast<uint32_t>(M);
+        const uint32_t W32 = static_cast<uint32_t>(K >> 5), SL = static_cast<uint32_t>((K + 511) >> 9);
+        const uint32_t gpr = static_cast<uint32_t>(K >> 7);
+        const uint32_t path_words = a.sliced ? SL * uM * 16u : uM * W32;   // < 2^30 (checked by the host)
+        using WV = typename std::conditional<WPS == 4, uint4, uint2>::type;
+        constexpr int PR = NP <= 2 ? 4 : 2;   // stages of this group loaded ahead
+        const int64_t n = hi - lo;
+        // (tile, stage-in-tile) of the next stage to load, stepping by 2
+        int64_t lt = (lo + grp) / S;
+        int lkb = static_cast<int>(lo + grp - lt * S);
+        WV ring[PR][NP];
+        uint32_t nring[PR][NP];
+        auto load_stage = [&](WV (&dst)[NP], uint32_t (&ndst)[NP]) {
+            const int64_t row64 = lt * BM + r;
+            const uint32_t row = static_cast<uint32_t>(row64 < M ? row64 : M - 1);   // rows past M read a real row
+            const uint32_t w = static_cast<uint32_t>(lkb) * WPS;
+            const uint32_t off = a.sliced ? ((w >> 4) * uM + row) * 16u + (w & 15u) : row * W32 + w;
+#pragma unroll
+            for (int p = 0; p < NP; ++p) {
+                dst[p] = __ldg(reinterpret_cast<const WV*>(a.planes + static_cast<size_t>(p) * path_words + off));
+                if (G128) {
+                    const uint32_t g = static_cast<uint32_t>(lkb) * SW / 128u;
+                    const uint32_t hv = static_cast<const unsigned short*>(a.alpha)[(p * uM + row) * gpr + g] | 0x8000u;
+                    ndst[p] = hv | (hv << 16);
+                } else {
+                    ndst[p] = 0xBC00BC00u;   // -1.0 in both halves
+                }
+            }
+            lkb += 2;
+            while (lkb >= S) {
+                lkb -= static_cast<int>(S);
+                ++lt;
+            }
+        };
+        // +-v pairs of one plane word into 16 tensor-memory columns
+        auto expand_store = [&](uint32_t w, uint32_t ng, uint32_t col) {
+            uint32_t h[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) h[k] = ((w << (15 - k)) & 0x80008000u) ^ ng;
+            tmem_store16(tmem_base + lane_q + col, h);
+        };
+        auto word = [](const WV& v, int i) -> uint32_t {
+            if constexpr (WPS == 4) return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+            else return i == 0 ? v.x : v.y;
+        };
+#pragma unroll
+        for (int d = 0; d < PR; ++d)
+            if (grp + 2 * d < n) load_stage(ring[d], nring[d]);
+        int s = grp % STAGES;
+        uint32_t ph = static_cast<uint32_t>(grp / STAGES) & 1u;
+        bool go = true;
+        for (int64_t i0 = grp; i0 < n && go; i0 += 2 * PR) {
+#pragma unroll
+            for (int d = 0; d < PR; ++d) {
+                const int64_t i = i0 + 2 * d;
+                if (i < n && go) {
+                    WV cur[NP];
+                    uint32_t ng[NP];
+#pragma unroll
+                    for (int p = 0; p < NP; ++p) {
+                        cur[p] = ring[d][p];
+                        ng[p] = nring[d][p];
+                    }
+                    if (i + 2 * PR < n) load_stage(ring[d], nring[d]);
+                    // warp-uniform: the tensor-memory stores below are .sync.aligned
+                    if (!__all_sync(FULL_MASK, mbar_wait(empty_bar(s), ph ^ 1u, abort_flag, err, 4u))) {
+                        go = false;
+                    } else {
+#pragma unroll
+                        for (int p = 0; p < NP; ++p)
+#pragma unroll
+                            for (int wi = 0; wi < WPS; ++wi) expand_store(word(cur[p], wi), ng[p], a_col(s, p) + 16u * wi);
+                        tmem_store_wait();
+                        fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(full_bar(s));
+                    }
+                    s += 2;
+                    if (s >= STAGES) {
+                        s -= STAGES;
+                        ph ^= 1u;
+                    }
+                }
+            }
+        }
+    } else if (warp >= EPI_WARP0 && warp < EPI_WARP0 + 4) {
+        // ----------------------------------------------------------- epilogue
+        const int q = warp & 3;
+        const int r = 32 * q + lane;
+        const uint32_t lane_q = static_cast<uint32_t>(32 * q) << 16;
+        constexpr int CW = BN < 32 ? BN : 32;
+        int j = 0;
+        for (int64_t t = lo / S; t * S < hi; ++t, ++j) {
+            const int64_t k0 = (lo > t * S ? lo - t * S : 0), k1 = (hi < (t + 1) * S ? hi - t * S : S);
+            const int b = j % ACC_BUF;
+            const int64_t row = t * BM + r;
+            const int64_t crow = row < M ? row : M - 1;
+            const bool ok =   // warp-uniform: tcgen05.ld is .sync.aligned
+                __all_sync(FULL_MASK, mbar_wait(acc_full(b), static_cast<uint32_t>(j / ACC_BUF) & 1u, abort_flag, err, 8u));
+            fence_after();
+            const bool full = k0 == 0 && k1 == S;
+            const int T = a.T;
+            const int slot = (t == lo / S) ? 0 : 1;
+            float* mine = a.partials + ((me * 2 + slot) * BN) * BM;
+            // one output value of token column c of this thread's row
+            auto store_y1 = [&](int c, float v) {
+                if (row < M && c < T) {
+                    if (a.y_f16) static_cast<__half*>(a.y)[c * a.ldy + row] = __float2half_rn(v);
+                    else static_cast<float*>(a.y)[c * a.ldy + row] = v;
+                }
+            };
+            if (ok) {
+                float al[C::NACC];
+#pragma unroll
+                for (int p = 0; p < C::NACC; ++p) {
+                    if (G128) al[p] = 1.0f;
+                    else al[p] = a.alpha_f16 ? __half2float(static_cast<const __half*>(a.alpha)[p * M + crow])
+                                             : static_cast<const float*>(a.alpha)[p * M + crow];
+                }
+                // CW token columns at a time: sum_k alpha_k acc_k, then Y or
+                // the partial-sum slot of this CTA
+#pragma unroll 1
+                for (int c0 = 0; c0 < BN; c0 += CW) {
+                    float yv[CW];
+#pragma unroll
+                    for (int c = 0; c < CW; ++c) yv[c] = 0.0f;
+#pragma unroll
+                    for (int p = 0; p < C::NACC; ++p) {
+                        uint32_t v[CW];
+                        tmem_load<CW>(tmem_base + lane_q +
+                                          static_cast<uint32_t>((b * C::NACC + p) * C::ACC_STRIDE + c0), v);
+#pragma unroll
+                        for (int c = 0; c < CW; ++c) yv[c] = fmaf(al[p], __uint_as_float(v[c]), yv[c]);
+                    }
+#pragma unroll
+                    for (int c = 0; c < CW; ++c) {
+                        if (full) store_y1(c0 + c, yv[c]);
+                        else if (c0 + c < T) mine[(c0 + c) * BM + r] = yv[c];
+                    }
+                }
+            }
+            fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty(b));   // the buffer may take the next tile
+            if (full) continue;
+            // partial tile: the same sequence of named barriers whatever happened
+            const int64_t first = cta_of(t * S, total, G), last = cta_of((t + 1) * S - 1, total, G);
+            if (ok) __threadfence();
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (threadIdx.x == EPI_WARP0 * 32) {
+                uint32_t prev = 0;
+                if (!*abort_flag) prev = atomicAdd(a.counters + t, 1u);
+                *last_flag = (!*abort_flag && prev == static_cast<uint32_t>(last - first)) ? 1u : 0u;
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (*last_flag && ok) {
+                // every part, this CTA's own included, is read back from the
+                // workspace and added in CTA order: the result does not
+                // depend on which CTA finished last
+                __threadfence();
+#pragma unroll 1
+                for (int c0 = 0; c0 < BN; c0 += CW) {
+                    float yv[CW];
+#pragma unroll
+                    for (int c = 0; c < CW; ++c) yv[c] = 0.0f;
+                    for (int64_t cc = first; cc <= last; ++cc) {
+                        const int sl = (t == range_lo(cc, total, G) / S) ? 0 : 1;
+                        const float* part = a.partials + ((cc * 2 + sl) * BN) * BM;
+#pragma unroll
+                        for (int c = 0; c < CW; ++c)
+                            if (c0 + c < T) yv[c] += __ldcg(part + (c0 + c) * BM + r);
+                    }
+#pragma unroll
+                    for (int c = 0; c < CW; ++c) store_y1(c0 + c, yv[c]);
+                }
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");   // last_flag is reused by the next tile
+        }
+    }
+
+    __syncwarp();
+    fence_before();
+    __syncthreads();
+    if (warp == MMA_WARP) {
+        mbar_drain(fin_bar, 0u);   // no MMA still reads or writes tensor memory
+        __syncwarp();
+        fence_after();
+        tmem_dealloc(tmem_base, 512);
+    }
+}
+
+// X' = X with the columns of every 32-column block reordered so that
+// position 2k holds column k and position 2k + 1 column k + 16 (the operand
+// order the expansion above produces). One thread per (token, block).
+__global__ void permute_x_kernel(const __half* __restrict__ X, int64_t ldx, int T, int64_t K,
+                                 __half* __restrict__ Xp) {
+    const int64_t blocks = K >> 5;
+    const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (idx >= blocks * T) return;
+    const int64_t t = idx / blocks, bl = idx - t * blocks;
+    const uint4* src = reinterpret_cast<const uint4*>(X + t * ldx + 32 * bl);
+    const uint4 l0 = __ldg(src), l1 = __ldg(src + 1), h0 = __ldg(src + 2), h1 = __ldg(src + 3);
+    const uint32_t lw[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};   // columns 2m, 2m + 1
+    const uint32_t hw[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};   // columns 16 + 2m, 17 + 2m
+    uint32_t o[16];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+        o[2 * m] = __byte_perm(lw[m], hw[m], 0x5410);       // (column 2m, column 16 + 2m)
+        o[2 * m + 1] = __byte_perm(lw[m], hw[m], 0x7632);   // (column 2m + 1, column 17 + 2m)
+    }
+    uint4* dst = reinterpret_cast<uint4*>(Xp + t * K + 32 * bl);
+    dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+    dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+    dst[2] = make_uint4(o[8], o[9], o[10], o[11]);
+    dst[3] = make_uint4(o[12], o[13], o[14], o[15]);
+}
+
+template <int NP, int BN, bool G128>
+cudaError_t launch_dec(const DecArgs& a, const void* Xp, int grid, cudaStream_t s) {
+    using C = DecCfg<NP, BN, G128>;
+    CUtensorMap map;
+    cudaError_t e = make_x_map(&map, Xp, a.K, a.T, a.K, BN);
+    if (e != cudaSuccess) return e;
+    auto kern = gemm_dec_kernel<NP, BN, G128>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, THREADS, C::SMEM_BYTES, s>>>(map, a);
+    return cudaGetLastError();
+}
+
+template <int NP, bool G128>
+cudaError_t launch_dec_np(const DecArgs& a, const void* Xp, int grid, cudaStream_t s) {
+    if (a.T <= 16) return launch_dec<NP, 16, G128>(a, Xp, grid, s);
+    if (a.T <= 32) return launch_dec<NP, 32, G128>(a, Xp, grid, s);
+    return launch_dec<NP, 64, G128>(a, Xp, grid, s);
+}
+
+}  // namespace
+
+static size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
+
+static int dec_bn(int T) { return T <= 16 ? 16 : T <= 32 ? 32 : 64; }
+
+GemmDecPlan gemm_dec_plan(int64_t M, int64_t K, int n_paths, int T, int num_sms) {
+    GemmDecPlan pl{};
+    const int64_t tiles = (M + tc::BM - 1) / tc::BM;
+    const int64_t total = tiles * (K / stage_cols(n_paths));
+    pl.tiles = tiles;
+    pl.total = total;
+    pl.grid = static_cast<int>(total < num_sms ? total : num_sms);
+    pl.bn = dec_bn(T);
+    pl.counters_bytes = align256(static_cast<size_t>(tiles) * 4);
+    pl.partials_bytes = align256(static_cast<size_t>(pl.grid) * 2 * pl.bn * tc::BM * 4);
+    pl.xp_bytes = align256(static_cast<size_t>(T) * K * 2);
+    return pl;
+}
+
+cudaError_t launch_gemm_dec(const uint32_t* planes, const void* alpha, bool alpha_f16, int64_t M, int64_t K,
+                            int n_paths, int group, bool sliced, const void* X, int64_t ldx, int T, void* Y,
+                            bool y_f16, int64_t ldy, void* workspace, const GemmDecPlan& pl, cudaStream_t s) {
+    // workspace: header | counters | partial sums | permuted X
+    char* ws = static_cast<char*>(workspace);
+    uint32_t* counters = reinterpret_cast<uint32_t*>(ws + GEMM_HEADER_BYTES);
+    float* partials = reinterpret_cast<float*>(ws + GEMM_HEADER_BYTES + pl.counters_bytes);
+    __half* Xp = reinterpret_cast<__half*>(ws + GEMM_HEADER_BYTES + pl.counters_bytes + pl.partials_bytes);
+    const int64_t nthr = (K >> 5) * T;
+    permute_x_kernel<<<static_cast<unsigned>((nthr + 255) / 256), 256, 0, s>>>(
+        static_cast<const __half*>(X), ldx, T, K, Xp);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    DecArgs a{reinterpret_cast<uint32_t*>(ws) + 1, counters, partials, planes, alpha, Y, M, K, ldy, pl.tiles,
+              pl.total, T, sliced, alpha_f16, y_f16};
+    const bool g128 = group == 128;
+    switch (n_paths) {
+        case 1: return g128 ? launch_dec_np<1, true>(a, Xp, pl.grid, s) : launch_dec_np<1, false>(a, Xp, pl.grid, s);
+        case 2: return g128 ? launch_dec_np<2, true>(a, Xp, pl.grid, s) : launch_dec_np<2, false>(a, Xp, pl.grid, s);
+        case 3: return g128 ? launch_dec_np<3, true>(a, Xp, pl.grid, s) : launch_dec_np<3, false>(a, Xp, pl.grid, s);
+        case 4: return g128 ? launch_dec_np<4, true>(a, Xp, pl.grid, s) : launch_dec_np<4, false>(a, Xp, pl.grid, s);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace rb

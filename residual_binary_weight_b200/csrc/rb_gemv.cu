@@ -353,6 +353,14 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_lut_kernel(GvArgs p, uint32_t
     }
     scan_jobs<C::R>(p, lo, n_jobs);
     const uint32_t total_units = lo.unit_prefix[n_jobs];
+    // the device descriptors must give the plan the host sized the workspace
+    // for (they are a copy the caller uploaded; a stale copy would write
+    // counters and partial sums past the workspace)
+    if (total_units != p.expect_units || lo.ctr_prefix[n_jobs] != p.expect_ctrs ||
+        lo.part_prefix[n_jobs] != p.expect_parts) {
+        if (tid == 0) atomicOr(hdr + 1, GV_ERR_BAD_JOB);
+        return;   // uniform: every thread read the same shared values
+    }
 
     // The 8 lanes sharing t8 & 3 (t8 in {a, a + 4}, 4 items) would hit the
     // same banks; lane z = (t8 >> 2) + 2 q4 swaps its two words when z is odd

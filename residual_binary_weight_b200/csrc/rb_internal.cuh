@@ -54,13 +54,18 @@ struct GvArgs {
     int chunk_slices;       // 512-column slices per K chunk
     void* workspace;
     size_t ws_bytes;
+    // the plan the host sized the workspace for; a launch whose device
+    // descriptors give another plan flags GV_ERR_BAD_JOB and does nothing
+    uint32_t expect_units, expect_ctrs, expect_parts;
 };
 
 // Workspace layout: a 256-byte header (word 1: error flags), then one
 // arrival counter per (job, row block, token) of every K-split job, then the
 // fp32 partial sums of the split jobs.
 constexpr size_t GV_HEADER_BYTES = 256;
-enum : uint32_t { GV_ERR_SMEM_LAYOUT = 1u, GV_ERR_BAD_JOB = 2u, GV_ERR_TOO_MANY_JOBS = 4u, GV_ERR_WAIT = 8u };
+// GV_ERR_BAD_JOB: the device descriptors do not give the plan the host sized
+// the workspace for (they differ from the host copy)
+enum : uint32_t { GV_ERR_SMEM_LAYOUT = 1u, GV_ERR_BAD_JOB = 2u, GV_ERR_TOO_MANY_JOBS = 4u };
 
 struct GvPlan {
     int rows_per_cta;       // R
@@ -76,12 +81,30 @@ cudaError_t launch_gemv(const GvArgs& a, const GvPlan& plan, cudaStream_t s);
 int gemv_max_jobs();
 
 // ---------------------------------------------------------------- rb_gemm
-bool gemm_supported(int n_paths, int group);
-cudaError_t launch_gemm(const uint32_t* planes, const void* alpha, bool alpha_f16, int64_t M, int64_t K, int n_paths,
-                        int group, bool sliced, const void* X, int64_t ldx, int T, void* Y, bool y_f16, int64_t ldy,
-                        cudaStream_t s);
-cudaError_t gemm_read_error(unsigned int* code);
+// Workspace: a 256-byte header (word 1: error flags of the call's kernels);
+// for decode batches (T <= GEMM_DEC_MAX_T) then the row-tile arrival
+// counters, the fp32 partial sums of tiles shared by two CTAs, and the
+// column-permuted copy of X.
+constexpr size_t GEMM_HEADER_BYTES = 256;
+constexpr int GEMM_DEC_MAX_T = 64;
+
+struct GemmDecPlan {
+    int64_t tiles, total;   // row tiles, stages (tiles * K / stage width)
+    int grid, bn;
+    size_t counters_bytes, partials_bytes, xp_bytes;
+};
+GemmDecPlan gemm_dec_plan(int64_t M, int64_t K, int n_paths, int T, int num_sms);
+cudaError_t launch_gemm_dec(const uint32_t* planes, const void* alpha, bool alpha_f16, int64_t M, int64_t K,
+                            int n_paths, int group, bool sliced, const void* X, int64_t ldx, int T, void* Y,
+                            bool y_f16, int64_t ldy, void* workspace, const GemmDecPlan& plan, cudaStream_t s);
+cudaError_t launch_gemm_prefill(const uint32_t* planes, const void* alpha, bool alpha_f16, int64_t M, int64_t K,
+                                int n_paths, int group, bool sliced, const void* X, int64_t ldx, int T, void* Y,
+                                bool y_f16, int64_t ldy, uint32_t* err, cudaStream_t s);
 
 int device_sm_count();
+
+// Device address of the static scratch array of rb_gemv_noalloc on the
+// current device (looked up once per device).
+cudaError_t noalloc_scratch(void** out);
 
 }  // namespace rb

@@ -22,10 +22,15 @@ constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void* g_scratch[kMaxDevices] = {};
 
+}  // namespace
+
+namespace rb {
+
 // The device address of the array on the current device. In host code the
 // symbol is only a host-side stand-in, so it is looked up once per device,
-// with that device current, and cached.
-cudaError_t scratch_on_current_device(void** out) {
+// with that device current, and cached. rb_gemv_check(NULL, ...) reads the
+// error word of the array through this address too.
+cudaError_t noalloc_scratch(void** out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
@@ -41,7 +46,7 @@ cudaError_t scratch_on_current_device(void** out) {
     return cudaSuccess;
 }
 
-}  // namespace
+}  // namespace rb
 
 extern "C" rb_status rb_gemv_noalloc(const uint32_t* planes, const void* alpha, rb_dtype alpha_dtype,
                                      rb_layout L, const void* x, int64_t ldx, int32_t T,
@@ -57,7 +62,7 @@ extern "C" rb_status rb_gemv_noalloc(const uint32_t* planes, const void* alpha, 
         return RB_ERR_UNSUPPORTED;
     }
     void* scratch = nullptr;
-    const cudaError_t e = scratch_on_current_device(&scratch);
+    const cudaError_t e = rb::noalloc_scratch(&scratch);
     if (e != cudaSuccess) {
         char msg[200];
         snprintf(msg, sizeof(msg), "rb_gemv_noalloc: cudaGetSymbolAddress: %s", cudaGetErrorString(e));

@@ -150,3 +150,72 @@ def test_missing_library_fails_loudly(monkeypatch):
     monkeypatch.setattr(_lib, "LIB_PATH", "/nonexistent/librb.so")
     with pytest.raises(ImportError):
         _lib.load()
+
+
+def test_grouped_checks_every_descriptor_alignment():
+    """alpha and y of every descriptor, not only the first, must be aligned
+    for their dtypes (a misaligned one would fault on the device)."""
+    lib = _lib.load()
+    p = ctypes.c_void_p
+    d = (GemvDesc * 3)()
+    for i in range(3):
+        d[i] = GemvDesc(FAKE, FAKE, FAKE, FAKE, 128, 256)
+    host = ctypes.cast(d, p)
+    args = (host, p(FAKE), 3, 2, 0, 0, 0, 1, 1, p(FAKE), 1 << 20, None)   # fp32 alpha, fp16 y
+    assert lib.rb_gemv_grouped_workspace_bytes(host, 3, 2, 1) <= 1 << 20
+    d[2] = GemvDesc(FAKE, FAKE + 2, FAKE, FAKE, 128, 256)          # fp32 alpha at +2
+    assert _status(lib.rb_gemv_grouped(*args)) == "RB_ERR_ALIGNMENT"
+    assert b"descriptor 2" in lib.rb_last_error()
+    d[2] = GemvDesc(FAKE, FAKE, FAKE, FAKE + 1, 128, 256)          # fp16 y at +1
+    assert _status(lib.rb_gemv_grouped(*args)) == "RB_ERR_ALIGNMENT"
+    assert b"descriptor 2" in lib.rb_last_error()
+    d[1] = GemvDesc(FAKE, FAKE + 2, FAKE, FAKE, 128, 256)          # fp16 alpha at +2 is fine ...
+    d[2] = GemvDesc(FAKE, FAKE, FAKE, FAKE, 128, 256)
+    args16 = (host, p(FAKE), 3, 2, 0, 0, 1, 1, 1, p(FAKE), 8, None)  # ... but the workspace is too small
+    assert _status(lib.rb_gemv_grouped(*args16)) == "RB_ERR_WORKSPACE"
+
+
+def test_gemm_rejects_bad_arguments_before_launch():
+    lib = _lib.load()
+    p = ctypes.c_void_p
+    L = Layout(256, 512, 2, 0, 0, 0)
+    ok = [p(FAKE), p(FAKE), 0, L, p(FAKE), 512, 16, p(FAKE), 1, 256, p(FAKE), 1 << 30, None]
+    names = ["planes", "alpha", "adt", "L", "X", "ldx", "T", "Y", "ydt", "ldy", "ws", "wsb", "s"]
+
+    def call(**kw):
+        args = list(ok)
+        for k, v in kw.items():
+            args[names.index(k)] = v
+        return _status(lib.rb_gemm(*args))
+
+    assert call(planes=None) == "RB_ERR_INVALID_ARG"
+    assert call(T=0) == "RB_ERR_UNSUPPORTED"
+    assert call(T=(1 << 22) + 1) == "RB_ERR_UNSUPPORTED"
+    assert call(L=Layout(256, 512, 5, 0, 0, 0)) == "RB_ERR_UNSUPPORTED"
+    # fp32 scales per 128 columns would be rounded to fp16 operands: refused
+    assert call(L=Layout(256, 512, 2, 128, 0, 0), adt=0) == "RB_ERR_UNSUPPORTED"
+    assert b"fp16 scales" in lib.rb_last_error()
+    assert call(ldx=500) == "RB_ERR_INVALID_ARG"
+    assert call(X=p(FAKE + 8)) == "RB_ERR_ALIGNMENT"
+    assert call(alpha=p(FAKE + 2)) == "RB_ERR_ALIGNMENT"
+    assert call(Y=p(FAKE + 1)) == "RB_ERR_ALIGNMENT"
+    assert call(ws=None) == "RB_ERR_WORKSPACE"
+    need = lib.rb_gemm_workspace_bytes(L, 16)
+    assert call(wsb=need - 1) == "RB_ERR_WORKSPACE"
+    assert call(ws=p(FAKE + 8)) == "RB_ERR_WORKSPACE"
+
+
+def test_gemm_workspace_sizes():
+    """Decode batches (T <= 64) need the header, one counter per 128-row tile,
+    two partial-sum slots per CTA and a permuted copy of X; prefill blocks
+    only the header."""
+    lib = _lib.load()
+    L = Layout(28672, 8192, 2, 0, 1, 0)
+    for T in (1, 16, 64):
+        b = lib.rb_gemm_workspace_bytes(L, T)
+        bn = 16 if T <= 16 else 32 if T <= 32 else 64
+        assert b >= 256 + 4 * 224 + T * 8192 * 2 + 2 * bn * 128 * 4
+    assert lib.rb_gemm_workspace_bytes(L, 65) == 256
+    assert lib.rb_gemm_workspace_bytes(L, 2048) == 256
+    assert lib.rb_gemm_workspace_bytes(L, 0) == 0
+    assert lib.rb_gemm_workspace_bytes(Layout(28672, 8000, 2, 0, 1, 0), 16) == 0

@@ -19,23 +19,15 @@ pytestmark = pytest.mark.gpu
 def _run(W, X, n_paths, group, alpha_f16, order="rows", y_dtype=torch.float16, ldx_pad=0, ldy_pad=0):
     ref_p, ref_a, _ = oracle.pack(W, n_paths, group)
     stored = oracle.alpha_to_f16(ref_a) if alpha_f16 else ref_a.astype(np.float32)
-    if group == 128 and not alpha_f16:
-        # with per-group scales the kernel multiplies by the fp16 rounding of fp32 scales
-        used = stored.astype(np.float16).astype(np.float64)
-    else:
-        used = stored.astype(np.float64)
-    y_ref, den = oracle.matvec(ref_p, used, X.astype(np.float64))
+    y_ref, den = oracle.matvec(ref_p, stored.astype(np.float64), X.astype(np.float64))
     T, K = X.shape
     M = W.shape[0]
     xt = torch.zeros((T, K + ldx_pad), dtype=torch.float16)
     xt[:, :K] = torch.from_numpy(X)
     Xd = xt.cuda()[:, :K]
     Yd = torch.full((T, M + ldy_pad), float("nan"), dtype=y_dtype, device="cuda")
-    rb.gemm(to_dev_planes(ref_p, order=order), torch.from_numpy(stored).cuda(), Xd, group=group, Y=Yd[:, :M])
-    torch.cuda.synchronize()
-    rb.load()
-    from residual_binary_weight_b200._lib import check
-    check(rb.load().rb_gemm_check(None))
+    rb.gemm(to_dev_planes(ref_p, order=order), torch.from_numpy(stored).cuda(), Xd, group=group, Y=Yd[:, :M],
+            check_device=True)
     Yh = Yd.float().cpu().numpy()
     if ldy_pad:
         assert np.all(np.isnan(Yh[:, M:])), "wrote past the row"
@@ -64,13 +56,26 @@ def test_ragged_shapes(M, K, T):
     _ok(_run(W, X, 2, 0, False, "sliced"), (M, K, T, "sliced"))
 
 
+@pytest.mark.parametrize("T", [130, 16])
 @pytest.mark.parametrize("n_paths", [1, 2, 3, 4])
-@pytest.mark.parametrize("group,alpha_f16", [(0, False), (0, True), (128, True), (128, False)])
-def test_paths_and_scales(n_paths, group, alpha_f16):
-    rng = np.random.default_rng(10 * n_paths + group)
+@pytest.mark.parametrize("group,alpha_f16", [(0, False), (0, True), (128, True)])
+def test_paths_and_scales(n_paths, group, alpha_f16, T):
+    rng = np.random.default_rng(10 * n_paths + group + T)
     W = (rng.standard_t(4, (260, 1024)) * 0.014).astype(np.float16)
-    X = rng.standard_normal((130, 1024)).astype(np.float16)
-    _ok(_run(W, X, n_paths, group, alpha_f16), (n_paths, group, alpha_f16))
+    X = rng.standard_normal((T, 1024)).astype(np.float16)
+    _ok(_run(W, X, n_paths, group, alpha_f16), (n_paths, group, alpha_f16, T))
+
+
+@pytest.mark.parametrize("T", [16, 130])
+def test_fp32_group_scales_are_refused(T):
+    """With one scale per 128 columns the scales become fp16 operand values;
+    fp32 scales would be rounded, so the call refuses them instead."""
+    rng = np.random.default_rng(3)
+    W = (rng.standard_normal((128, 256)) * 0.02).astype(np.float16)
+    ref_p, ref_a, _ = oracle.pack(W, 2, 128)
+    X = torch.from_numpy(rng.standard_normal((T, 256)).astype(np.float16)).cuda()
+    with pytest.raises(rb.RbError, match="RB_ERR_UNSUPPORTED"):
+        rb.gemm(to_dev_planes(ref_p), torch.from_numpy(ref_a.astype(np.float32)).cuda(), X, group=128)
 
 
 def test_dtypes_and_pitches():
@@ -108,15 +113,13 @@ def test_prefill_full_size_sampled(matrix):
     del W
     ref_p, ref_a, rabs = oracle.pack(Wr, 2, 0, want_rabs=True)
     rep = oracle.compare_planes(planes_np(planes[:, :, idx], spec.K), ref_p, rabs, ref_a)
-    assert rep.bad == 0, rep
+    print(f"{matrix}: {rep.flipped} allowed flips in {rep.entries} sampled entries")
+    assert rep.ok, rep
     planes[:, :, idx] = to_dev_planes(ref_p, order="sliced")
     a32 = ref_a.astype(np.float32)
     alpha[:, idx] = torch.from_numpy(a32).cuda()
     X = synth.device_activations(wl, 0, matrix, 2048, "cuda")
-    Y = rb.gemm(planes, alpha, X)
-    torch.cuda.synchronize()
-    from residual_binary_weight_b200._lib import check
-    check(rb.load().rb_gemm_check(None))
+    Y = rb.gemm(planes, alpha, X, check_device=True)
     toks = np.sort(rng.choice(2048, 48, replace=False))
     Xs = X[torch.from_numpy(toks).cuda()].cpu().numpy().astype(np.float64)
     y_ref, den = oracle.matvec(ref_p, a32.astype(np.float64), Xs)
@@ -136,11 +139,12 @@ def test_token_tile_widths(T, n_paths, group):
     _ok(_run(W, X, n_paths, group, group == 128, "sliced"), (T, n_paths, group))
 
 
-@pytest.mark.parametrize("T", [16, 64])
+@pytest.mark.parametrize("T", [1, 4, 16, 64])
 @pytest.mark.parametrize("matrix", ["attn", "up", "down"])
 def test_llama3_full_size_sampled(matrix, T):
-    """The Llama-3-70B-shaped projections at batch 16 and 64 on the tensor-core
-    path: weight drawn and packed on the device, 32 sampled rows replaced by
+    """The Llama-3-70B-shaped projections at batches 1, 4, 16 and 64 on the
+    tensor-core path (the decode-batch kernel: stream-K over all SMs, partial
+    tiles reduced through the workspace): weight drawn and packed on the device, 32 sampled rows replaced by
     the oracle's planes and scales, all tokens of those rows checked."""
     wl = synth.WORKLOADS["llama3_70b_decode"]
     spec = {m.name: m for m in wl.matrices}[matrix]
@@ -156,10 +160,7 @@ def test_llama3_full_size_sampled(matrix, T):
     a32 = ref_a.astype(np.float32)
     alpha[:, idx] = torch.from_numpy(a32).cuda()
     X = synth.device_activations(wl, 0, matrix, T, "cuda")
-    Y = rb.gemm(planes, alpha, X)
-    torch.cuda.synchronize()
-    from residual_binary_weight_b200._lib import check
-    check(rb.load().rb_gemm_check(None))
+    Y = rb.gemm(planes, alpha, X, check_device=True)
     y_ref, den = oracle.matvec(ref_p, a32.astype(np.float64), X.cpu().numpy().astype(np.float64))
     got = Y[:, idx].float().cpu().numpy()
     nbad, worst = oracle.compare_outputs(got, y_ref, den)

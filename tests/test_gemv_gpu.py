@@ -230,7 +230,8 @@ def test_full_size_layer_sampled_rows():
         Wr = W.index_select(0, idx).cpu().numpy()
         ref_p, ref_a, rabs = oracle.pack(Wr, 2, 0, want_rabs=True)
         rep = oracle.compare_planes(planes_np(planes[:, :, idx], spec.K), ref_p, rabs, ref_a)
-        assert rep.bad == 0, (spec.name, rep)
+        print(f"{spec.name}: {rep.flipped} allowed flips in {rep.entries} sampled entries")
+        assert rep.ok, (spec.name, rep)
         assert oracle.compare_scales(alpha[:, idx].cpu().numpy(), ref_a)[0] == 0
         planes[:, :, idx] = to_dev_planes(ref_p, order="sliced")
         a32 = ref_a.astype(np.float32)
@@ -279,3 +280,41 @@ def test_llama3_full_size_sampled(matrix, T):
     y_ref, den = oracle.matvec(ref_p, a32.astype(np.float64), xs)
     got = y[torch.from_numpy(toks).cuda()][:, idx].float().cpu().numpy()
     _ok(oracle.compare_outputs(got, y_ref, den), (matrix, T))
+
+
+def _qbb_full(matrix):
+    """The full QBB matrix drawn on the host, packed by the oracle; planes
+    (sliced order) and fp16 scales uploaded."""
+    wl = synth.WORKLOADS["qbb_g128"]
+    W = synth.host_weight(wl, 0, matrix)
+    ref_p, ref_a, _ = oracle.pack(W, 4, 128)
+    a16 = oracle.alpha_to_f16(ref_a)
+    return wl, ref_p, a16
+
+
+@pytest.mark.parametrize("T", [1, 16])
+def test_qbb_full_size_single_and_grouped(T):
+    """Both QBB matrices (11008 x 4096, 4096 x 11008; 4 paths, fp16 scales per
+    128 columns) at full size, every row, at batch 1 and 16: through the
+    single-matrix launch and through one grouped launch of both."""
+    items, refs = [], []
+    for matrix in ("up", "down"):
+        wl, ref_p, a16 = _qbb_full(matrix)
+        x = synth.host_activations(wl, 0, matrix, T)
+        toks = np.arange(T) if T <= 4 else np.array([0, 5, 10, 15])
+        y_ref, den = oracle.matvec(ref_p, a16.astype(np.float64), x[toks].astype(np.float64))
+        planes = to_dev_planes(ref_p, order="sliced")
+        alpha = torch.from_numpy(a16).cuda()
+        xd = torch.from_numpy(x).cuda()
+        y = rb.gemv(planes, alpha, xd, group=128, check_device=True)
+        nbad, worst = oracle.compare_outputs(y[torch.from_numpy(toks).cuda()].float().cpu().numpy(), y_ref, den)
+        assert nbad == 0, (matrix, T, worst)
+        yg = torch.full((T, ref_p.shape[1]), float("nan"), dtype=torch.float16, device="cuda")
+        items.append((planes, alpha, xd, yg))
+        refs.append((toks, y_ref, den))
+    g = rb.GroupedGemv(items, n_paths=4, group=128, T=T)
+    g.run()
+    g.check_device_flag()
+    for (_, _, _, yg), (toks, y_ref, den) in zip(items, refs):
+        nbad, worst = oracle.compare_outputs(yg[torch.from_numpy(toks).cuda()].float().cpu().numpy(), y_ref, den)
+        assert nbad == 0, (T, worst)

@@ -54,6 +54,8 @@ def test_noalloc_matches_workspace_entry_point():
         assert nbad == 0, (call, worst)
         nbad, worst = oracle.compare_outputs(got, y_ref, den)
         assert nbad == 0, (call, worst)
+        # no kernel-side failure recorded in the static scratch
+        assert lib.rb_gemv_check(None, stream) == 0, lib.rb_last_error()
 
 
 def _shape_beyond_scratch(lib):
