@@ -4,12 +4,17 @@ One step = one decode token through 32 layers x 7 linears (q, k, v, o, gate,
 up, down; 224 matrices, 6.48e9 weights, 2 residual paths with one fp32 scale
 per row) = one persistent rb_gemv_grouped launch that streams 1.635 GB of
 packed planes. Synthetic seeded weights drawn on the device and packed with
-rb_pack once before timing; activations are refreshed every step.
+rb_pack once before timing; the device-timed steps reuse the resident
+activations, the e2e leg copies them from pinned host memory every step.
 
 Metric: achieved HBM GB/s of that launch (algorithmic bytes: planes + scales
 + x + y), with the fraction of the measured copy bandwidth. The JSON line also
-carries the one-time rb_pack throughput and, when the library has it, rb_gemm
-TFLOP/s on the 2048-token prefill block.
+carries, under "parts": rb_gemm TFLOP/s on the 2048-token prefill block (the
+metric's second half, with cuBLAS fp16 on the dense equivalent as context),
+rb_pack GB/s, the 70B-shaped projections at T = 1, 4, 16, 64 and the QBB
+layout at T = 1, 16 (matvec and tensor path, roofline fractions), each as
+the median / p10 / p90 over CUDA-graph replays of the time per call, and a
+read-only streaming ceiling for context.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
@@ -167,79 +172,153 @@ def build_stack(torch, rb, synth, device, layers=32):
     return items, xbuf, ybuf, alg_bytes
 
 
-def _graph_time_us(torch, fn, n=20):
-    """Device time of fn() replayed from a CUDA graph (no host overhead between
-    launches); fn must only enqueue work on the current stream."""
+def time_calls_us(torch, fn, calls=20, replays=15):
+    """Device time per call of fn(i) (i = call index): `calls` calls captured
+    into one CUDA graph (so no host gaps sit between them), the graph replayed
+    `replays` times, each replay bracketed by CUDA events on the current
+    stream. Returns (median, p10, p90) over the replays of the time per call,
+    in microseconds. fn may only enqueue work on the current stream."""
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(side):
-        for _ in range(3):
-            fn()
+        for i in range(3):
+            fn(i)
     torch.cuda.current_stream().wait_stream(side)
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
-        fn()
-    for _ in range(3):
+        for i in range(calls):
+            fn(i)
+    for _ in range(2):
         graph.replay()
     torch.cuda.synchronize()
-    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s.record()
-    for _ in range(n):
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(replays)]
+    for a, b in ev:
+        a.record()
         graph.replay()
-    e.record()
+        b.record()
     torch.cuda.synchronize()
-    us = s.elapsed_time(e) / n * 1e3
+    t = sorted(a.elapsed_time(b) * 1e3 / calls for a, b in ev)
     del graph
-    return us
+    q = lambda f: t[min(len(t) - 1, int(f * (len(t) - 1) + 0.5))]
+    return q(0.5), q(0.1), q(0.9)
 
 
-def time_pack(torch, rb, synth, device):
-    """rb_pack on the 7B gate matrix (2 paths, per-row scales) and on the QBB
-    up matrix (4 paths, fp16 scales per 128 columns)."""
+def _copies_for(nbytes: int, budget: int = 512 << 20) -> int:
+    """Distinct copies to rotate through so that one pass over them moves at
+    least 4x the 126 MB L2 (consecutive calls then read from HBM)."""
+    return max(2, -(-budget // max(nbytes, 1)))
+
+
+def _stats(us, p10, p90):
+    return {"us": round(us, 2), "p10_us": round(p10, 2), "p90_us": round(p90, 2)}
+
+
+def time_pack(torch, rb, synth, device, hbm_peak):
+    """rb_pack on the 7B gate matrix (2 paths, per-row scales) and on both QBB
+    matrices (4 paths, fp16 scales per 128 columns); W is 90-180 MB, larger
+    than L2, and the same W is packed on every call (pack reads it once)."""
     out = {}
-    for wl_name, name, n_paths, group in (("llama2_7b_decode", "gate", 2, 0), ("qbb_g128", "up", 4, 128)):
+    for wl_name, name, n_paths, group in (("llama2_7b_decode", "gate", 2, 0), ("qbb_g128", "up", 4, 128),
+                                          ("qbb_g128", "down", 4, 128)):
         wl = synth.WORKLOADS[wl_name]
         W = synth.device_weight(wl, 0, name, device)
         M, K = W.shape
         a16 = group == 128
-        us = _graph_time_us(torch, lambda: rb.pack(W, n_paths, group, alpha_f16=a16))
         G = K if group == 0 else group
+        planes, alpha, al16 = rb.pack(W, n_paths, group, alpha_f16=a16)   # output buffers, reused below
+        us, p10, p90 = time_calls_us(torch, lambda i: rb.pack(W, n_paths, group, alpha_f16=a16, planes=planes,
+                                                              alpha=alpha, alpha16=al16))
         b = M * K * W.element_size() + n_paths * M * K // 8 + n_paths * M * (K // G) * (4 + (2 if a16 else 0))
-        out[f"{wl_name}/{name}"] = {"shape": [M, K], "n_paths": n_paths, "group": group, "us": round(us, 2),
-                                   "GB/s": round(b / us / 1e3, 1), "bytes": b}
-        del W
+        out[f"{wl_name}/{name}"] = dict(_stats(us, p10, p90), shape=[M, K], n_paths=n_paths, group=group,
+                                        bytes=b, **{"GB/s": round(b / us / 1e3, 1),
+                                                    "frac_of_hbm": round(b / us / 1e3 / hbm_peak, 3)})
+        del W, planes, alpha, al16
     return out
 
 
 def time_gemm(torch, rb, synth, device, peak_tf):
-    lib = rb.load()
-    if not hasattr(lib, "rb_gemm"):
-        return None
+    """rb_gemm on the 2048-token prefill block (second headline of the metric),
+    with cuBLAS fp16 torch.matmul on the dense equivalent as context."""
     wl = synth.WORKLOADS["prefill"]
     out = {}
     for name in ("up", "down"):
         sp = {m.name: m for m in wl.matrices}[name]
         W = synth.device_weight(wl, 0, name, device)
         planes, alpha, _ = rb.pack(W, 2, 0, order="sliced")
+        Wd = W.to(torch.float16)
         del W
         X = synth.device_activations(wl, 0, name, 2048, device)
         Y = torch.empty((2048, sp.M), dtype=torch.float16, device=device)
-        for _ in range(3):
-            rb.gemm(planes, alpha, X, Y=Y)
-        torch.cuda.synchronize()
-        n = 10
-        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s.record()
-        for _ in range(n):
-            rb.gemm(planes, alpha, X, Y=Y)
-        e.record()
-        torch.cuda.synchronize()
-        ms = s.elapsed_time(e) / n
+        ws = torch.empty(max(16, rb.gemm_workspace_bytes(sp.M, sp.K, 2, 0, 2048)), dtype=torch.uint8, device=device)
+        us, p10, p90 = time_calls_us(torch, lambda i: rb.gemm(planes, alpha, X, Y=Y, workspace=ws), calls=10,
+                                     replays=10)
+        rb.gemm(planes, alpha, X, Y=Y, workspace=ws, check_device=True)
         flops = 2.0 * 2 * 2048 * sp.M * sp.K
-        tf = flops / ms / 1e9
-        out[name] = {"shape": [sp.M, sp.K], "T": 2048, "us": round(ms * 1e3, 1), "TFLOP/s": round(tf, 1),
-                     "frac_of_bf16_peak": round(tf / peak_tf, 3) if peak_tf else None}
+        tf = flops / us / 1e6
+        Yd = torch.empty((2048, sp.M), dtype=torch.float16, device=device)
+        cu, _, _ = time_calls_us(torch, lambda i: torch.matmul(X, Wd.t(), out=Yd), calls=10, replays=10)
+        out[name] = dict(_stats(us, p10, p90), shape=[sp.M, sp.K], T=2048, **{
+            "TFLOP/s": round(tf, 1), "frac_of_bf16_peak": round(tf / peak_tf, 3) if peak_tf else None,
+            "cublas_fp16_dense_us": round(cu, 1),
+            "cublas_fp16_dense_TFLOP/s": round(2.0 * 2048 * sp.M * sp.K / cu / 1e6, 1),
+            "flops_counted": "2 * paths * T * M * K (one +-1 contraction per path)"})
+        del planes, alpha, Wd, X, Y, Yd
     return out
+
+
+def time_decode_shapes(torch, rb, synth, device, hbm_peak, tf_peak, wl_name, batches, n_paths, group):
+    """Decode batches on one matrix at a time (the 70B-shaped projections at
+    T = 1, 4, 16, 64; the QBB layout at T = 1, 16): the CUDA-core matvec and
+    the tensor-core rb_gemm, each with its roofline fraction:
+    max(bytes / HBM peak, 2 N T M K / tensor peak) / measured time. Enough
+    packed copies are rotated that every call reads its planes from HBM."""
+    wl = synth.WORKLOADS[wl_name]
+    out = {}
+    for sp in wl.matrices:
+        W = synth.device_weight(wl, 0, sp.name, device)
+        a16 = group == 128
+        planes, alpha, al16 = rb.pack(W, n_paths, group, alpha_f16=a16, order="sliced")
+        del W
+        sc = al16 if a16 else alpha
+        nbytes = planes.numel() * 4 + sc.numel() * sc.element_size()
+        copies = [(planes, sc)] + [(planes.clone(), sc.clone()) for _ in range(_copies_for(nbytes) - 1)]
+        rows = {}
+        for T in batches:
+            X = synth.device_activations(wl, 0, sp.name, T, device)
+            Y = torch.empty((T, sp.M), dtype=torch.float16, device=device)
+            wsv = torch.empty(max(16, rb.gemv_workspace_bytes(sp.M, sp.K, n_paths, group, T)), dtype=torch.uint8,
+                              device=device)
+            wsg = torch.empty(max(16, rb.gemm_workspace_bytes(sp.M, sp.K, n_paths, group, T)), dtype=torch.uint8,
+                              device=device)
+            nc = len(copies)
+            v = time_calls_us(torch, lambda i: rb.gemv(copies[i % nc][0], copies[i % nc][1], X, group=group, y=Y,
+                                                      workspace=wsv))
+            g = time_calls_us(torch, lambda i: rb.gemm(copies[i % nc][0], copies[i % nc][1], X, group=group, Y=Y,
+                                                      workspace=wsg))
+            rb.gemm(planes, sc, X, group=group, Y=Y, workspace=wsg, check_device=True)
+            rb.gemv(planes, sc, X, group=group, y=Y, workspace=wsv, check_device=True)
+            bytes_ = n_paths * sp.M * sp.K // 8 + sc.numel() * sc.element_size() + T * sp.K * 2 + T * sp.M * 2
+            flops = 2.0 * n_paths * T * sp.M * sp.K
+            t_bound = max(bytes_ / (hbm_peak * 1e3), flops / (tf_peak * 1e6))   # us
+            best = "rb_gemv" if v[0] <= g[0] else "rb_gemm"
+            bu = min(v[0], g[0])
+            rows[f"T{T}"] = {"rb_gemv": _stats(*v), "rb_gemm": _stats(*g), "best": best, "best_us": round(bu, 2),
+                             "bytes": bytes_, "GB/s": round(bytes_ / bu / 1e3, 1),
+                             "bound": "hbm" if bytes_ / (hbm_peak * 1e3) >= flops / (tf_peak * 1e6) else "tensor",
+                             "roofline_us": round(t_bound, 2), "roofline_frac": round(t_bound / bu, 3)}
+        out[f"{sp.name} {sp.M}x{sp.K}"] = rows
+        del copies, planes, alpha, al16
+    return out
+
+
+def read_ceiling_gbs(torch, device):
+    """Context: a plain streaming read of 4 GiB (torch.sum over fp32 words) --
+    the HBM read rate a library reduction reaches on this GPU."""
+    buf = torch.ones(1 << 30, dtype=torch.float32, device=device)
+    out = torch.empty((), dtype=torch.float32, device=device)
+    us, _, _ = time_calls_us(torch, lambda i: torch.sum(buf, dtype=torch.float32, out=out), calls=4, replays=5)
+    del buf
+    return {"GB/s": round((4 << 30) / us / 1e3, 1), "how": "torch.sum over 4 GiB of fp32 (read only)"}
 
 
 def oracle_sample_inputs(rows_per: int = 96):
@@ -417,10 +496,13 @@ def run_gpu(args):
 
     parts = {}
     if rank == 0 and not args.no_parts:
-        parts["rb_pack"] = time_pack(torch, rb, synth, device)
-        gm = time_gemm(torch, rb, synth, device, bf16_peak)
-        if gm is not None:
-            parts["rb_gemm_prefill"] = gm
+        parts["read_ceiling"] = read_ceiling_gbs(torch, device)
+        parts["rb_pack"] = time_pack(torch, rb, synth, device, hbm_peak)
+        parts["rb_gemm_prefill"] = time_gemm(torch, rb, synth, device, bf16_peak)
+        parts["llama3_70b_decode"] = time_decode_shapes(torch, rb, synth, device, hbm_peak, bf16_peak,
+                                                        "llama3_70b_decode", (1, 4, 16, 64), 2, 0)
+        parts["qbb_g128_decode"] = time_decode_shapes(torch, rb, synth, device, hbm_peak, bf16_peak,
+                                                      "qbb_g128", (1, 16), 4, 128)
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu:
