@@ -316,7 +316,7 @@ def read_ceiling_gbs(torch, device):
     the HBM read rate a library reduction reaches on this GPU."""
     buf = torch.ones(1 << 30, dtype=torch.float32, device=device)
     out = torch.empty((), dtype=torch.float32, device=device)
-    us, _, _ = time_calls_us(torch, lambda i: torch.sum(buf, dtype=torch.float32, out=out), calls=4, replays=5)
+    us, _, _ = time_calls_us(torch, lambda i: torch.sum(buf, dim=0, out=out), calls=4, replays=5)
     del buf
     return {"GB/s": round((4 << 30) / us / 1e3, 1), "how": "torch.sum over 4 GiB of fp32 (read only)"}
 

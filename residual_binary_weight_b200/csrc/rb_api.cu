@@ -265,7 +265,7 @@ rb_status rb_gemv_grouped(const rb_gemv_desc* descs_host, const rb_gemv_desc* de
 size_t rb_gemm_workspace_bytes(rb_layout L, int32_t T) {
     if (check_layout(L) != RB_OK || T < 1) return 0;
     if (T > GEMM_DEC_MAX_T) return GEMM_HEADER_BYTES;
-    const GemmDecPlan pl = gemm_dec_plan(L.M, L.K, L.n_paths, T, device_sm_count());
+    const GemmDecPlan pl = gemm_dec_plan(L.M, L.K, L.n_paths, L.group, T, device_sm_count());
     return GEMM_HEADER_BYTES + pl.counters_bytes + pl.partials_bytes + pl.xp_bytes;
 }
 
@@ -292,7 +292,7 @@ rb_status rb_gemm(const uint32_t* planes, const void* alpha, rb_dtype alpha_dtyp
     GemmDecPlan pl{};
     size_t need = GEMM_HEADER_BYTES, clear = GEMM_HEADER_BYTES;
     if (dec) {
-        pl = gemm_dec_plan(L.M, L.K, L.n_paths, T, device_sm_count());
+        pl = gemm_dec_plan(L.M, L.K, L.n_paths, L.group, T, device_sm_count());
         need += pl.counters_bytes + pl.partials_bytes + pl.xp_bytes;
         clear += pl.counters_bytes;
     }

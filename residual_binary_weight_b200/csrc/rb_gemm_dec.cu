@@ -45,6 +45,8 @@
 // word and the CTA winds down after draining what it issued.
 #include "rb_tc.cuh"
 
+#include <cuda_fp8.h>
+
 #include <type_traits>
 
 namespace rb {
@@ -71,29 +73,36 @@ struct DecArgs {
     bool sliced, alpha_f16, y_f16;
 };
 
-__host__ __device__ constexpr int stage_cols(int np) { return np <= 2 ? 128 : 64; }
+__host__ __device__ constexpr int stage_cols(int np, bool f8) { return f8 ? 256 : np <= 2 ? 128 : 64; }
 
-template <int NP, int BN, bool G128>
+// F8: fp8 operands (kind::f8f6f4): the weights as e4m3 +-1, X as four
+// scaled e5m2 terms (TERMS rows per token, see split_x_f8_kernel),
+// 256-column stages.
+template <int NP, int BN, bool G128, bool F8>
 struct DecCfg {
-    static constexpr int SW = stage_cols(NP);             // K columns per stage
+    static constexpr int SW = stage_cols(NP, F8);         // K columns per stage
     static constexpr int WPS = SW / 32;                    // plane words per row, path and stage
-    static constexpr int SUB = SW / BK;                    // 64-column X boxes per stage
+    static constexpr int TERMS = F8 ? 4 : 1;               // B rows per token
+    static constexpr int NMMA = TERMS * BN;                // MMA N
+    static constexpr int SUB = F8 ? SW / 128 : SW / BK;    // 128-byte X boxes per stage
     static constexpr int NACC = G128 ? 1 : NP;             // accumulators per buffer
-    static constexpr int ACC_STRIDE = BN;                  // 16, 32 or 64 columns
-    static constexpr int A_STAGE_COLS = NP * SW / 2;       // fp16 pairs of all paths of one stage
+    static constexpr int ACC_STRIDE = NMMA;                // MMA N: 16, 32 or 64 columns
+    static constexpr int COLS_PER_WORD = F8 ? 8 : 16;      // tensor-memory columns of one plane word
+    static constexpr int A_STAGE_COLS = NP * WPS * COLS_PER_WORD;
     // two accumulator buffers (the epilogue of one tile overlaps the next
     // tile's MMAs) when that still leaves three operand stages
     static constexpr int ACC_BUF = (512 - 2 * NACC * ACC_STRIDE) / A_STAGE_COLS >= 3 ? 2 : 1;
     static constexpr int ACC_COLS = ACC_BUF * NACC * ACC_STRIDE;
     static constexpr int STAGES_FIT = (512 - ACC_COLS) / A_STAGE_COLS;
     static constexpr int STAGES = STAGES_FIT < 8 ? STAGES_FIT : 8;
-    static constexpr uint32_t SUB_BYTES = BN * BK * 2;     // one 64-column box of BN rows
+    static constexpr uint32_t SUB_BYTES = NMMA * 128;      // one 128-byte-wide box of NMMA rows
     static constexpr uint32_t B_TILE_BYTES = SUB * SUB_BYTES;
     static constexpr uint32_t SMEM_USED = STAGES * B_TILE_BYTES + 1024 /*align*/ + 512 /*barriers*/;
     // at least 120 KB, so that two CTAs never share an SM's tensor memory
     static constexpr uint32_t SMEM_BYTES = SMEM_USED < 120u * 1024u ? 120u * 1024u : SMEM_USED;
     static_assert(STAGES >= 2, "operand stages do not fit beside the accumulators");
-    static_assert(BN == 16 || BN == 32 || BN == 64, "token tile");
+    static_assert(F8 ? (BN == 4 || BN == 8 || BN == 16) : (BN == 16 || BN == 32 || BN == 64), "token tile");
+    static_assert(!F8 || (!G128 && NP <= 2), "fp8 operands: per-row scales, 1-2 paths");
     static_assert(SUB_BYTES % 1024 == 0, "X box must keep the 1024-byte swizzle alignment");
 };
 
@@ -101,10 +110,10 @@ struct DecCfg {
 __device__ __forceinline__ int64_t range_lo(int64_t c, int64_t total, int64_t G) { return c * total / G; }
 __device__ __forceinline__ int64_t cta_of(int64_t g, int64_t total, int64_t G) { return ((g + 1) * G - 1) / total; }
 
-template <int NP, int BN, bool G128>
+template <int NP, int BN, bool G128, bool F8>
 __global__ void __launch_bounds__(THREADS, 1)
 gemm_dec_kernel(const __grid_constant__ CUtensorMap xmap, DecArgs a) {
-    using C = DecCfg<NP, BN, G128>;
+    using C = DecCfg<NP, BN, G128, F8>;
     constexpr int STAGES = C::STAGES, ACC_BUF = C::ACC_BUF, SW = C::SW, WPS = C::WPS;
     extern __shared__ __align__(1024) unsigned char dsm[];
     const uint32_t raw = smem_addr(dsm);
@@ -121,7 +130,9 @@ gemm_dec_kernel(const __grid_constant__ CUtensorMap xmap, DecArgs a) {
     volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(dsm + (abort_slot - raw));
     volatile uint32_t* last_flag = reinterpret_cast<volatile uint32_t*>(dsm + (last_slot - raw));
     auto b_tile = [&](int s) { return tiles_s + static_cast<uint32_t>(s) * C::B_TILE_BYTES; };
-    auto a_col = [&](int s, int p) { return static_cast<uint32_t>(C::ACC_COLS + (s * NP + p) * (SW / 2)); };
+    auto a_col = [&](int s, int p) {
+        return static_cast<uint32_t>(C::ACC_COLS + (s * NP + p) * (WPS * C::COLS_PER_WORD));
+    };
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t M = a.M, K = a.K, S = K / SW, total = a.total, G = gridDim.x, me = blockIdx.x;
@@ -157,8 +168,10 @@ gemm_dec_kernel(const __grid_constant__ CUtensorMap xmap, DecArgs a) {
             if (elect_one()) {
                 mbar_arrive_expect_tx(full_bar(s), C::B_TILE_BYTES);
 #pragma unroll
-                for (int u = 0; u < C::SUB; ++u)
-                    tma_load_2d(b_tile(s) + u * C::SUB_BYTES, &xmap, kb * SW + u * BK, 0, full_bar(s));
+                for (int u = 0; u < C::SUB; ++u) {
+                    if (F8) tma_load_3d(b_tile(s) + u * C::SUB_BYTES, &xmap, kb * SW + u * 128, 0, 0, full_bar(s));
+                    else tma_load_2d(b_tile(s) + u * C::SUB_BYTES, &xmap, kb * SW + u * BK, 0, full_bar(s));
+                }
             }
             __syncwarp();
             issued = i + 1;
@@ -173,7 +186,7 @@ gemm_dec_kernel(const __grid_constant__ CUtensorMap xmap, DecArgs a) {
                 mbar_drain(full_bar(static_cast<int>(i % STAGES)), static_cast<uint32_t>(i / STAGES) & 1u);
     } else if (warp == MMA_WARP) {
         // ---------------------------------------------------------------- MMA
-        constexpr uint32_t idesc = instr_desc(BN);
+        constexpr uint32_t idesc = F8 ? instr_desc_f8(C::NMMA) : instr_desc(BN);
         int st = 0;          // stage slot and phase of the next stage
         uint32_t sph = 0;
         int j = 0;           // segment counter
@@ -205,13 +218,15 @@ gemm_dec_kernel(const __grid_constant__ CUtensorMap xmap, DecArgs a) {
 #pragma unroll
                 for (int p = 0; p < NP; ++p) {
                     const uint32_t d = dbase + static_cast<uint32_t>(G128 ? 0 : p * C::ACC_STRIDE);
+                    // one MMA per 32 bytes of K (16 fp16 or 32 fp8 columns):
+                    // box kk / 4, and +32 bytes inside a swizzled box is +2
+                    // in the descriptor's address field
 #pragma unroll
-                    for (int kk = 0; kk < SW / 16; ++kk) {
-                        // 64-column box kk / 4; +32 bytes along K inside a
-                        // swizzled box is +2 in the descriptor's address field
+                    for (int kk = 0; kk < WPS * C::COLS_PER_WORD / 8; ++kk) {
                         const uint64_t bd = bd0 + ((kk >> 2) * C::SUB_BYTES >> 4) + 2u * (kk & 3);
                         const uint32_t acc = (kk > 0 || (G128 && p > 0)) ? 1u : acc0;
-                        umma_f16_ta_elect(d, tmem_base + a_col(s, p) + 8u * kk, bd, idesc, acc);
+                        if (F8) umma_f8_ta_elect(d, tmem_base + a_col(s, p) + 8u * kk, bd, idesc, acc);
+                        else umma_f16_ta_elect(d, tmem_base + a_col(s, p) + 8u * kk, bd, idesc, acc);
                     }
                 }
                 umma_commit_elect(empty_bar(s));
@@ -231,22 +246,25 @@ gemm_dec_kernel(const __grid_constant__ CUtensorMap xmap, DecArgs a) {
         const uint32_t W32 = static_cast<uint32_t>(K >> 5), SL = static_cast<uint32_t>((K + 511) >> 9);
         const uint32_t gpr = static_cast<uint32_t>(K >> 7);
         const uint32_t path_words = a.sliced ? SL * uM * 16u : uM * W32;   // < 2^30 (checked by the host)
-        using WV = typename std::conditional<WPS == 4, uint4, uint2>::type;
-        constexpr int PR = NP <= 2 ? 4 : 2;   // stages of this group loaded ahead
+        using WV = typename std::conditional<WPS == 2, uint2, uint4>::type;
+        constexpr int NV = WPS == 2 ? 1 : WPS / 4;   // vector loads per path and stage
+        constexpr int PR = F8 ? 2 : NP <= 2 ? 4 : 2;   // stages of this group loaded ahead
         const int64_t n = hi - lo;
         // (tile, stage-in-tile) of the next stage to load, stepping by 2
         int64_t lt = (lo + grp) / S;
         int lkb = static_cast<int>(lo + grp - lt * S);
-        WV ring[PR][NP];
+        WV ring[PR][NP][NV];
         uint32_t nring[PR][NP];
-        auto load_stage = [&](WV (&dst)[NP], uint32_t (&ndst)[NP]) {
+        auto load_stage = [&](WV (&dst)[NP][NV], uint32_t (&ndst)[NP]) {
             const int64_t row64 = lt * BM + r;
             const uint32_t row = static_cast<uint32_t>(row64 < M ? row64 : M - 1);   // rows past M read a real row
             const uint32_t w = static_cast<uint32_t>(lkb) * WPS;
             const uint32_t off = a.sliced ? ((w >> 4) * uM + row) * 16u + (w & 15u) : row * W32 + w;
 #pragma unroll
             for (int p = 0; p < NP; ++p) {
-                dst[p] = __ldg(reinterpret_cast<const WV*>(a.planes + static_cast<size_t>(p) * path_words + off));
+#pragma unroll
+                for (int v = 0; v < NV; ++v)
+                    dst[p][v] = __ldg(reinterpret_cast<const WV*>(a.planes + static_cast<size_t>(p) * path_words + off) + v);
                 if (G128) {
                     const uint32_t g = static_cast<uint32_t>(lkb) * SW / 128u;
                     const uint32_t hv = static_cast<const unsigned short*>(a.alpha)[(p * uM + row) * gpr + g] | 0x8000u;
@@ -261,16 +279,34 @@ gemm_dec_kernel(const __grid_constant__ CUtensorMap xmap, DecArgs a) {
                 ++lt;
             }
         };
-        // +-v pairs of one plane word into 16 tensor-memory columns
+        // fp16: +-v pairs of one plane word into 16 tensor-memory columns
         auto expand_store = [&](uint32_t w, uint32_t ng, uint32_t col) {
             uint32_t h[16];
 #pragma unroll
             for (int k = 0; k < 16; ++k) h[k] = ((w << (15 - k)) & 0x80008000u) ^ ng;
             tmem_store16(tmem_base + lane_q + col, h);
         };
-        auto word = [](const WV& v, int i) -> uint32_t {
-            if constexpr (WPS == 4) return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
-            else return i == 0 ? v.x : v.y;
+        // fp8: two plane words into 16 tensor-memory columns of e4m3 +-1.
+        // The columns of X'' are ordered so that byte b of column r of a
+        // word holds column 8b + r: shifting left by 7 - r puts bits r,
+        // 8 + r, 16 + r, 24 + r at the four byte sign bits, and xor with
+        // four e4m3 -1.0 (0xB8) gives +1.0 (0x38) where the bit is set.
+        auto expand_store8 = [&](uint32_t w0, uint32_t w1, uint32_t col) {
+            uint32_t h[16];
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                h[r] = ((w0 << (7 - r)) & 0x80808080u) ^ 0xB8B8B8B8u;
+                h[8 + r] = ((w1 << (7 - r)) & 0x80808080u) ^ 0xB8B8B8B8u;
+            }
+            tmem_store16(tmem_base + lane_q + col, h);
+        };
+        auto word = [](const WV (&v)[NV], int i) -> uint32_t {
+            if constexpr (WPS == 2) return i == 0 ? v[0].x : v[0].y;
+            else {
+                const uint4& u = v[i >> 2];
+                const int j = i & 3;
+                return j == 0 ? u.x : j == 1 ? u.y : j == 2 ? u.z : u.w;
+            }
         };
 #pragma unroll
         for (int d = 0; d < PR; ++d)
@@ -283,11 +319,12 @@ gemm_dec_kernel(const __grid_constant__ CUtensorMap xmap, DecArgs a) {
             for (int d = 0; d < PR; ++d) {
                 const int64_t i = i0 + 2 * d;
                 if (i < n && go) {
-                    WV cur[NP];
+                    WV cur[NP][NV];
                     uint32_t ng[NP];
 #pragma unroll
                     for (int p = 0; p < NP; ++p) {
-                        cur[p] = ring[d][p];
+#pragma unroll
+                        for (int v = 0; v < NV; ++v) cur[p][v] = ring[d][p][v];
                         ng[p] = nring[d][p];
                     }
                     if (i + 2 * PR < n) load_stage(ring[d], nring[d]);
@@ -296,9 +333,17 @@ gemm_dec_kernel(const __grid_constant__ CUtensorMap xmap, DecArgs a) {
                         go = false;
                     } else {
 #pragma unroll
-                        for (int p = 0; p < NP; ++p)
+                        for (int p = 0; p < NP; ++p) {
+                            if constexpr (F8) {
 #pragma unroll
-                            for (int wi = 0; wi < WPS; ++wi) expand_store(word(cur[p], wi), ng[p], a_col(s, p) + 16u * wi);
+                                for (int wi = 0; wi < WPS; wi += 2)
+                                    expand_store8(word(cur[p], wi), word(cur[p], wi + 1), a_col(s, p) + 8u * wi);
+                            } else {
+#pragma unroll
+                                for (int wi = 0; wi < WPS; ++wi)
+                                    expand_store(word(cur[p], wi), ng[p], a_col(s, p) + 16u * wi);
+                            }
+                        }
                         tmem_store_wait();
                         fence_before();
                         __syncwarp();
@@ -347,7 +392,9 @@ gemm_dec_kernel(const __grid_constant__ CUtensorMap xmap, DecArgs a) {
                                              : static_cast<const float*>(a.alpha)[p * M + crow];
                 }
                 // CW token columns at a time: sum_k alpha_k acc_k, then Y or
-                // the partial-sum slot of this CTA
+                // the partial-sum slot of this CTA. With one chunk (BN <= 32)
+                // the accumulator buffer is released before the stores, so
+                // the next tile's MMAs need not wait for them.
 #pragma unroll 1
                 for (int c0 = 0; c0 < BN; c0 += CW) {
                     float yv[CW];
@@ -355,11 +402,26 @@ gemm_dec_kernel(const __grid_constant__ CUtensorMap xmap, DecArgs a) {
                     for (int c = 0; c < CW; ++c) yv[c] = 0.0f;
 #pragma unroll
                     for (int p = 0; p < C::NACC; ++p) {
-                        uint32_t v[CW];
-                        tmem_load<CW>(tmem_base + lane_q +
-                                          static_cast<uint32_t>((b * C::NACC + p) * C::ACC_STRIDE + c0), v);
+                        // token c0 + c of term m sits at column m * BN + c0 + c
+                        float acc[CW];
 #pragma unroll
-                        for (int c = 0; c < CW; ++c) yv[c] = fmaf(al[p], __uint_as_float(v[c]), yv[c]);
+                        for (int c = 0; c < CW; ++c) acc[c] = 0.0f;
+#pragma unroll
+                        for (int m = 0; m < C::TERMS; ++m) {
+                            uint32_t v[CW];
+                            tmem_load<CW>(tmem_base + lane_q +
+                                              static_cast<uint32_t>((b * C::NACC + p) * C::ACC_STRIDE + m * BN + c0), v);
+                            const float wm = F8 ? 1.0f / static_cast<float>(1 << (2 * m)) : 1.0f;   // 4^-m
+#pragma unroll
+                            for (int c = 0; c < CW; ++c) acc[c] = fmaf(wm, __uint_as_float(v[c]), acc[c]);
+                        }
+#pragma unroll
+                        for (int c = 0; c < CW; ++c) yv[c] = fmaf(al[p], acc[c], yv[c]);
+                    }
+                    if (CW == BN) {
+                        fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(acc_empty(b));   // the buffer may take the next tile
                     }
 #pragma unroll
                     for (int c = 0; c < CW; ++c) {
@@ -368,9 +430,11 @@ gemm_dec_kernel(const __grid_constant__ CUtensorMap xmap, DecArgs a) {
                     }
                 }
             }
-            fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(acc_empty(b));   // the buffer may take the next tile
+            if (!ok || CW != BN) {
+                fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(acc_empty(b));   // the buffer may take the next tile
+            }
             if (full) continue;
             // partial tile: the same sequence of named barriers whatever happened
             const int64_t first = cta_of(t * S, total, G), last = cta_of((t + 1) * S - 1, total, G);
@@ -444,13 +508,64 @@ __global__ void permute_x_kernel(const __half* __restrict__ X, int64_t ldx, int 
     dst[3] = make_uint4(o[12], o[13], o[14], o[15]);
 }
 
-template <int NP, int BN, bool G128>
+// X'' for the fp8 operands: every fp16 value x is written as four e5m2
+// terms, each the rounding of the previous residual scaled by 4:
+//   s1 = RN(x), s2 = RN(4 (x - s1)), s3 = RN(4 (4 (x - s1) - s2)), ...
+// so that x = s1 + s2/4 + s3/16 + s4/64 + e. e5m2 has the exponent range of
+// fp16 and 3 significant bits, each residual is at most 2^-3 of the value it
+// was taken from, and the scaled residuals are exact in fp16 and stay below
+// |x| / 2 (no overflow): |e| <= 2^-12 |x| + 2^-23, and e = 0 for every normal
+// fp16 x (4 x 3 bits cover its 11). The epilogue weights the accumulators of
+// the four terms by 1, 1/4, 1/16, 1/64. Layout: [term][token][K] bytes, and
+// inside every 32-column block byte 4r + b holds column 8b + r (the order
+// the fp8 expansion produces). One thread per (token, block).
+__global__ void split_x_f8_kernel(const __half* __restrict__ X, int64_t ldx, int T, int64_t K,
+                                  uint8_t* __restrict__ Xq) {
+    const int64_t blocks = K >> 5;
+    const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (idx >= blocks * T) return;
+    const int64_t t = idx / blocks, bl = idx - t * blocks;
+    const uint4* src = reinterpret_cast<const uint4*>(X + t * ldx + 32 * bl);
+    __half res[32];
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+        const uint4 u = __ldg(src + v);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            __half2_raw h2;
+            h2.x = static_cast<unsigned short>(w[i] & 0xFFFFu);
+            h2.y = static_cast<unsigned short>(w[i] >> 16);
+            res[8 * v + 2 * i] = __half(__half_raw{h2.x});
+            res[8 * v + 2 * i + 1] = __half(__half_raw{h2.y});
+        }
+    }
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        uint32_t q[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+            const __nv_fp8_storage_t b8 = __nv_cvt_halfraw_to_fp8(static_cast<__half_raw>(res[c]), __NV_SATFINITE, __NV_E5M2);
+            q[c] = b8;
+            if (m < 3)   // exact: the residual and its product with 4
+                res[c] = __hmul(__hsub(res[c], __half(__nv_cvt_fp8_to_halfraw(b8, __NV_E5M2))), __float2half(4.0f));
+        }
+        uint32_t o[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) o[r] = q[r] | (q[8 + r] << 8) | (q[16 + r] << 16) | (q[24 + r] << 24);
+        uint4* dst = reinterpret_cast<uint4*>(Xq + (static_cast<int64_t>(m) * T + t) * K + 32 * bl);
+        dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+        dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+    }
+}
+
+template <int NP, int BN, bool G128, bool F8>
 cudaError_t launch_dec(const DecArgs& a, const void* Xp, int grid, cudaStream_t s) {
-    using C = DecCfg<NP, BN, G128>;
+    using C = DecCfg<NP, BN, G128, F8>;
     CUtensorMap map;
-    cudaError_t e = make_x_map(&map, Xp, a.K, a.T, a.K, BN);
+    cudaError_t e = F8 ? make_x8_map(&map, Xp, a.K, a.T, 4, BN) : make_x_map(&map, Xp, a.K, a.T, a.K, BN);
     if (e != cudaSuccess) return e;
-    auto kern = gemm_dec_kernel<NP, BN, G128>;
+    auto kern = gemm_dec_kernel<NP, BN, G128, F8>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     kern<<<grid, THREADS, C::SMEM_BYTES, s>>>(map, a);
@@ -458,29 +573,48 @@ cudaError_t launch_dec(const DecArgs& a, const void* Xp, int grid, cudaStream_t 
 }
 
 template <int NP, bool G128>
-cudaError_t launch_dec_np(const DecArgs& a, const void* Xp, int grid, cudaStream_t s) {
-    if (a.T <= 16) return launch_dec<NP, 16, G128>(a, Xp, grid, s);
-    if (a.T <= 32) return launch_dec<NP, 32, G128>(a, Xp, grid, s);
-    return launch_dec<NP, 64, G128>(a, Xp, grid, s);
+cudaError_t launch_dec_np(const DecArgs& a, const void* Xp, int grid, bool f8, cudaStream_t s) {
+    if constexpr (NP <= 2 && !G128) {
+        if (f8) {
+            if (a.T <= 4) return launch_dec<NP, 4, false, true>(a, Xp, grid, s);
+            if (a.T <= 8) return launch_dec<NP, 8, false, true>(a, Xp, grid, s);
+            return launch_dec<NP, 16, false, true>(a, Xp, grid, s);
+        }
+    }
+    if (a.T <= 16) return launch_dec<NP, 16, G128, false>(a, Xp, grid, s);
+    if (a.T <= 32) return launch_dec<NP, 32, G128, false>(a, Xp, grid, s);
+    return launch_dec<NP, 64, G128, false>(a, Xp, grid, s);
 }
 
 }  // namespace
 
 static size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
 
-static int dec_bn(int T) { return T <= 16 ? 16 : T <= 32 ? 32 : 64; }
+// tokens per tile: fp16 operands 16/32/64; fp8 operands 4/8/16 (x 4 terms)
+static int dec_bn(int T, bool f8) {
+    if (f8) return T <= 4 ? 4 : T <= 8 ? 8 : 16;
+    return T <= 16 ? 16 : T <= 32 ? 32 : 64;
+}
 
-GemmDecPlan gemm_dec_plan(int64_t M, int64_t K, int n_paths, int T, int num_sms) {
+// fp8 operands for T <= 16 tokens with one or two paths and per-row scales
+// (the scales stay out of the operands), when K splits into 256-column stages
+static bool dec_f8(int64_t K, int n_paths, int group, int T) {
+    return T <= 16 && n_paths <= 2 && group == 0 && K % 256 == 0;
+}
+
+GemmDecPlan gemm_dec_plan(int64_t M, int64_t K, int n_paths, int group, int T, int num_sms) {
     GemmDecPlan pl{};
+    const bool f8 = dec_f8(K, n_paths, group, T);
     const int64_t tiles = (M + tc::BM - 1) / tc::BM;
-    const int64_t total = tiles * (K / stage_cols(n_paths));
+    const int64_t total = tiles * (K / stage_cols(n_paths, f8));
     pl.tiles = tiles;
     pl.total = total;
     pl.grid = static_cast<int>(total < num_sms ? total : num_sms);
-    pl.bn = dec_bn(T);
+    pl.bn = dec_bn(T, f8);
+    pl.f8 = f8;
     pl.counters_bytes = align256(static_cast<size_t>(tiles) * 4);
     pl.partials_bytes = align256(static_cast<size_t>(pl.grid) * 2 * pl.bn * tc::BM * 4);
-    pl.xp_bytes = align256(static_cast<size_t>(T) * K * 2);
+    pl.xp_bytes = align256(static_cast<size_t>(T) * K * (f8 ? 4 : 2));
     return pl;
 }
 
@@ -493,18 +627,26 @@ cudaError_t launch_gemm_dec(const uint32_t* planes, const void* alpha, bool alph
     float* partials = reinterpret_cast<float*>(ws + GEMM_HEADER_BYTES + pl.counters_bytes);
     __half* Xp = reinterpret_cast<__half*>(ws + GEMM_HEADER_BYTES + pl.counters_bytes + pl.partials_bytes);
     const int64_t nthr = (K >> 5) * T;
-    permute_x_kernel<<<static_cast<unsigned>((nthr + 255) / 256), 256, 0, s>>>(
-        static_cast<const __half*>(X), ldx, T, K, Xp);
+    if (pl.f8)
+        split_x_f8_kernel<<<static_cast<unsigned>((nthr + 127) / 128), 128, 0, s>>>(
+            static_cast<const __half*>(X), ldx, T, K, reinterpret_cast<uint8_t*>(Xp));
+    else
+        permute_x_kernel<<<static_cast<unsigned>((nthr + 255) / 256), 256, 0, s>>>(
+            static_cast<const __half*>(X), ldx, T, K, Xp);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     DecArgs a{reinterpret_cast<uint32_t*>(ws) + 1, counters, partials, planes, alpha, Y, M, K, ldy, pl.tiles,
               pl.total, T, sliced, alpha_f16, y_f16};
     const bool g128 = group == 128;
     switch (n_paths) {
-        case 1: return g128 ? launch_dec_np<1, true>(a, Xp, pl.grid, s) : launch_dec_np<1, false>(a, Xp, pl.grid, s);
-        case 2: return g128 ? launch_dec_np<2, true>(a, Xp, pl.grid, s) : launch_dec_np<2, false>(a, Xp, pl.grid, s);
-        case 3: return g128 ? launch_dec_np<3, true>(a, Xp, pl.grid, s) : launch_dec_np<3, false>(a, Xp, pl.grid, s);
-        case 4: return g128 ? launch_dec_np<4, true>(a, Xp, pl.grid, s) : launch_dec_np<4, false>(a, Xp, pl.grid, s);
+        case 1: return g128 ? launch_dec_np<1, true>(a, Xp, pl.grid, pl.f8, s)
+                     : launch_dec_np<1, false>(a, Xp, pl.grid, pl.f8, s);
+        case 2: return g128 ? launch_dec_np<2, true>(a, Xp, pl.grid, pl.f8, s)
+                     : launch_dec_np<2, false>(a, Xp, pl.grid, pl.f8, s);
+        case 3: return g128 ? launch_dec_np<3, true>(a, Xp, pl.grid, pl.f8, s)
+                     : launch_dec_np<3, false>(a, Xp, pl.grid, pl.f8, s);
+        case 4: return g128 ? launch_dec_np<4, true>(a, Xp, pl.grid, pl.f8, s)
+                     : launch_dec_np<4, false>(a, Xp, pl.grid, pl.f8, s);
     }
     return cudaErrorInvalidValue;
 }

@@ -91,9 +91,10 @@ constexpr int GEMM_DEC_MAX_T = 64;
 struct GemmDecPlan {
     int64_t tiles, total;   // row tiles, stages (tiles * K / stage width)
     int grid, bn;
+    bool f8;                // fp8 operands with X split into four e5m2 terms
     size_t counters_bytes, partials_bytes, xp_bytes;
 };
-GemmDecPlan gemm_dec_plan(int64_t M, int64_t K, int n_paths, int T, int num_sms);
+GemmDecPlan gemm_dec_plan(int64_t M, int64_t K, int n_paths, int group, int T, int num_sms);
 cudaError_t launch_gemm_dec(const uint32_t* planes, const void* alpha, bool alpha_f16, int64_t M, int64_t K,
                             int n_paths, int group, bool sliced, const void* X, int64_t ldx, int T, void* Y,
                             bool y_f16, int64_t ldy, void* workspace, const GemmDecPlan& plan, cudaStream_t s);

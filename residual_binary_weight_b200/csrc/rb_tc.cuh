@@ -153,6 +153,24 @@ __device__ __forceinline__ void umma_f16_ta_elect(uint32_t d_tmem, uint32_t a_tm
         ::"r"(d_tmem), "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
 
+// kind::f8f6f4 (fp8 A from tensor memory, fp8 B from shared memory, K = 32)
+__device__ __forceinline__ void umma_f8_ta_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                                 uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+// kind::f8f6f4 instruction descriptor: fp32 accumulator, A e4m3, B e5m2,
+// both K-major, M = 128, N = n
+__host__ __device__ constexpr uint32_t instr_desc_f8(int n) {
+    return (1u << 4) | (0u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
+           (static_cast<uint32_t>(BM >> 4) << 24);
+}
+
 __device__ __forceinline__ void umma_commit_elect(uint32_t bar) {
     asm volatile(
         "{\n\t.reg .pred e;\n\t"
@@ -222,6 +240,23 @@ __device__ __forceinline__ void tmem_load<16>(uint32_t taddr, uint32_t (&v)[16])
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+template <>
+__device__ __forceinline__ void tmem_load<8>(uint32_t taddr, uint32_t (&v)[8]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+template <>
+__device__ __forceinline__ void tmem_load<4>(uint32_t taddr, uint32_t (&v)[4]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3])
+                 : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
 __device__ __forceinline__ void tmem_alloc(uint32_t slot, uint32_t cols) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot), "r"(cols)
                  : "memory");
@@ -230,6 +265,15 @@ __device__ __forceinline__ void tmem_alloc(uint32_t slot, uint32_t cols) {
 
 __device__ __forceinline__ void tmem_dealloc(uint32_t base, uint32_t cols) {
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(base), "r"(cols) : "memory");
+}
+
+// TMA load of one 3-D box of a tensor map into shared memory; completes by
+// transaction bytes on `bar` (no multicast)
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
+        ::"r"(dst), "l"(map), "r"(x), "r"(y), "r"(z), "r"(bar)
+        : "memory");
 }
 
 // TMA load of one 2-D tile of a tensor map into shared memory; completes by
@@ -253,5 +297,9 @@ EncodeTiledFn encode_fn();
 // Tensor map of a row-major fp16 [rows][ld] matrix with `cols` valid columns,
 // read in boxes of 64 columns x box_rows rows with the 128-byte swizzle.
 cudaError_t make_x_map(CUtensorMap* map, const void* X, int64_t cols, int64_t rows, int64_t ld, int box_rows);
+
+// Tensor map of a byte array [terms][rows][cols] (dense), read in boxes of
+// 128 bytes x box_rows rows x terms with the 128-byte swizzle.
+cudaError_t make_x8_map(CUtensorMap* map, const void* X, int64_t cols, int64_t rows, int terms, int box_rows);
 
 }  // namespace rb
