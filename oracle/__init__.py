@@ -46,6 +46,10 @@ def _load():
             lib.rbo_pack.restype = ctypes.c_int
             lib.rbo_matvec.argtypes = [p, p, i64, i64, i32, i64, p, i64, p, p]
             lib.rbo_matvec.restype = ctypes.c_int
+            lib.rbo_pack_fixed.argtypes = [p, i64, i64, i32, p, p, p, p]
+            lib.rbo_pack_fixed.restype = ctypes.c_int
+            lib.rbo_dual_matvec.argtypes = [p, p, i64, i64, i32, p, i64, p, p]
+            lib.rbo_dual_matvec.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -92,6 +96,65 @@ def matvec(planes: np.ndarray, alpha: np.ndarray, x: np.ndarray):
     y = np.zeros((T, M), dtype=np.float64)
     den = np.zeros((T, M), dtype=np.float64)
     rc = _load().rbo_matvec(_ptr(planes), _ptr(alpha), M, K, N, G, _ptr(x), T, _ptr(y), _ptr(den))
+    if rc != 0:
+        raise ValueError("bad shape")
+    return y, den
+
+
+def pack_fixed(W: np.ndarray, h: np.ndarray, g: np.ndarray | None = None, want_rabs: bool = False):
+    """Sign planes of the dual-scale block for given scales (RaBiT 4.1-4.2).
+
+    W (M, K); h (N, M) output-channel scales; g (N, K) input-channel scales or
+    None (all ones). R_0 = W, B_k = sign(R_{k-1}),
+    R_k = R_{k-1} - h_k[i] g_k[j] B_k. Returns (planes uint32 [N, M, K/32],
+    rabs float64 [N, M, K] or None).
+    """
+    W = np.ascontiguousarray(W, dtype=np.float64)
+    M, K = W.shape
+    h = np.ascontiguousarray(h, dtype=np.float64)
+    N = h.shape[0]
+    if h.shape != (N, M):
+        raise ValueError("h must be (N, M)")
+    if g is not None:
+        g = np.ascontiguousarray(g, dtype=np.float64)
+        if g.shape != (N, K):
+            raise ValueError("g must be (N, K)")
+    planes = np.zeros((N, M, K // 32), dtype=np.uint32)
+    rabs = np.zeros((N, M, K), dtype=np.float64) if want_rabs else None
+    rc = _load().rbo_pack_fixed(_ptr(W), M, K, N, _ptr(h), _ptr(g) if g is not None else None, _ptr(planes),
+                                _ptr(rabs) if rabs is not None else None)
+    if rc != 0:
+        raise ValueError(f"bad shape M={M} K={K} N={N}")
+    return planes, rabs
+
+
+def dual_inputs(g: np.ndarray | None, x: np.ndarray, n_paths: int) -> np.ndarray:
+    """x_k = g_k (.) x rounded to the nearest fp16 (the activation the binary
+    core of path k sees): [N, T, K] float64 holding fp16 values."""
+    x = np.atleast_2d(np.asarray(x, dtype=np.float64))
+    if g is None:
+        g = np.ones((n_paths, x.shape[1]))
+    g = np.asarray(g, dtype=np.float64)
+    return (g[:, None, :] * x[None, :, :]).astype(np.float16).astype(np.float64)
+
+
+def dual_matvec(planes: np.ndarray, h: np.ndarray, xk: np.ndarray):
+    """y[t, i] = sum_k h_k[i] sum_j (+-1) xk[k, t, j] and its tolerance scale.
+
+    planes uint32 [N, M, K/32]; h [N, M]; xk [N, T, K] (from dual_inputs).
+    Returns (y float64 [T, M], denom float64 [T, M]).
+    """
+    planes = np.ascontiguousarray(planes, dtype=np.uint32)
+    h = np.ascontiguousarray(h, dtype=np.float64)
+    xk = np.ascontiguousarray(xk, dtype=np.float64)
+    N, M, W32 = planes.shape
+    K = W32 * 32
+    T = xk.shape[1]
+    if h.shape != (N, M) or xk.shape != (N, T, K):
+        raise ValueError("shape mismatch")
+    y = np.zeros((T, M), dtype=np.float64)
+    den = np.zeros((T, M), dtype=np.float64)
+    rc = _load().rbo_dual_matvec(_ptr(planes), _ptr(h), M, K, N, _ptr(xk), T, _ptr(y), _ptr(den))
     if rc != 0:
         raise ValueError("bad shape")
     return y, den

@@ -27,6 +27,22 @@
  *               fp64 sum of +x_j / -x_j, with no masked-sum identity, so it is
  *               independent of the way the kernels evaluate it.
  *
+ *  rbo_pack_fixed -- the same sequential derivation with scales the caller
+ *               gives instead of mean |R|: RaBiT section 4.1 ("dual-scale"
+ *               binary cores with per-channel output and input scaling
+ *               vectors, W^_k = diag(h_k) B_k diag(g_k)) and section 4.2
+ *               (paths derived in turn from the shared weight, scales
+ *               learned). Signs only: B_k = sign(R_{k-1}),
+ *               R_k[i][j] = R_{k-1}[i][j] - h_k[i] g_k[j] B_k[i][j].
+ *
+ *  rbo_dual_matvec -- the dual-scale block's output
+ *               y = sum_k h_k (.) (B_k (g_k (.) x)), RaBiT section 4.1, with
+ *               g_k (.) x taken as an fp16 activation (A16): each product is
+ *               rounded to the nearest fp16 before the binary core sees it
+ *               (a reading; the pages do not say in which precision the
+ *               input vector is applied). Direct fp64 sum of +-x, as in
+ *               rbo_matvec.
+ *
  * Bit layout (a reading; RaBiT appendix D only says 32 columns go into one
  * uint32): bit j of word w of a row holds column 32*w + j, and a set bit
  * means +1. Planes are stored [N][M][K/32].
@@ -123,6 +139,68 @@ int rbo_matvec(const uint32_t* planes, const double* alpha, int64_t M, int64_t K
                     const int bit = (int)((row[j / 32] >> (j % 32)) & 1u);
                     acc += bit ? a * xv : -(a * xv);
                     den += fabs(a * xv);
+                }
+            }
+            y[t * M + i] = acc;
+            if (denom) denom[t * M + i] = den;
+        }
+    }
+    return 0;
+}
+
+/*
+ * W      : M x K weights as doubles, row-major.
+ * h      : N x M output-channel scales (h_k[i] >= 0).
+ * g      : N x K input-channel scales, or NULL for all ones.
+ * planes : out, N*M*(K/32) words.
+ * rabs   : out (nullable), N*M*K values |R_{k-1}[i][j]|.
+ */
+int rbo_pack_fixed(const double* W, int64_t M, int64_t K, int32_t N, const double* h, const double* g,
+                   uint32_t* planes, double* rabs) {
+    if (M < 0 || K <= 0 || N < 1 || K % 32 != 0) return -1;
+    const int64_t words = K / 32;
+    memset(planes, 0, sizeof(uint32_t) * (size_t)(N * M * words));
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t i = 0; i < M; ++i) {
+        for (int64_t j = 0; j < K; ++j) {
+            double r = W[i * K + j];   /* R_0 = W */
+            for (int32_t k = 0; k < N; ++k) {
+                const double scale = h[(int64_t)k * M + i] * (g ? g[(int64_t)k * K + j] : 1.0);
+                if (rabs) rabs[((int64_t)k * M + i) * K + j] = fabs(r);
+                /* B_k = sign(R_{k-1}), sign(0) = +1 */
+                const double b = (r >= 0.0) ? 1.0 : -1.0;
+                if (b > 0.0) planes[((int64_t)k * M + i) * words + j / 32] |= (uint32_t)1u << (j % 32);
+                /* R_k = R_{k-1} - h_k[i] g_k[j] B_k */
+                r = r - scale * b;
+            }
+        }
+    }
+    return 0;
+}
+
+/*
+ * planes : N*M*(K/32) words.   h : N x M.   g : N x K (NULL: all ones).
+ * xk     : N x T x K, the fp16-rounded products g_k[j] * x_t[j] (the caller
+ *          rounds them; see the header comment), as doubles.
+ * y      : out, T x M.  denom : out (nullable), T x M values
+ *          sum_k sum_j |h_k[i] * xk[k][t][j]|, the tolerance scale.
+ */
+int rbo_dual_matvec(const uint32_t* planes, const double* h, int64_t M, int64_t K, int32_t N,
+                    const double* xk, int64_t T, double* y, double* denom) {
+    if (M < 0 || K <= 0 || N < 1 || K % 32 != 0 || T < 0) return -1;
+    const int64_t words = K / 32;
+#pragma omp parallel for collapse(2) schedule(dynamic, 16)
+    for (int64_t t = 0; t < T; ++t) {
+        for (int64_t i = 0; i < M; ++i) {
+            double acc = 0.0, den = 0.0;
+            for (int32_t k = 0; k < N; ++k) {
+                const uint32_t* row = planes + ((int64_t)k * M + i) * words;
+                const double hk = h[(int64_t)k * M + i];
+                const double* xr = xk + ((int64_t)k * T + t) * K;
+                for (int64_t j = 0; j < K; ++j) {
+                    const int bit = (int)((row[j / 32] >> (j % 32)) & 1u);
+                    acc += bit ? hk * xr[j] : -(hk * xr[j]);
+                    den += fabs(hk * xr[j]);
                 }
             }
             y[t * M + i] = acc;

@@ -451,3 +451,88 @@ def test_alpha_to_f16_bit_patterns():
     want = [0x3555, 0x2E66, 0x7BFF, 0x0001, 0x3C00, 0x3C02, 0x3C01]
     got = oracle.alpha_to_f16(vals).view(np.uint16).tolist()
     assert got == want, [hex(g) for g in got]
+
+
+# ---------------------------------------------------------------- dual-scale block
+def test_pack_fixed_hand_worked_row():
+    """tests/golden/fixed_scales.txt: words and |R_{k-1}| of a 4-path row with
+    given output scales h and input scales g."""
+    rows = list(_golden_lines("fixed_scales.txt"))
+    assert len(rows) == 4
+    W = np.repeat([3.0, -1.0], 16)[None, :]
+    h = np.array([[float(r[1])] for r in rows])
+    g = np.array([np.repeat([float(v) for v in r[2].split(",")], 16) for r in rows])
+    planes, rabs = oracle.pack_fixed(W, h, g, want_rabs=True)
+    for k, (_, _, _, word, ra) in enumerate(rows):
+        assert int(planes[k, 0, 0]) == int(word, 16), k
+        assert np.array_equal(rabs[k, 0], np.repeat([float(v) for v in ra.split(",")], 16)), k
+
+
+@pytest.mark.parametrize("group", [0, 128])
+def test_pack_fixed_with_mean_abs_scales_is_pack(group):
+    """Given the scales the analytical derivation computes (mean |R|, g = 1),
+    the fixed-scale derivation takes the same signs (pinned pack above)."""
+    rng = np.random.default_rng(41)
+    W = rng.standard_normal((12, 256)) * 0.02
+    planes, alpha, _ = oracle.pack(W, 3, 0)
+    pf, _ = oracle.pack_fixed(W, alpha[:, :, 0])
+    assert np.array_equal(pf, planes)
+    pf1, _ = oracle.pack_fixed(W, alpha[:, :, 0], np.ones((3, 256)))
+    assert np.array_equal(pf1, planes)
+
+
+def test_pack_fixed_energy_identity():
+    """R_k = R_{k-1} - h g B with B = sign(R_{k-1}) gives, per row,
+    sum R_k^2 = sum R_{k-1}^2 - 2 h sum g |R_{k-1}| + h^2 sum g^2 (R B = |R|):
+    a dropped term, a wrong sign or a transposed g fails it."""
+    rng = np.random.default_rng(42)
+    M, K, N = 10, 192, 3
+    W = rng.standard_normal((M, K))
+    h = rng.uniform(0.1, 1.0, (N, M))
+    g = rng.uniform(0.2, 2.0, (N, K))
+    planes, rabs = oracle.pack_fixed(W, h, g, want_rabs=True)
+    S = _signs(planes)
+    R = W.copy()
+    for k in range(N):
+        assert np.allclose(np.abs(R), rabs[k], rtol=0, atol=1e-12)
+        assert np.array_equal(S[k], np.where(R >= 0, 1.0, -1.0))
+        Rn = R - h[k][:, None] * g[k][None, :] * S[k]
+        lhs = (Rn ** 2).sum(1)
+        rhs = (R ** 2).sum(1) - 2 * h[k] * (g[k][None, :] * np.abs(R)).sum(1) + h[k] ** 2 * (g[k] ** 2).sum()
+        assert np.allclose(lhs, rhs, rtol=1e-12)
+        R = Rn
+
+
+def test_dual_inputs_round_to_fp16():
+    """x_k = RN_fp16(g_k x): 1/3 * 1 -> 0x3555, 0.1 * 1 -> 0x2E66, 3 * (1/3 in fp64) -> 1.0."""
+    g = np.array([[1 / 3, 0.1, 3.0]])
+    x = np.array([[1.0, 1.0, 1 / 3]])
+    xk = oracle.dual_inputs(g, x, 1)
+    assert xk.astype(np.float16).view(np.uint16).tolist() == [[[0x3555, 0x2E66, 0x3C00]]]
+
+
+def test_dual_matvec_against_blas_and_single_scale_matvec():
+    rng = np.random.default_rng(43)
+    M, K, N, T = 20, 256, 2, 3
+    W = rng.standard_normal((M, K))
+    h = rng.uniform(0.1, 1.0, (N, M))
+    g = rng.uniform(0.2, 2.0, (N, K))
+    planes, _ = oracle.pack_fixed(W, h, g)
+    x = rng.standard_normal((T, K)).astype(np.float16).astype(np.float64)
+    xk = oracle.dual_inputs(g, x, N)
+    y, den = oracle.dual_matvec(planes, h, xk)
+    S = _signs(planes)
+    ref = sum(xk[k] @ (h[k][:, None] * S[k]).T for k in range(N))
+    assert np.allclose(y, ref, rtol=0, atol=1e-12 * den.max())
+    assert np.allclose(den, sum(np.abs(xk[k]) @ np.repeat(h[k][:, None], K, 1).T for k in range(N)), rtol=1e-12)
+    # g = 1: the dual block is the single-scale layer with alpha_k = h_k (pinned matvec)
+    y1, den1 = oracle.dual_matvec(planes, h, oracle.dual_inputs(None, x, N))
+    y2, den2 = oracle.matvec(planes, h[:, :, None], x)
+    assert np.allclose(y1, y2, rtol=0, atol=1e-12 * den2.max()) and np.allclose(den1, den2, rtol=1e-13)
+    # x = e_j reads column j of sum_k h_k B_k g_k (with g_k[j] rounded as an fp16 activation)
+    for j in (0, 100, 255):
+        e = np.zeros((1, K))
+        e[0, j] = 1.0
+        ye, _ = oracle.dual_matvec(planes, h, oracle.dual_inputs(g, e, N))
+        col = sum(h[k] * S[k][:, j] * float(np.float16(g[k, j])) for k in range(N))
+        assert np.allclose(ye[0], col, rtol=0, atol=1e-14)
