@@ -227,6 +227,47 @@ RB_API size_t rb_gemm_workspace_bytes(rb_layout L, int32_t T);
 RB_API rb_status rb_gemm_check(const void* workspace, void* stream);
 
 /*
+ * rb_pack_fixed -- the sign planes of the dual-scale binary block for scales
+ * the caller gives (RaBiT section 4.1: binary cores with per-channel output
+ * and input scaling vectors, W^_k = diag(h_k) B_k diag(g_k); section 4.2:
+ * paths derived in turn from the shared weight, scales learned). Signs only:
+ *     R_0 = W;  for k = 1..N:  B_k = sign(R_{k-1})  (sign(0) = +1),
+ *     R_k[i][j] = R_{k-1}[i][j] - h_k[i] g_k[j] B_k[i][j].
+ * Arithmetic: residuals in fp32, h_k[i] g_k[j] rounded to fp32 once.
+ *
+ * W       device, as rb_pack (fp16 or fp32, pitch ldw, 16-byte aligned).
+ * L       group must be 0 (the scales are per row and per column).
+ * h       device, fp32 [N][M] output-channel scales, 4-byte aligned.
+ * g       device, fp32 [N][K] input-channel scales, or NULL for all ones.
+ * planes  device, out, rb_planes_words(L) words in L.order.
+ * Errors: as rb_pack; RB_ERR_UNSUPPORTED for group != 0.
+ */
+RB_API rb_status rb_pack_fixed(const void* W, rb_dtype w_dtype, int64_t ldw, rb_layout L, const float* h,
+                               const float* g, uint32_t* planes, void* stream);
+
+/*
+ * rb_dual_gemv -- the dual-scale block's output for T <= 64 tokens,
+ *     y_t = sum_k h_k (.) (B_k x_{k,t}),   x_{k,t} = RN_fp16(g_k (.) x_t)
+ * (RaBiT section 4.1). The input scaling is taken as an fp16 activation (the
+ * A16 reading): each product g_k[j] x_t[j] is rounded to the nearest fp16
+ * (from its exact value) before the binary core sees it. Runs the CUDA-core
+ * table matvec once per path (one grouped launch; alpha = h_k), then sums
+ * the paths in fp32.
+ *
+ * planes  device, rb_planes_words(L) words in L.order (group 0).
+ * h, g    device fp32 scales as in rb_pack_fixed (g may be NULL).
+ * x, y    as rb_gemv (x fp16 [T][ldx]; y [T][ldy] of y_dtype).
+ * workspace  device scratch of rb_dual_gemv_workspace_bytes(L, T) bytes,
+ *         16-byte aligned, not shared by calls that may overlap on the GPU;
+ *         its header's error word is read by rb_gemv_check(workspace, s).
+ */
+RB_API rb_status rb_dual_gemv(const uint32_t* planes, rb_layout L, const float* h, const float* g, const void* x,
+                              int64_t ldx, int32_t T, void* y, rb_dtype y_dtype, int64_t ldy, void* workspace,
+                              size_t ws_bytes, void* stream);
+
+RB_API size_t rb_dual_gemv_workspace_bytes(rb_layout L, int32_t T);
+
+/*
  * rb_gemv_noalloc -- rb_gemv for callers that cannot allocate device memory.
  * (An addition of this library; the paper has no counterpart.) Some callers
  * have no way to obtain a workspace: code that runs where cudaMalloc is not

@@ -14,15 +14,17 @@ library's CUDA kernels.
 from ._lib import RbError, load  # noqa: F401
 from .api import (  # noqa: F401
     GroupedGemv,
+    dual_gemv,
     gemm,
     gemm_workspace_bytes,
     gemv,
     gemv_workspace_bytes,
     layout,
     pack,
+    pack_fixed,
     planes_words,
     scales_count,
 )
 
-__all__ = ["pack", "gemv", "gemm", "GroupedGemv", "layout", "planes_words", "scales_count",
+__all__ = ["pack", "pack_fixed", "gemv", "dual_gemv", "gemm", "GroupedGemv", "layout", "planes_words", "scales_count",
            "gemv_workspace_bytes", "gemm_workspace_bytes", "RbError", "load"]

@@ -23,7 +23,8 @@ RB_ROWS, RB_SLICED = 0, 1
 EXPORTED = ("rb_planes_words", "rb_scales_count", "rb_status_string", "rb_last_error",
             "rb_pack", "rb_gemv", "rb_gemv_workspace_bytes", "rb_gemv_grouped",
             "rb_gemv_grouped_workspace_bytes", "rb_gemv_check", "rb_gemv_noalloc",
-            "rb_gemm", "rb_gemm_workspace_bytes", "rb_gemm_check")
+            "rb_gemm", "rb_gemm_workspace_bytes", "rb_gemm_check",
+            "rb_pack_fixed", "rb_dual_gemv", "rb_dual_gemv_workspace_bytes")
 
 
 class RbError(RuntimeError):
@@ -87,6 +88,12 @@ def load() -> ctypes.CDLL:
         lib.rb_gemm_workspace_bytes.restype = sz
         lib.rb_gemm_check.argtypes = [vp, vp]
         lib.rb_gemm_check.restype = st
+        lib.rb_pack_fixed.argtypes = [vp, st, i64, Layout, vp, vp, vp, vp]
+        lib.rb_pack_fixed.restype = st
+        lib.rb_dual_gemv.argtypes = [vp, Layout, vp, vp, vp, i64, i32, vp, st, i64, vp, sz, vp]
+        lib.rb_dual_gemv.restype = st
+        lib.rb_dual_gemv_workspace_bytes.argtypes = [Layout, i32]
+        lib.rb_dual_gemv_workspace_bytes.restype = sz
         _lib = lib
         return lib
 

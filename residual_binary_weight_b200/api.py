@@ -244,3 +244,57 @@ def gemm(planes: torch.Tensor, alpha: torch.Tensor, X: torch.Tensor, group: int 
         if check_device:
             check(lib.rb_gemm_check(_p(workspace), _stream(dev)))
     return Y
+
+
+def pack_fixed(W: torch.Tensor, h: torch.Tensor, g: Optional[torch.Tensor] = None, order: str = "rows",
+               planes: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Sign planes of the dual-scale block for given scales: h fp32 [N, M]
+    (output channels), g fp32 [N, K] (input channels) or None.
+    B_k = sign(R_{k-1}), R_k = R_{k-1} - h_k[i] g_k[j] B_k."""
+    lib = _lib.load()
+    dev = _require_cuda(W, h, g, planes)
+    if W.dim() != 2 or W.stride(1) != 1 or W.dtype not in _DT:
+        raise ValueError("W must be a 2-D fp16/fp32 tensor with unit column stride")
+    M, K = W.shape
+    N = h.shape[0]
+    if h.shape != (N, M) or h.dtype != torch.float32 or not h.is_contiguous():
+        raise ValueError("h must be contiguous fp32 [N, M]")
+    if g is not None and (g.shape != (N, K) or g.dtype != torch.float32 or not g.is_contiguous()):
+        raise ValueError("g must be contiguous fp32 [N, K]")
+    shape = (N, M, K // 32) if order == "rows" else (N, (K + 511) // 512, M, 16)
+    if planes is None:
+        planes = torch.empty(shape, dtype=torch.int32, device=dev)
+    elif tuple(planes.shape) != shape or planes.dtype != torch.int32 or not planes.is_contiguous():
+        raise ValueError(f"planes must be contiguous int32 of shape {shape}")
+    with torch.cuda.device(dev):
+        check(lib.rb_pack_fixed(_p(W), _DT[W.dtype], W.stride(0), layout(M, K, N, 0, order), _p(h), _p(g),
+                                _p(planes), _stream(dev)))
+    return planes
+
+
+def dual_gemv(planes: torch.Tensor, h: torch.Tensor, g: Optional[torch.Tensor], x: torch.Tensor,
+              y: Optional[torch.Tensor] = None, y_dtype: torch.dtype = torch.float16,
+              workspace: Optional[torch.Tensor] = None, check_device: bool = False) -> torch.Tensor:
+    """y[t] = sum_k h_k (.) (B_k RN_fp16(g_k (.) x[t])) for T <= 64 tokens."""
+    lib = _lib.load()
+    x = _x2d(x)
+    dev = _require_cuda(planes, h, g, x, y, workspace)
+    K = x.shape[1]
+    N, M, order = _planes_geometry(planes, K)
+    T = x.shape[0]
+    if h.shape != (N, M) or h.dtype != torch.float32 or not h.is_contiguous():
+        raise ValueError("h must be contiguous fp32 [N, M]")
+    if g is not None and (g.shape != (N, K) or g.dtype != torch.float32 or not g.is_contiguous()):
+        raise ValueError("g must be contiguous fp32 [N, K]")
+    if y is None:
+        y = torch.empty((T, M), dtype=y_dtype, device=dev)
+    L = layout(M, K, N, 0, order)
+    need = lib.rb_dual_gemv_workspace_bytes(L, T)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        check(lib.rb_dual_gemv(_p(planes), L, _p(h), _p(g), _p(x), x.stride(0), T, _p(y), _DT[y.dtype], y.stride(0),
+                               _p(workspace), workspace.numel() * workspace.element_size(), _stream(dev)))
+        if check_device:
+            check(lib.rb_gemv_check(_p(workspace), _stream(dev)))
+    return y

@@ -262,6 +262,54 @@ rb_status rb_gemv_grouped(const rb_gemv_desc* descs_host, const rb_gemv_desc* de
     return RB_OK;
 }
 
+rb_status rb_pack_fixed(const void* W, rb_dtype w_dtype, int64_t ldw, rb_layout L, const float* h, const float* g,
+                        uint32_t* planes, void* stream) {
+    g_last_error.clear();
+    rb_status st = check_layout(L);
+    if (st != RB_OK) return st;
+    if (!W || !h || !planes) return fail(RB_ERR_INVALID_ARG, "null W, h or planes");
+    if (L.group != 0) return fail(RB_ERR_UNSUPPORTED, "given scales are per row (h) and per column (g): group must be 0");
+    if (!valid_dtype(w_dtype)) return fail(RB_ERR_INVALID_ARG, "bad w_dtype %d", (int)w_dtype);
+    if (ldw < L.K) return fail(RB_ERR_INVALID_ARG, "ldw=%lld < K=%lld", (long long)ldw, (long long)L.K);
+    if (!aligned16(W) || (ldw * dtype_size(w_dtype)) % 16 != 0)
+        return fail(RB_ERR_ALIGNMENT, "W and its row pitch must be 16-byte aligned");
+    if (!aligned16(planes)) return fail(RB_ERR_ALIGNMENT, "planes must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(h) & 3u) || (reinterpret_cast<uintptr_t>(g) & 3u))
+        return fail(RB_ERR_ALIGNMENT, "h and g must be 4-byte aligned");
+    cudaError_t e = launch_pack_fixed(W, w_dtype == RB_F16, ldw, L.M, L.K, L.n_paths, L.order == RB_SLICED, h, g, planes,
+                                      static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "rb_pack_fixed launch");
+    return RB_OK;
+}
+
+size_t rb_dual_gemv_workspace_bytes(rb_layout L, int32_t T) {
+    if (check_layout(L) != RB_OK || L.group != 0 || T < 1 || T > 64) return 0;
+    return dual_plan(L.M, L.K, L.n_paths, T, true).total;
+}
+
+rb_status rb_dual_gemv(const uint32_t* planes, rb_layout L, const float* h, const float* g, const void* x, int64_t ldx,
+                       int32_t T, void* y, rb_dtype y_dtype, int64_t ldy, void* workspace, size_t ws_bytes,
+                       void* stream) {
+    g_last_error.clear();
+    rb_status st = check_layout(L);
+    if (st != RB_OK) return st;
+    if (!planes || !h || !x || !y) return fail(RB_ERR_INVALID_ARG, "null planes, h, x or y");
+    if (L.group != 0) return fail(RB_ERR_UNSUPPORTED, "given scales are per row (h) and per column (g): group must be 0");
+    if ((st = check_gemv_common(h, RB_F32, y_dtype, T)) != RB_OK) return st;
+    if ((reinterpret_cast<uintptr_t>(g) & 3u)) return fail(RB_ERR_ALIGNMENT, "g must be 4-byte aligned");
+    if (ldx < L.K || ldy < L.M) return fail(RB_ERR_INVALID_ARG, "ldx < K or ldy < M");
+    if (!aligned16(planes) || !aligned16(x) || (ldx * 2) % 16 != 0)
+        return fail(RB_ERR_ALIGNMENT, "planes, x and the row pitch of x must be 16-byte aligned");
+    if (reinterpret_cast<uintptr_t>(y) & (dtype_size(y_dtype) - 1)) return fail(RB_ERR_ALIGNMENT, "y misaligned");
+    const DualPlan d = dual_plan(L.M, L.K, L.n_paths, T, true);
+    if (!workspace || ws_bytes < d.total || !aligned16(workspace))
+        return fail(RB_ERR_WORKSPACE, "workspace needs %zu bytes (16-byte aligned), got %zu", d.total, ws_bytes);
+    cudaError_t e = launch_dual_gemv(planes, L.order == RB_SLICED, L.M, L.K, L.n_paths, h, g, x, ldx, T, y,
+                                     y_dtype == RB_F16, ldy, workspace, d, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "rb_dual_gemv launch");
+    return RB_OK;
+}
+
 size_t rb_gemm_workspace_bytes(rb_layout L, int32_t T) {
     if (check_layout(L) != RB_OK || T < 1) return 0;
     if (T > GEMM_DEC_MAX_T) return GEMM_HEADER_BYTES;

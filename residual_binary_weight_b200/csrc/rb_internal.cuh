@@ -102,6 +102,22 @@ cudaError_t launch_gemm_prefill(const uint32_t* planes, const void* alpha, bool 
                                 int n_paths, int group, bool sliced, const void* X, int64_t ldx, int T, void* Y,
                                 bool y_f16, int64_t ldy, uint32_t* err, cudaStream_t s);
 
+// ------------------------------------------------------- dual-scale block
+cudaError_t launch_pack_fixed(const void* W, bool w_f16, int64_t ldw, int64_t M, int64_t K, int N, bool sliced,
+                              const float* h, const float* g, uint32_t* planes, cudaStream_t s);
+
+// Workspace of the dual-scale matvec: the grouped matvec's own workspace
+// (header with the error word first), N single-path descriptors, the scaled
+// activations x_k and the fp32 per-path outputs.
+struct DualPlan {
+    GvPlan gv;
+    size_t gv_bytes, desc_bytes, xk_bytes, yk_bytes, total;
+};
+DualPlan dual_plan(int64_t M, int64_t K, int N, int T, bool scaled_x);
+cudaError_t launch_dual_gemv(const uint32_t* planes, bool sliced, int64_t M, int64_t K, int N, const float* h,
+                             const float* g, const void* x, int64_t ldx, int T, void* y, bool y_f16, int64_t ldy,
+                             void* workspace, const DualPlan& d, cudaStream_t s);
+
 int device_sm_count();
 
 // Device address of the static scratch array of rb_gemv_noalloc on the

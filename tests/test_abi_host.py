@@ -219,3 +219,32 @@ def test_gemm_workspace_sizes():
     assert lib.rb_gemm_workspace_bytes(L, 2048) == 256
     assert lib.rb_gemm_workspace_bytes(L, 0) == 0
     assert lib.rb_gemm_workspace_bytes(Layout(28672, 8000, 2, 0, 1, 0), 16) == 0
+
+
+def test_dual_block_rejects_bad_arguments_before_launch():
+    lib = _lib.load()
+    p = ctypes.c_void_p
+    L = Layout(64, 256, 2, 0, 0, 0)
+    assert _status(lib.rb_pack_fixed(p(FAKE), 0, 256, Layout(64, 256, 2, 128, 0, 0), p(FAKE), None, p(FAKE),
+                                     None)) == "RB_ERR_UNSUPPORTED"
+    assert _status(lib.rb_pack_fixed(p(FAKE), 0, 256, L, None, None, p(FAKE), None)) == "RB_ERR_INVALID_ARG"
+    assert _status(lib.rb_pack_fixed(p(FAKE), 0, 256, L, p(FAKE + 2), None, p(FAKE), None)) == "RB_ERR_ALIGNMENT"
+    assert _status(lib.rb_pack_fixed(p(FAKE), 0, 256, L, p(FAKE), p(FAKE + 1), p(FAKE), None)) == "RB_ERR_ALIGNMENT"
+    need = lib.rb_dual_gemv_workspace_bytes(L, 4)
+    assert need > 256
+    assert lib.rb_dual_gemv_workspace_bytes(Layout(64, 256, 2, 128, 0, 0), 4) == 0
+    ok = [p(FAKE), L, p(FAKE), p(FAKE), p(FAKE), 256, 4, p(FAKE), 1, 64, p(FAKE), need, None]
+    names = ["planes", "L", "h", "g", "x", "ldx", "T", "y", "ydt", "ldy", "ws", "wsb", "s"]
+
+    def call(**kw):
+        args = list(ok)
+        for k, v in kw.items():
+            args[names.index(k)] = v
+        return _status(lib.rb_dual_gemv(*args))
+
+    assert call(L=Layout(64, 256, 2, 128, 0, 0)) == "RB_ERR_UNSUPPORTED"
+    assert call(T=65) == "RB_ERR_UNSUPPORTED"
+    assert call(h=None) == "RB_ERR_INVALID_ARG"
+    assert call(g=p(FAKE + 2)) == "RB_ERR_ALIGNMENT"
+    assert call(x=p(FAKE + 2)) == "RB_ERR_ALIGNMENT"
+    assert call(wsb=need - 1) == "RB_ERR_WORKSPACE"
