@@ -160,6 +160,29 @@ def dual_matvec(planes: np.ndarray, h: np.ndarray, xk: np.ndarray):
     return y, den
 
 
+def reconstruct_f16(planes: np.ndarray, alpha: np.ndarray) -> np.ndarray:
+    """W^ = sum_k alpha_k (.) B_k (RaBiT 4.1), summed exactly in fp64 and
+    rounded once to the nearest fp16: the operand of the reconstruct-once
+    contraction. planes uint32 [N, M, K/32]; alpha [N, M, K/G]. Returns
+    float16 [M, K]."""
+    planes = np.ascontiguousarray(planes, dtype="<u4")
+    N, M, W32 = planes.shape
+    K = W32 * 32
+    G = K // alpha.shape[2]
+    bits = np.unpackbits(planes.view(np.uint8), axis=-1, bitorder="little").reshape(N, M, K)
+    signs = np.where(bits == 1, 1.0, -1.0)
+    What = (np.repeat(np.asarray(alpha, dtype=np.float64), G, axis=2) * signs).sum(0)
+    return What.astype(np.float16)
+
+
+def dense_matvec(W: np.ndarray, x: np.ndarray):
+    """y = x W^T in fp64 (BLAS) for a dense weight, with the tolerance scale
+    D = |x| |W|^T. W [M, K]; x [T, K]. Returns (y [T, M], D [T, M])."""
+    W = np.asarray(W, dtype=np.float64)
+    x = np.atleast_2d(np.asarray(x, dtype=np.float64))
+    return x @ W.T, np.abs(x) @ np.abs(W).T
+
+
 def alpha_to_f16(alpha: np.ndarray) -> np.ndarray:
     """Round fp64 scales to the nearest fp16 (ties to even): the stored fp16 copy."""
     return np.asarray(alpha, dtype=np.float64).astype(np.float16)

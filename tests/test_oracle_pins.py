@@ -536,3 +536,41 @@ def test_dual_matvec_against_blas_and_single_scale_matvec():
         ye, _ = oracle.dual_matvec(planes, h, oracle.dual_inputs(g, e, N))
         col = sum(h[k] * S[k][:, j] * float(np.float16(g[k, j])) for k in range(N))
         assert np.allclose(ye[0], col, rtol=0, atol=1e-14)
+
+
+# ------------------------------------------------------------ reconstruct-once
+def test_reconstruct_hand_values_and_single_rounding():
+    """Two paths, scales (0.75, 0.25): the four weight values are +-1.0 and
+    +-0.5 by sign pattern. And the sum is rounded once from its exact value:
+    1 + 2^-11 + 2^-30 rounds up to 1 + 2^-10 (0x3C01); rounding through fp32
+    first would land on the tie 1 + 2^-11 and give 0x3C00."""
+    w = np.array([[1.0, 1.0, -1.0, -1.0] * 8])
+    w2 = np.array([[1.0, -1.0, 1.0, -1.0] * 8])
+    p1, _, _ = oracle.pack(w, 1, 0)
+    p2, _, _ = oracle.pack(w2, 1, 0)
+    planes = np.concatenate([p1, p2])
+    alpha = np.array([[[0.75]], [[0.25]]])
+    Wr = oracle.reconstruct_f16(planes, alpha)
+    assert Wr.dtype == np.float16
+    assert Wr[0, :4].tolist() == [1.0, 0.5, -0.5, -1.0]
+    alpha = np.array([[[1 + 2.0 ** -11]], [[2.0 ** -30]]])
+    ones = np.full((1, 1, 1), 0xFFFFFFFF, dtype=np.uint32)
+    Wr = oracle.reconstruct_f16(np.concatenate([ones, ones]), alpha)
+    assert Wr.view(np.uint16)[0, 0] == 0x3C01
+
+
+def test_reconstruct_matches_the_paths_and_dense_matvec_is_blas():
+    """Before rounding, W^ x equals sum_k alpha_k (B_k x) (the pinned matvec);
+    after rounding each weight moves by at most half an fp16 ulp."""
+    rng = np.random.default_rng(51)
+    W = rng.standard_normal((16, 384)) * 0.02
+    for group in (0, 128):
+        planes, alpha, _ = oracle.pack(W, 2, group)
+        Wr = oracle.reconstruct_f16(planes, alpha).astype(np.float64)
+        exact = (np.repeat(alpha, 384 // alpha.shape[2], axis=2) * _signs(planes)).sum(0)
+        assert np.all(np.abs(Wr - exact) <= np.abs(exact) * 2.0 ** -11 + 2.0 ** -25)
+        x = rng.standard_normal((3, 384))
+        y, den = oracle.dense_matvec(exact, x)
+        y2, den2 = oracle.matvec(planes, alpha, x)
+        assert np.allclose(y, y2, rtol=0, atol=1e-12 * den2.max())
+        assert np.all(den <= den2 * (1 + 1e-12))
