@@ -257,11 +257,18 @@ def time_gemm(torch, rb, synth, device, peak_tf):
         tf = flops / us / 1e6
         Yd = torch.empty((2048, sp.M), dtype=torch.float16, device=device)
         cu, _, _ = time_calls_us(torch, lambda i: torch.matmul(X, Wd.t(), out=Yd), calls=10, replays=10)
+        rec = time_calls_us(torch, lambda i: rb.gemm(planes, alpha, X, Y=Y, workspace=ws, reconstruct=True), calls=10,
+                            replays=10)
+        rb.gemm(planes, alpha, X, Y=Y, workspace=ws, check_device=True, reconstruct=True)
+        rec_tf = 2.0 * 2048 * sp.M * sp.K / rec[0] / 1e6
         out[name] = dict(_stats(us, p10, p90), shape=[sp.M, sp.K], T=2048, **{
             "TFLOP/s": round(tf, 1), "frac_of_bf16_peak": round(tf / peak_tf, 3) if peak_tf else None,
             "cublas_fp16_dense_us": round(cu, 1),
             "cublas_fp16_dense_TFLOP/s": round(2.0 * 2048 * sp.M * sp.K / cu / 1e6, 1),
-            "flops_counted": "2 * paths * T * M * K (one +-1 contraction per path)"})
+            "flops_counted": "2 * paths * T * M * K (one +-1 contraction per path)",
+            "reconstruct_once": dict(_stats(*rec), **{
+                "TFLOP/s": round(rec_tf, 1), "frac_of_bf16_peak": round(rec_tf / peak_tf, 3) if peak_tf else None,
+                "flops_counted": "2 * T * M * K (one contraction with the fp16 operand sum_k alpha_k B_k)"})})
         del planes, alpha, Wd, X, Y, Yd
     return out
 

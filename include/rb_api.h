@@ -218,6 +218,24 @@ RB_API rb_status rb_gemm(const uint32_t* planes, const void* alpha, rb_dtype alp
                          const void* X, int64_t ldx, int32_t T, void* Y, rb_dtype y_dtype, int64_t ldy,
                          void* workspace, size_t ws_bytes, void* stream);
 
+/*
+ * rb_gemm_reconstruct -- Y_t = W^ X_t with the reconstructed weight
+ * W^[i][j] = RN_fp16(alpha_0[i] B_0[i][j] + alpha_1[i] B_1[i][j]) (RaBiT
+ * section 4.1, W ~= sum_k alpha_k (.) B_k): the two paths are folded into one
+ * fp16 operand per weight (rounded once from the exact sum of the two scales)
+ * and contracted in one tcgen05 MMA chain, half the tensor work of rb_gemm.
+ * Each weight differs from sum_k alpha_k B_k by at most 2^-11 of its
+ * magnitude, so the result is within 2^-11 sum_j |W^_ij x_j| (plus the
+ * output rounding) of rb_gemm's. For prefill-sized blocks (any T >= 1).
+ *
+ * Arguments as rb_gemm; L: two paths, one scale per row (RB_ERR_UNSUPPORTED
+ * otherwise). workspace: at least 256 bytes (the header with the error word,
+ * read by rb_gemm_check).
+ */
+RB_API rb_status rb_gemm_reconstruct(const uint32_t* planes, const void* alpha, rb_dtype alpha_dtype, rb_layout L,
+                                     const void* X, int64_t ldx, int32_t T, void* Y, rb_dtype y_dtype, int64_t ldy,
+                                     void* workspace, size_t ws_bytes, void* stream);
+
 /* Workspace bytes rb_gemm needs for layout L and T tokens on the current
  * device (0 for an invalid layout or T < 1). */
 RB_API size_t rb_gemm_workspace_bytes(rb_layout L, int32_t T);

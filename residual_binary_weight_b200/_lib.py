@@ -24,7 +24,7 @@ EXPORTED = ("rb_planes_words", "rb_scales_count", "rb_status_string", "rb_last_e
             "rb_pack", "rb_gemv", "rb_gemv_workspace_bytes", "rb_gemv_grouped",
             "rb_gemv_grouped_workspace_bytes", "rb_gemv_check", "rb_gemv_noalloc",
             "rb_gemm", "rb_gemm_workspace_bytes", "rb_gemm_check",
-            "rb_pack_fixed", "rb_dual_gemv", "rb_dual_gemv_workspace_bytes")
+            "rb_pack_fixed", "rb_dual_gemv", "rb_dual_gemv_workspace_bytes", "rb_gemm_reconstruct")
 
 
 class RbError(RuntimeError):
@@ -84,6 +84,8 @@ def load() -> ctypes.CDLL:
         lib.rb_gemv_noalloc.restype = st
         lib.rb_gemm.argtypes = [vp, vp, st, Layout, vp, i64, i32, vp, st, i64, vp, sz, vp]
         lib.rb_gemm.restype = st
+        lib.rb_gemm_reconstruct.argtypes = [vp, vp, st, Layout, vp, i64, i32, vp, st, i64, vp, sz, vp]
+        lib.rb_gemm_reconstruct.restype = st
         lib.rb_gemm_workspace_bytes.argtypes = [Layout, i32]
         lib.rb_gemm_workspace_bytes.restype = sz
         lib.rb_gemm_check.argtypes = [vp, vp]

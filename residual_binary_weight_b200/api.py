@@ -219,11 +219,15 @@ def gemm_workspace_bytes(M: int, K: int, n_paths: int, group: int, T: int) -> in
 
 def gemm(planes: torch.Tensor, alpha: torch.Tensor, X: torch.Tensor, group: int = 0,
          Y: Optional[torch.Tensor] = None, y_dtype: torch.dtype = torch.float16,
-         workspace: Optional[torch.Tensor] = None, check_device: bool = False) -> torch.Tensor:
+         workspace: Optional[torch.Tensor] = None, check_device: bool = False,
+         reconstruct: bool = False) -> torch.Tensor:
     """Y[t] = sum_k alpha_k (.) (B_k X[t]) on the tcgen05 tensor cores (any T).
 
-    With check_device=True the call waits for the stream and raises if a
-    kernel recorded a failure in its workspace (rb_gemm_check).
+    reconstruct=True (two paths, per-row scales): one fp16 operand
+    RN(alpha_0 B_0 + alpha_1 B_1) per weight and one MMA chain
+    (rb_gemm_reconstruct). With check_device=True the call waits for the
+    stream and raises if a kernel recorded a failure in its workspace
+    (rb_gemm_check).
     """
     lib = _lib.load()
     X = _x2d(X)
@@ -234,13 +238,14 @@ def gemm(planes: torch.Tensor, alpha: torch.Tensor, X: torch.Tensor, group: int 
     if Y is None:
         Y = torch.empty((T, M), dtype=y_dtype, device=dev)
     L = layout(M, K, N, group, order)
-    need = lib.rb_gemm_workspace_bytes(L, T)
+    need = 256 if reconstruct else lib.rb_gemm_workspace_bytes(L, T)
     if workspace is None or workspace.numel() * workspace.element_size() < need:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    fn = lib.rb_gemm_reconstruct if reconstruct else lib.rb_gemm
     with torch.cuda.device(dev):
-        check(lib.rb_gemm(_p(planes), _p(alpha), _DT[alpha.dtype], L, _p(X), X.stride(0), T,
-                          _p(Y), _DT[Y.dtype], Y.stride(0), _p(workspace),
-                          workspace.numel() * workspace.element_size(), _stream(dev)))
+        check(fn(_p(planes), _p(alpha), _DT[alpha.dtype], L, _p(X), X.stride(0), T,
+                 _p(Y), _DT[Y.dtype], Y.stride(0), _p(workspace),
+                 workspace.numel() * workspace.element_size(), _stream(dev)))
         if check_device:
             check(lib.rb_gemm_check(_p(workspace), _stream(dev)))
     return Y

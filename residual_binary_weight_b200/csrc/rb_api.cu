@@ -355,9 +355,39 @@ rb_status rb_gemm(const uint32_t* planes, const void* alpha, rb_dtype alpha_dtyp
     else
         e = launch_gemm_prefill(planes, alpha, alpha_dtype == RB_F16, L.M, L.K, L.n_paths, L.group,
                                 L.order == RB_SLICED, X, ldx, T, Y, y_dtype == RB_F16, ldy,
-                                static_cast<uint32_t*>(workspace) + 1, s);
+                                static_cast<uint32_t*>(workspace) + 1, false, s);
     if (e == cudaErrorNotSupported) return fail(RB_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
     if (e != cudaSuccess) return cuda_fail(e, "rb_gemm launch");
+    return RB_OK;
+}
+
+rb_status rb_gemm_reconstruct(const uint32_t* planes, const void* alpha, rb_dtype alpha_dtype, rb_layout L,
+                              const void* X, int64_t ldx, int32_t T, void* Y, rb_dtype y_dtype, int64_t ldy,
+                              void* workspace, size_t ws_bytes, void* stream) {
+    g_last_error.clear();
+    rb_status st = check_layout(L);
+    if (st != RB_OK) return st;
+    if (!planes || !alpha || !X || !Y) return fail(RB_ERR_INVALID_ARG, "null planes, alpha, X or Y");
+    if (!valid_dtype(alpha_dtype) || !valid_dtype(y_dtype)) return fail(RB_ERR_INVALID_ARG, "bad dtype");
+    if (L.n_paths != 2 || L.group != 0)
+        return fail(RB_ERR_UNSUPPORTED, "rb_gemm_reconstruct takes two paths with one scale per row");
+    if (T < 1 || T > (1 << 22)) return fail(RB_ERR_UNSUPPORTED, "T=%d outside 1..2^22", T);
+    if (ldx < L.K || ldy < L.M) return fail(RB_ERR_INVALID_ARG, "ldx < K or ldy < M");
+    if (!aligned16(planes) || !aligned16(X) || (ldx * 2) % 16 != 0)
+        return fail(RB_ERR_ALIGNMENT, "planes, X and the row pitch of X must be 16-byte aligned");
+    if (reinterpret_cast<uintptr_t>(alpha) & (dtype_size(alpha_dtype) - 1))
+        return fail(RB_ERR_ALIGNMENT, "alpha misaligned for its dtype");
+    if (reinterpret_cast<uintptr_t>(Y) & (dtype_size(y_dtype) - 1)) return fail(RB_ERR_ALIGNMENT, "Y misaligned");
+    if (!workspace || ws_bytes < GEMM_HEADER_BYTES || !aligned16(workspace))
+        return fail(RB_ERR_WORKSPACE, "workspace needs %zu bytes (16-byte aligned), got %zu",
+                    (size_t)GEMM_HEADER_BYTES, ws_bytes);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(workspace, 0, GEMM_HEADER_BYTES, s);
+    if (e != cudaSuccess) return cuda_fail(e, "rb_gemm_reconstruct workspace clear");
+    e = launch_gemm_prefill(planes, alpha, alpha_dtype == RB_F16, L.M, L.K, 2, 0, L.order == RB_SLICED, X, ldx, T, Y,
+                            y_dtype == RB_F16, ldy, static_cast<uint32_t*>(workspace) + 1, true, s);
+    if (e == cudaErrorNotSupported) return fail(RB_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+    if (e != cudaSuccess) return cuda_fail(e, "rb_gemm_reconstruct launch");
     return RB_OK;
 }
 

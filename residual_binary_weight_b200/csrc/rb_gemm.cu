@@ -70,6 +70,32 @@ __device__ __forceinline__ void expand_word(uint32_t w, uint32_t val2, uint32_t 
     }
 }
 
+// Reconstruct-once expansion of one 32-column word pair (paths 0 and 1) into
+// 16 half2 of W^ = alpha_0 B_0 + alpha_1 B_1: the magnitude is p2 (both
+// signs equal) or q2 (signs differ), chosen by a full-width mask of
+// ~(w0 ^ w1); the sign is that of path 0 (q may itself be negative, and the
+// sign flip of an fp16 is exact). Half2 i holds columns 2i, 2i+1.
+__device__ __forceinline__ void expand_word_rec(uint32_t w0, uint32_t w1, uint32_t p2, uint32_t q2,
+                                                uint32_t (&h)[16]) {
+    const uint32_t e = ~(w0 ^ w1);
+    uint32_t s0[8], se[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        s0[k] = w0 << (7 - k);
+        se[k] = e << (7 - k);
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const int m = i & 3, b = i >> 2;
+        const uint32_t lo = 8u | b, hi = 8u | (4u + b);
+        // bytes 0-1 <- sign of byte b of se[2m] (column 2i), bytes 2-3 <- sign of byte b of se[2m+1]
+        const uint32_t mask = prmt(se[2 * m], se[2 * m + 1], lo | (lo << 4) | (hi << 8) | (hi << 12));
+        const uint32_t mag = (mask & p2) | (~mask & q2);
+        const uint32_t sgn = prmt(s0[2 * m], s0[2 * m + 1], (lo << 4) | (hi << 12));
+        h[i] = mag ^ (~sgn & 0x80008000u);
+    }
+}
+
 struct GemmArgs {
     uint32_t* err;          // device error word of the call (workspace header word 1)
     const uint32_t* planes;
@@ -87,16 +113,19 @@ struct GemmArgs {
 // ATM: the expanded A operand goes to tensor memory (tcgen05.st) instead of
 // shared memory, so shared memory only carries the X tiles; used for token
 // tiles of at most 128, where the accumulators leave room for A stages.
-template <int NP, int BN, int STAGES, bool G128, bool ATM>
+// REC: reconstruct-once -- one fp16 operand W^ = sum_k alpha_k B_k per
+// weight (two paths, per-row scales), one accumulator, one MMA chain.
+template <int NP, int BN, int STAGES, bool G128, bool ATM, bool REC = false>
 struct GemmCfg {
-    static constexpr int NACC = G128 ? 1 : NP;                         // accumulators
+    static constexpr int NA = REC ? 1 : NP;                            // operand tiles per stage
+    static constexpr int NACC = (G128 || REC) ? 1 : NP;                // accumulators
     // tensor-memory columns between accumulators: BN rounded up to a power of two
     static constexpr int ACC_STRIDE = BN <= 16 ? 16 : BN <= 32 ? 32 : BN <= 64 ? 64 : BN <= 128 ? 128 : 256;
     static constexpr uint32_t B_TILE_BYTES = BN * BK * 2;
-    static constexpr uint32_t STAGE_BYTES = (ATM ? 0 : NP * A_TILE_BYTES) + B_TILE_BYTES;
+    static constexpr uint32_t STAGE_BYTES = (ATM ? 0 : NA * A_TILE_BYTES) + B_TILE_BYTES;
     static constexpr int ACC_COLS = NACC * ACC_STRIDE;
     static constexpr int A_BASE = ACC_COLS;               // first tensor-memory column of the A stages
-    static constexpr int A_STAGE_COLS = NP * BK / 2;      // fp16 pairs of all paths of one stage
+    static constexpr int A_STAGE_COLS = NA * BK / 2;      // fp16 pairs of all operand tiles of one stage
     static constexpr uint32_t TMEM_COLS = ATM ? 512 : (ACC_COLS <= 32) ? 32 : (ACC_COLS <= 64) ? 64 :
                                           (ACC_COLS <= 128) ? 128 : (ACC_COLS <= 256) ? 256 : 512;
     // with A in tensor memory the shared memory is small; ask for enough that
@@ -107,12 +136,14 @@ struct GemmCfg {
     static_assert(ACC_COLS <= 512, "accumulators exceed tensor memory");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M = 128");
     static_assert(B_TILE_BYTES % 1024 == 0, "B tile must keep the 1024-byte swizzle alignment");
+    static_assert(!REC || (NP == 2 && !G128), "reconstruct-once: two paths, per-row scales");
 };
 
-template <int NP, int BN, int STAGES, bool G128, bool ATM>
+template <int NP, int BN, int STAGES, bool G128, bool ATM, bool REC>
 __global__ void __launch_bounds__(THREADS, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, GemmArgs a) {
-    using C = GemmCfg<NP, BN, STAGES, G128, ATM>;
+    using C = GemmCfg<NP, BN, STAGES, G128, ATM, REC>;
+    constexpr int NA = C::NA;
     extern __shared__ __align__(1024) unsigned char dsm[];
     // 1024-byte aligned tile area (the 128-byte swizzle repeats every 1024 B)
     const uint32_t raw = smem_addr(dsm);
@@ -128,9 +159,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, GemmArgs a) {
     const uint32_t abort_slot = tmem_slot + 4u;
     volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(dsm + (abort_slot - raw));
     auto a_tile = [&](int s, int p) { return tiles + s * C::STAGE_BYTES + p * A_TILE_BYTES; };
-    auto b_tile = [&](int s) { return tiles + s * C::STAGE_BYTES + (ATM ? 0u : NP * A_TILE_BYTES); };
-    // tensor-memory column of stage s, path p of the A operand (ATM)
-    auto a_col = [&](int s, int p) { return static_cast<uint32_t>(C::A_BASE + (s * NP + p) * (BK / 2)); };
+    auto b_tile = [&](int s) { return tiles + s * C::STAGE_BYTES + (ATM ? 0u : NA * A_TILE_BYTES); };
+    // tensor-memory column of stage s, operand tile p of the A operand (ATM)
+    auto a_col = [&](int s, int p) { return static_cast<uint32_t>(C::A_BASE + (s * NA + p) * (BK / 2)); };
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int row_tile = blockIdx.x, tok_tile = blockIdx.y;
@@ -174,37 +205,35 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, GemmArgs a) {
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
-        if (elect_lane0()) {
-            constexpr uint32_t idesc = instr_desc(BN);
-            bool ok = true;
-            for (int kb = 0; kb < nk && ok; ++kb) {
-                const int s = kb % STAGES;
-                const uint32_t ph = static_cast<uint32_t>(kb / STAGES) & 1u;
-                if (!mbar_wait(full_x(s), ph, abort_flag, err, 2u) || !mbar_wait(full_a(s), ph, abort_flag, err, 2u)) {
-                    ok = false;
-                    break;
-                }
-                fence_after();
-#pragma unroll
-                for (int p = 0; p < NP; ++p) {
-                    const uint32_t d = tmem_base + static_cast<uint32_t>(G128 ? 0 : p * C::ACC_STRIDE);
-#pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk) {
-                        const uint64_t bd = smem_desc(b_tile(s) + 32u * kk);
-                        const uint32_t acc = (kb > 0 || kk > 0 || (G128 && p > 0)) ? 1u : 0u;
-                        if (ATM) {
-                            umma_f16_ta(d, tmem_base + a_col(s, p) + 8u * kk, bd, idesc, acc);
-                        } else {
-                            const uint64_t ad = smem_desc(a_tile(s, p) + 32u * kk);
-                            umma_f16(d, ad, bd, idesc, acc);
-                        }
-                    }
-                }
-                umma_commit(empty_bar(s));      // stage s is free once these MMAs completed
+        // the whole warp runs the loop (warp-uniform operands); one elected
+        // lane issues each MMA
+        constexpr uint32_t idesc = instr_desc(BN);
+        bool ok = true;
+        for (int kb = 0; kb < nk && ok; ++kb) {
+            const int s = kb % STAGES;
+            const uint32_t ph = static_cast<uint32_t>(kb / STAGES) & 1u;
+            if (!__all_sync(FULL_MASK, mbar_wait(full_x(s), ph, abort_flag, err, 2u) &&
+                                           mbar_wait(full_a(s), ph, abort_flag, err, 2u))) {
+                ok = false;
+                break;
             }
-            umma_commit(acc_bar);               // accumulators complete (also after an abort:
-                                                // the teardown waits on it before freeing TMEM)
+            fence_after();
+            const uint64_t bd0 = smem_desc(b_tile(s));
+#pragma unroll
+            for (int p = 0; p < NA; ++p) {
+                const uint32_t d = tmem_base + static_cast<uint32_t>((G128 || REC) ? 0 : p * C::ACC_STRIDE);
+#pragma unroll
+                for (int kk = 0; kk < BK / 16; ++kk) {
+                    // +32 bytes along K inside the swizzled tile: +2 in the address field
+                    const uint32_t acc = (kb > 0 || kk > 0 || (G128 && p > 0)) ? 1u : 0u;
+                    if (ATM) umma_f16_ta_elect(d, tmem_base + a_col(s, p) + 8u * kk, bd0 + 2u * kk, idesc, acc);
+                    else umma_f16_elect(d, smem_desc(a_tile(s, p)) + 2u * kk, bd0 + 2u * kk, idesc, acc);
+                }
+            }
+            umma_commit_elect(empty_bar(s));      // stage s is free once these MMAs completed
         }
+        umma_commit_elect(acc_bar);               // accumulators complete (also after an abort:
+                                                  // the teardown waits on it before freeing TMEM)
     } else if (warp >= EXP_WARP0) {
         // ------------------------------------------------- expansion, then epilogue
         const int r = (warp - EXP_WARP0) * 32 + lane;            // row within the tile
@@ -234,6 +263,17 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, GemmArgs a) {
         // into a register ring, so a stage never waits for global memory even
         // when the tensor-core work per stage is short (few tokens).
         constexpr int PD = 16 / NP;
+        // reconstruct-once: this row's two weight magnitudes, each the fp16
+        // rounding of the exact sum or difference of its fp32 scales
+        uint2 pq2 = make_uint2(0u, 0u);
+        if (REC) {
+            const double a0 = a.alpha_f16 ? __half2float(static_cast<const __half*>(a.alpha)[crow])
+                                          : static_cast<const float*>(a.alpha)[crow];
+            const double a1 = a.alpha_f16 ? __half2float(static_cast<const __half*>(a.alpha)[M + crow])
+                                          : static_cast<const float*>(a.alpha)[M + crow];
+            const uint32_t p = __half_as_ushort(__double2half(a0 + a1)), q = __half_as_ushort(__double2half(a0 - a1));
+            pq2 = make_uint2(p | (p << 16), q | (q << 16));
+        }
         uint2 ring[PD][NP];
         uint32_t aring[PD][NP];
 #pragma unroll
@@ -272,12 +312,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, GemmArgs a) {
                         go = false;
                     } else {
 #pragma unroll
-                        for (int p = 0; p < NP; ++p) {
+                        for (int p = 0; p < NA; ++p) {
                             const uint32_t base = a_tile(s, p) + row_off;
 #pragma unroll
                             for (int half = 0; half < 2; ++half) {
                                 uint32_t h[16];
-                                expand_word(half ? cur[p].y : cur[p].x, v2[p], h);
+                                if (REC) expand_word_rec(half ? cur[0].y : cur[0].x, half ? cur[1].y : cur[1].x, pq2.x,
+                                                         pq2.y, h);
+                                else expand_word(half ? cur[p].y : cur[p].x, v2[p], h);
                                 if (ATM) {
                                     // row r is tensor-memory lane r; column j holds K-columns 2j, 2j+1
                                     tmem_store16(tmem_base + lane_addr_q + a_col(s, p) + 16u * half, h);
@@ -310,7 +352,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, GemmArgs a) {
             float al[C::NACC];
 #pragma unroll
             for (int p = 0; p < C::NACC; ++p) {
-                if (G128) al[p] = 1.0f;
+                if (G128 || REC) al[p] = 1.0f;
                 else al[p] = a.alpha_f16 ? __half2float(static_cast<const __half*>(a.alpha)[p * M + crow])
                                          : static_cast<const float*>(a.alpha)[p * M + crow];
             }
@@ -344,13 +386,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, GemmArgs a) {
         }
     }
 
-    __syncwarp();            // lanes 1..31 of warps 0 and 1 wait for their lane 0
+    __syncwarp();            // lanes 1..31 of warp 0 wait for their lane 0
     fence_before();
     __syncthreads();
     if (warp == 1) {
         // after an abort, the MMAs already issued finish before their tensor
-        // memory is released (the MMA thread committed them to acc_bar)
-        if (elect_lane0() && *abort_flag) mbar_drain(acc_bar, 0u);
+        // memory is released (the MMA warp committed them to acc_bar)
+        if (*abort_flag) mbar_drain(acc_bar, 0u);
         __syncwarp();
         fence_after();
         tmem_dealloc(tmem_base, C::TMEM_COLS);
@@ -358,13 +400,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, GemmArgs a) {
 }
 
 // ---------------------------------------------------------------- host side
-template <int NP, int BN, int STAGES, bool G128, bool ATM = false>
+template <int NP, int BN, int STAGES, bool G128, bool ATM, bool REC>
 cudaError_t launch_cfg(const GemmArgs& a, const void* X, int64_t ldx, cudaStream_t s) {
-    using C = GemmCfg<NP, BN, STAGES, G128, ATM>;
+    using C = GemmCfg<NP, BN, STAGES, G128, ATM, REC>;
     CUtensorMap map;
     cudaError_t me = make_x_map(&map, X, a.K, a.T, ldx, BN);
     if (me != cudaSuccess) return me;
-    auto kern = gemm_tc_kernel<NP, BN, STAGES, G128, ATM>;
+    auto kern = gemm_tc_kernel<NP, BN, STAGES, G128, ATM, REC>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     dim3 grid(static_cast<unsigned>((a.M + BM - 1) / BM), static_cast<unsigned>((a.T + BN - 1) / BN));
@@ -374,44 +416,48 @@ cudaError_t launch_cfg(const GemmArgs& a, const void* X, int64_t ldx, cudaStream
 
 }  // namespace
 
-// stages that fit in shared memory for a configuration (at most 8)
-constexpr int stages_for(int np, int bn) {
-    return ((210 * 1024) / static_cast<int>(np * A_TILE_BYTES + bn * BK * 2)) < 8
-               ? ((210 * 1024) / static_cast<int>(np * A_TILE_BYTES + bn * BK * 2))
+// stages that fit in shared memory for a configuration (at most 8); na
+// operand tiles per stage
+constexpr int stages_for(int na, int bn) {
+    return ((210 * 1024) / static_cast<int>(na * A_TILE_BYTES + bn * BK * 2)) < 8
+               ? ((210 * 1024) / static_cast<int>(na * A_TILE_BYTES + bn * BK * 2))
                : 8;
 }
 
-// stages of the A operand that fit in tensor memory beside the accumulators
-// of a token tile (0: fewer than two, use shared memory for A)
-constexpr int atm_stages(int np, int bn, bool g128) {
-    const int nacc = g128 ? 1 : np;
+// stages of the A operand (na tiles) that fit in tensor memory beside nacc
+// accumulators of a token tile (0: fewer than two, use shared memory for A)
+constexpr int atm_stages(int na, int nacc, int bn) {
     const int stride = bn <= 16 ? 16 : bn <= 32 ? 32 : bn <= 64 ? 64 : bn <= 128 ? 128 : 256;
-    const int st = (512 - nacc * stride) / (np * BK / 2);
+    const int st = (512 - nacc * stride) / (na * BK / 2);
     return st >= 2 ? (st < 8 ? st : 8) : 0;
 }
 
-// token tiles up to 128: A in tensor memory when it fits
-template <int NP, int BN, bool G128>
-cudaError_t launch_narrow(const GemmArgs& a, const void* X, int64_t ldx, cudaStream_t s) {
-    constexpr int SA = atm_stages(NP, BN, G128);
-    if constexpr (SA >= 2) return launch_cfg<NP, BN, SA, G128, true>(a, X, ldx, s);
-    else return launch_cfg<NP, BN, stages_for(NP, BN), G128>(a, X, ldx, s);
+// A in tensor memory when it fits (always for token tiles up to 128; for
+// wider tiles with a single accumulator), else in shared memory
+template <int NP, int BN, bool G128, bool REC>
+cudaError_t launch_tile(const GemmArgs& a, const void* X, int64_t ldx, cudaStream_t s) {
+    constexpr int NA = REC ? 1 : NP, NACC = (G128 || REC) ? 1 : NP;
+    // with A in tensor memory a stage is only the X tile: also bounded by shared memory
+    constexpr int SX = (210 * 1024) / (BN * BK * 2);
+    constexpr int SA = atm_stages(NA, NACC, BN) < SX ? atm_stages(NA, NACC, BN) : SX;
+    if constexpr (SA >= 2 && (BN <= 128 || REC)) return launch_cfg<NP, BN, SA, G128, true, REC>(a, X, ldx, s);
+    else return launch_cfg<NP, BN, stages_for(NA, BN), G128, false, REC>(a, X, ldx, s);
 }
 
-template <int NP, bool G128>
+template <int NP, bool G128, bool REC = false>
 cudaError_t launch_np(const GemmArgs& a, const void* X, int64_t ldx, cudaStream_t s) {
     // token tile: the narrowest of 16..256 that covers T (MMA N), so small
-    // batches do not pay for unused columns; NP accumulators must fit in
+    // batches do not pay for unused columns; the accumulators must fit in
     // 512 tensor-memory columns
-    constexpr int BN_MAX = G128 ? 256 : (NP <= 2 ? 256 : 128);
+    constexpr int BN_MAX = (G128 || REC) ? 256 : (NP <= 2 ? 256 : 128);
     const int T = a.T;
-    if (T <= 16) return launch_narrow<NP, 16, G128>(a, X, ldx, s);
-    if (T <= 32) return launch_narrow<NP, 32, G128>(a, X, ldx, s);
-    if (T <= 64) return launch_narrow<NP, 64, G128>(a, X, ldx, s);
+    if (T <= 16) return launch_tile<NP, 16, G128, REC>(a, X, ldx, s);
+    if (T <= 32) return launch_tile<NP, 32, G128, REC>(a, X, ldx, s);
+    if (T <= 64) return launch_tile<NP, 64, G128, REC>(a, X, ldx, s);
     if constexpr (BN_MAX == 128) {
-        return launch_narrow<NP, 128, G128>(a, X, ldx, s);
+        return launch_tile<NP, 128, G128, REC>(a, X, ldx, s);
     } else {
-    if (T <= 128) return launch_narrow<NP, 128, G128>(a, X, ldx, s);
+    if (T <= 128) return launch_tile<NP, 128, G128, REC>(a, X, ldx, s);
     // Wide token tiles: 240 instead of 256 when the last wave of 256-wide
     // tiles would leave most SMs idle and 240 needs no extra wave: e.g. 112
     // row tiles x 2048 tokens are 896 tiles of 256 (6 full waves on 148 SMs
@@ -422,16 +468,19 @@ cudaError_t launch_np(const GemmArgs& a, const void* X, int64_t ldx, cudaStream_
     const int64_t tiles256 = rows * ((T + 255) / 256), tiles240 = rows * ((T + 239) / 240);
     const int64_t waves256 = (tiles256 + sms - 1) / sms, waves240 = (tiles240 + sms - 1) / sms;
     const int64_t last256 = tiles256 - (waves256 - 1) * sms;
-    if (waves240 <= waves256 && 2 * last256 < sms)
-        return launch_cfg<NP, 240, stages_for(NP, 240), G128>(a, X, ldx, s);
-    return launch_cfg<NP, BN_MAX, stages_for(NP, BN_MAX), G128>(a, X, ldx, s);
+    if (waves240 <= waves256 && 2 * last256 < sms) return launch_tile<NP, 240, G128, REC>(a, X, ldx, s);
+    return launch_tile<NP, BN_MAX, G128, REC>(a, X, ldx, s);
     }
 }
 
 cudaError_t launch_gemm_prefill(const uint32_t* planes, const void* alpha, bool alpha_f16, int64_t M, int64_t K,
                                 int n_paths, int group, bool sliced, const void* X, int64_t ldx, int T, void* Y,
-                                bool y_f16, int64_t ldy, uint32_t* err, cudaStream_t s) {
+                                bool y_f16, int64_t ldy, uint32_t* err, bool reconstruct, cudaStream_t s) {
     GemmArgs a{err, planes, alpha, Y, M, K, ldy, T, n_paths, group == 128, sliced, alpha_f16, y_f16};
+    if (reconstruct) {
+        if (n_paths != 2 || group != 0) return cudaErrorInvalidValue;
+        return launch_np<2, false, true>(a, X, ldx, s);
+    }
     if (group == 0) {
         switch (n_paths) {
             case 1: return launch_np<1, false>(a, X, ldx, s);

@@ -100,7 +100,7 @@ cudaError_t launch_gemm_dec(const uint32_t* planes, const void* alpha, bool alph
                             bool y_f16, int64_t ldy, void* workspace, const GemmDecPlan& plan, cudaStream_t s);
 cudaError_t launch_gemm_prefill(const uint32_t* planes, const void* alpha, bool alpha_f16, int64_t M, int64_t K,
                                 int n_paths, int group, bool sliced, const void* X, int64_t ldx, int T, void* Y,
-                                bool y_f16, int64_t ldy, uint32_t* err, cudaStream_t s);
+                                bool y_f16, int64_t ldy, uint32_t* err, bool reconstruct, cudaStream_t s);
 
 // ------------------------------------------------------- dual-scale block
 cudaError_t launch_pack_fixed(const void* W, bool w_f16, int64_t ldw, int64_t M, int64_t K, int N, bool sliced,

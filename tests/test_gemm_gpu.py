@@ -165,3 +165,90 @@ def test_llama3_full_size_sampled(matrix, T):
     got = Y[:, idx].float().cpu().numpy()
     nbad, worst = oracle.compare_outputs(got, y_ref, den)
     assert nbad == 0, worst
+
+
+# --------------------------------------------------------------- reconstruct-once
+def _run_rec(W, X, alpha_f16, order="rows", y_dtype=torch.float16, ldx_pad=0, ldy_pad=0):
+    """Kernel parity of rb_gemm_reconstruct: the oracle reconstructs
+    RN_fp16(sum_k alpha_k B_k) from its own planes and stored scales and
+    multiplies in fp64 (BLAS); |dY| <= 1e-3 * |X| |W^|^T. Also returns the
+    error against the unrounded layer relative to its own tolerance scale."""
+    ref_p, ref_a, _ = oracle.pack(W, 2, 0)
+    stored = oracle.alpha_to_f16(ref_a) if alpha_f16 else ref_a.astype(np.float32)
+    Wr = oracle.reconstruct_f16(ref_p, stored.astype(np.float64))
+    y_ref, den = oracle.dense_matvec(Wr, X.astype(np.float64))
+    y_exact, den_exact = oracle.matvec(ref_p, stored.astype(np.float64), X.astype(np.float64))
+    T, K = X.shape
+    M = W.shape[0]
+    xt = torch.zeros((T, K + ldx_pad), dtype=torch.float16)
+    xt[:, :K] = torch.from_numpy(X)
+    Xd = xt.cuda()[:, :K]
+    Yd = torch.full((T, M + ldy_pad), float("nan"), dtype=y_dtype, device="cuda")
+    rb.gemm(to_dev_planes(ref_p, order=order), torch.from_numpy(stored).cuda(), Xd, Y=Yd[:, :M], check_device=True,
+            reconstruct=True)
+    Yh = Yd.float().cpu().numpy()
+    if ldy_pad:
+        assert np.all(np.isnan(Yh[:, M:])), "wrote past the row"
+    nbad, worst = oracle.compare_outputs(Yh[:, :M], y_ref, den)
+    _, worst_exact = oracle.compare_outputs(Yh[:, :M], y_exact, den_exact)
+    return nbad, worst, worst_exact
+
+
+@pytest.mark.parametrize("T", [1, 16, 100, 130, 241, 300])
+@pytest.mark.parametrize("alpha_f16,order", [(False, "rows"), (True, "sliced")])
+def test_reconstruct_matches_oracle(T, alpha_f16, order):
+    rng = np.random.default_rng(T + 3)
+    W = (rng.standard_normal((260, 1024)) * 0.02).astype(np.float16)
+    X = rng.standard_normal((T, 1024)).astype(np.float16)
+    nbad, worst, worst_exact = _run_rec(W, X, alpha_f16, order)
+    assert nbad == 0, worst
+    # against the unrounded layer: within the fp16 rounding of the weights and output
+    assert worst_exact < 2.0 ** -10, worst_exact
+
+
+def test_reconstruct_pitches_and_fp32_output():
+    rng = np.random.default_rng(8)
+    W = (rng.standard_normal((333, 640)) * 0.02).astype(np.float32)
+    X = rng.standard_normal((257, 640)).astype(np.float16)
+    nbad, worst, _ = _run_rec(W, X, False, "sliced", torch.float32, ldx_pad=8, ldy_pad=3)
+    assert nbad == 0, worst
+
+
+def test_reconstruct_refuses_other_layouts():
+    rng = np.random.default_rng(9)
+    W = (rng.standard_normal((128, 256)) * 0.02).astype(np.float16)
+    X = torch.from_numpy(rng.standard_normal((130, 256)).astype(np.float16)).cuda()
+    for n_paths, group in ((3, 0), (2, 128)):
+        p, a, _ = oracle.pack(W, n_paths, group)
+        with pytest.raises(rb.RbError, match="RB_ERR_UNSUPPORTED"):
+            rb.gemm(to_dev_planes(p), torch.from_numpy(oracle.alpha_to_f16(a)).cuda(), X, group=group,
+                    reconstruct=True)
+
+
+@pytest.mark.parametrize("matrix", ["up", "down"])
+def test_reconstruct_prefill_full_size_sampled(matrix):
+    """The 2048-token prefill block through a full 14336-wide projection with
+    the reconstructed operand: 64 sampled rows get the oracle's planes and
+    scales, and their outputs for 48 sampled tokens are checked against the
+    oracle's reconstruction."""
+    wl = synth.WORKLOADS["prefill"]
+    spec = {m.name: m for m in wl.matrices}[matrix]
+    W = synth.device_weight(wl, 0, matrix, "cuda")
+    planes, alpha, _ = rb.pack(W, 2, 0, order="sliced")
+    rng = np.random.default_rng(19)
+    rows = np.sort(rng.choice(spec.M, 64, replace=False))
+    idx = torch.from_numpy(rows).cuda()
+    Wr = W.index_select(0, idx).cpu().numpy()
+    del W
+    ref_p, ref_a, _ = oracle.pack(Wr, 2, 0)
+    planes[:, :, idx] = to_dev_planes(ref_p, order="sliced")
+    a32 = ref_a.astype(np.float32)
+    alpha[:, idx] = torch.from_numpy(a32).cuda()
+    X = synth.device_activations(wl, 0, matrix, 2048, "cuda")
+    Y = rb.gemm(planes, alpha, X, check_device=True, reconstruct=True)
+    toks = np.sort(rng.choice(2048, 48, replace=False))
+    Xs = X[torch.from_numpy(toks).cuda()].cpu().numpy().astype(np.float64)
+    y_ref, den = oracle.dense_matvec(oracle.reconstruct_f16(ref_p, a32.astype(np.float64)), Xs)
+    got = Y[torch.from_numpy(toks).cuda()][:, idx].float().cpu().numpy()
+    nbad, worst = oracle.compare_outputs(got, y_ref, den)
+    assert nbad == 0, worst
