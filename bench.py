@@ -541,6 +541,38 @@ def run_gpu(args):
     print(json.dumps(line), flush=True)
     return 0
 
+def run_case(args):
+    """One kernel on one matrix, called warmup + steps times, then checked
+    through the device error word: the small cases that profiler captures of
+    single launches use (no timing is printed)."""
+    import torch
+    import residual_binary_weight_b200 as rb
+    import synth
+    dev = "cuda"
+    prefill = args.case in ("gemm-prefill", "gemm-reconstruct")
+    wl = synth.WORKLOADS["prefill" if prefill else "llama3_70b_decode"]
+    sp = {m.name: m for m in wl.matrices}["up"]
+    T = 2048 if prefill else args.tokens
+    W = synth.device_weight(wl, 0, sp.name, dev)
+    if args.case == "pack":
+        for _ in range(args.warmup + args.steps):
+            rb.pack(W, 2, 0, order="sliced")
+        torch.cuda.synchronize()
+        print(json.dumps({"case": args.case, "shape": [sp.M, sp.K], "ok": True}))
+        return 0
+    planes, alpha, _ = rb.pack(W, 2, 0, order="sliced")
+    del W
+    X = synth.device_activations(wl, 0, sp.name, T, dev)
+    Y = torch.empty((T, sp.M), dtype=torch.float16, device=dev)
+    ws = torch.empty(max(16, rb.gemm_workspace_bytes(sp.M, sp.K, 2, 0, T)), dtype=torch.uint8, device=dev)
+    rec = args.case == "gemm-reconstruct"
+    for _ in range(args.warmup + args.steps):
+        rb.gemm(planes, alpha, X, Y=Y, workspace=ws, reconstruct=rec)
+    rb.gemm(planes, alpha, X, Y=Y, workspace=ws, reconstruct=rec, check_device=True)
+    torch.cuda.synchronize()
+    print(json.dumps({"case": args.case, "shape": [sp.M, sp.K], "T": T, "ok": True}))
+    return 0
+
 
 def main():
     ap = argparse.ArgumentParser()
@@ -552,7 +584,13 @@ def main():
     ap.add_argument("--layers", type=int, default=32,
                     help="decoder layers in the stack (32 for the benchmark; fewer for profiling captures)")
     ap.add_argument("--no-parts", action="store_true", help="skip the rb_pack / rb_gemm sub-measurements")
+    ap.add_argument("--case", choices=["gemm-decode", "gemm-prefill", "gemm-reconstruct", "pack"],
+                    help="run one kernel on one matrix (70B-shaped up projection for gemm-decode and pack, "
+                         "14336x4096 at T=2048 for the prefill cases) for profiler captures, and exit")
+    ap.add_argument("--tokens", type=int, default=16, help="decode batch T for --case gemm-decode")
     args = ap.parse_args()
+    if args.case:
+        return run_case(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_gpu(args)
