@@ -29,20 +29,24 @@
 // into the workspace, and the last of its CTAs to finish adds the parts in
 // CTA order (deterministic) and stores Y.
 //
-// Roles (14 warps):
+// Roles (16 warps):
 //   warps 0-7   expansion: warp w writes rows 32 (w % 4) .. + 31 (its tensor
 //               memory lane quarter) of every path, for the stages i of the
 //               CTA's range with i % 2 == w / 4;
 //   warps 8-11  epilogue: tcgen05.ld of the accumulators, per-row scales,
 //               store or partial sums;
 //   warp 12     TMA loads of the permuted X tiles;
-//   warp 13     allocates tensor memory and issues the MMAs.
-// Warps 12 and 13 run their loops converged (warp-uniform operands) and
-// issue through one elected lane. mbarriers: full[s] (TMA bytes + the 4
-// warps of the stage's group), empty[s] (MMAs of stage s done),
-// acc_full[b] / acc_empty[b] (accumulator buffer b filled / read). Every
-// wait is bounded; a wait that runs out records a code in the call's error
-// word and the CTA winds down after draining what it issued.
+//   warps 13-14 MMA issue, alternate stages (warp 13 allocates tensor memory);
+//   warp 15     TMA loads of the plane words (per-row scales, >= 4 words per
+//               row and stage) into an 8-stage shared-memory ring, so that
+//               the expansion warps issue no global loads.
+// Warps 12-15 run their loops converged (warp-uniform operands) and issue
+// through one elected lane. mbarriers: full[s] (TMA bytes + the 4 warps of
+// the stage's group), empty[s] (MMAs of stage s done), acc_full[b] /
+// acc_empty[b] (accumulator buffer b filled / read), pfull[k] / pempty[k]
+// (plane ring), baton[u] (issue order between the two MMA warps). Every wait
+// is bounded; a wait that runs out records a code in the call's error word
+// and the CTA winds down after draining what it issued.
 #include "rb_tc.cuh"
 
 #include <cuda_fp8.h>
@@ -54,10 +58,11 @@ namespace {
 
 using namespace tc;
 
-constexpr int THREADS = 448;
+constexpr int THREADS = 512;
 constexpr int EPI_WARP0 = 8;
 constexpr int TMA_WARP = 12;
-constexpr int MMA_WARP = 13;
+constexpr int MMA_WARP = 13;   // and MMA_WARP + 1
+constexpr int PL_WARP = 15;
 
 struct DecArgs {
     uint32_t* err;          // the call's device error word
@@ -97,7 +102,13 @@ struct DecCfg {
     static constexpr int STAGES = STAGES_FIT < 8 ? STAGES_FIT : 8;
     static constexpr uint32_t SUB_BYTES = NMMA * 128;      // one 128-byte-wide box of NMMA rows
     static constexpr uint32_t B_TILE_BYTES = SUB * SUB_BYTES;
-    static constexpr uint32_t SMEM_USED = STAGES * B_TILE_BYTES + 1024 /*align*/ + 512 /*barriers*/;
+    // plane words through TMA into a shared-memory ring (per-row scales, at
+    // least 4 words per row and stage: the TMA x coordinate stays 16-byte aligned)
+    static constexpr bool PTMA = !G128 && WPS >= 4;
+    static constexpr int PS = PTMA ? 8 : 0;                            // plane ring stages
+    static constexpr uint32_t P_PATH_BYTES = BM * WPS * 4;             // [128 rows][WPS words]
+    static constexpr uint32_t P_STAGE_BYTES = NP * P_PATH_BYTES;
+    static constexpr uint32_t SMEM_USED = STAGES * B_TILE_BYTES + PS * P_STAGE_BYTES + 1024 /*align*/ + 512 /*barriers*/;
     // at least 120 KB, so that two CTAs never share an SM's tensor memory
     static constexpr uint32_t SMEM_BYTES = SMEM_USED < 120u * 1024u ? 120u * 1024u : SMEM_USED;
     static_assert(STAGES >= 2, "operand stages do not fit beside the accumulators");
@@ -112,19 +123,23 @@ __device__ __forceinline__ int64_t cta_of(int64_t g, int64_t total, int64_t G) {
 
 template <int NP, int BN, bool G128, bool F8>
 __global__ void __launch_bounds__(THREADS, 1)
-gemm_dec_kernel(const __grid_constant__ CUtensorMap xmap, DecArgs a) {
+gemm_dec_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap pmap, DecArgs a) {
     using C = DecCfg<NP, BN, G128, F8>;
     constexpr int STAGES = C::STAGES, ACC_BUF = C::ACC_BUF, SW = C::SW, WPS = C::WPS;
     extern __shared__ __align__(1024) unsigned char dsm[];
     const uint32_t raw = smem_addr(dsm);
     const uint32_t tiles_s = (raw + 1023u) & ~1023u;
-    const uint32_t bars = tiles_s + STAGES * C::B_TILE_BYTES;
+    const uint32_t planes_s = tiles_s + STAGES * C::B_TILE_BYTES;
+    const uint32_t bars = planes_s + C::PS * C::P_STAGE_BYTES;
     auto full_bar = [&](int s) { return bars + 8u * s; };
     auto empty_bar = [&](int s) { return bars + 8u * (STAGES + s); };
     auto acc_full = [&](int b) { return bars + 8u * (2 * STAGES + b); };
     auto acc_empty = [&](int b) { return bars + 8u * (2 * STAGES + 2 + b); };
     const uint32_t fin_bar = bars + 8u * (2 * STAGES + 4);
-    const uint32_t tmem_slot = fin_bar + 8u;
+    auto baton = [&](int u) { return bars + 8u * (2 * STAGES + 5 + u); };
+    auto pfull = [&](int k) { return bars + 8u * (2 * STAGES + 7 + k); };
+    auto pempty = [&](int k) { return bars + 8u * (2 * STAGES + 7 + C::PS + k); };
+    const uint32_t tmem_slot = bars + 8u * (2 * STAGES + 7 + 2 * C::PS);
     const uint32_t abort_slot = tmem_slot + 4u;
     const uint32_t last_slot = abort_slot + 4u;
     volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(dsm + (abort_slot - raw));
@@ -145,10 +160,15 @@ gemm_dec_kernel(const __grid_constant__ CUtensorMap xmap, DecArgs a) {
             mbar_init(empty_bar(s), 1);
         }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(acc_full(b), 1);
+            mbar_init(acc_full(b), 2);
             mbar_init(acc_empty(b), 4);
+            mbar_init(baton(b), 1);
         }
-        mbar_init(fin_bar, 1);
+        mbar_init(fin_bar, 2);
+        for (int k = 0; k < C::PS; ++k) {
+            mbar_init(pfull(k), 1);
+            mbar_init(pempty(k), 4);   // the four warps of the expansion group that reads it
+        }
         *abort_flag = 0u;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -184,61 +204,125 @@ gemm_dec_kernel(const __grid_constant__ CUtensorMap xmap, DecArgs a) {
         if (*abort_flag)   // loads still in flight land before the CTA exits
             for (int64_t i = issued - 1; i >= 0 && i >= issued - STAGES; --i)
                 mbar_drain(full_bar(static_cast<int>(i % STAGES)), static_cast<uint32_t>(i / STAGES) & 1u);
-    } else if (warp == MMA_WARP) {
+    } else if (warp == PL_WARP) {
+        // ------------------------------------------------------ plane words
+        // One TMA load per path and stage: the WPS words of the stage for the
+        // tile's 128 rows (rows past M read as zero), into ring slot i % PS.
+        if constexpr (C::PTMA) {
+            int64_t issued = 0;
+            int64_t lt = lo / S;
+            int lkb = static_cast<int>(lo - lt * S);
+            for (int64_t i = 0; i < hi - lo; ++i) {
+                const int ps = static_cast<int>(i % C::PS);
+                const uint32_t pph = static_cast<uint32_t>(i / C::PS) & 1u;
+                if (!__all_sync(FULL_MASK, mbar_wait(pempty(ps), pph ^ 1u, abort_flag, err, 1u))) break;
+                if (elect_one()) {
+                    mbar_arrive_expect_tx(pfull(ps), C::P_STAGE_BYTES);
+                    const int w = lkb * WPS;
+                    const int row0 = static_cast<int>(lt * BM);
+#pragma unroll
+                    for (int p = 0; p < NP; ++p)
+                        tma_load_4d(planes_s + ps * C::P_STAGE_BYTES + p * C::P_PATH_BYTES, &pmap,
+                                    a.sliced ? (w & 15) : w, row0, a.sliced ? (w >> 4) : 0, p, pfull(ps));
+                }
+                __syncwarp();
+                issued = i + 1;
+                if (++lkb == S) {
+                    lkb = 0;
+                    ++lt;
+                }
+            }
+            if (*abort_flag)   // loads still in flight land before the CTA exits
+                for (int64_t i = issued - 1; i >= 0 && i >= issued - C::PS; --i)
+                    mbar_drain(pfull(static_cast<int>(i % C::PS)), static_cast<uint32_t>(i / C::PS) & 1u);
+        }
+    } else if (warp == MMA_WARP || warp == MMA_WARP + 1) {
         // ---------------------------------------------------------------- MMA
+        // Two issuers take alternate stages of the range (issuer u the
+        // stages i with i % 2 == u), so that one does its bookkeeping
+        // (barrier waits, commit) while the other's MMAs keep the tensor pipe
+        // busy. Both add into the same accumulators, so the order of issue
+        // is handed over: after issuing stage i the issuer fences
+        // (tcgen05.fence::before_thread_sync) and arrives on its baton
+        // barrier; the issuer of stage i + 1 waits for that arrival and
+        // fences (after_thread_sync) before its first MMA. Each issuer
+        // commits its own MMAs: empty[s] for its stages, and acc_full / the
+        // final barrier (two arrivals each) for every tile.
+        const int u = warp - MMA_WARP;
         constexpr uint32_t idesc = F8 ? instr_desc_f8(C::NMMA) : instr_desc(BN);
         int st = 0;          // stage slot and phase of the next stage
         uint32_t sph = 0;
+        uint32_t bph = 0;    // phase of the other issuer's baton waited for next
+        int64_t i = 0;       // stage ordinal in the CTA's range
         int j = 0;           // segment counter
         bool ok = true;
         for (int64_t t = lo / S; ok && t * S < hi; ++t, ++j) {
             const int64_t k0 = (lo > t * S ? lo - t * S : 0), k1 = (hi < (t + 1) * S ? hi - t * S : S);
             const int b = j % ACC_BUF;
-            if (j >= ACC_BUF && !__all_sync(FULL_MASK, mbar_wait(acc_empty(b), static_cast<uint32_t>(j / ACC_BUF - 1) & 1u,
-                                                                  abort_flag, err, 2u))) {
-                ok = false;
-                break;
-            }
-            fence_after();
             const uint32_t dbase = tmem_base + static_cast<uint32_t>(b * C::NACC * C::ACC_STRIDE);
-            for (int64_t kb = k0; kb < k1; ++kb) {
+            for (int64_t kb = k0; kb < k1; ++kb, ++i) {
                 const int s = st;
                 const uint32_t ph = sph;
                 if (++st == STAGES) {
                     st = 0;
                     sph ^= 1u;
                 }
+                if ((i & 1) != u) continue;
+                // the tile's first stage: its accumulator buffer must have been read out
+                if (kb == k0 && j >= ACC_BUF &&
+                    !__all_sync(FULL_MASK, mbar_wait(acc_empty(b), static_cast<uint32_t>(j / ACC_BUF - 1) & 1u,
+                                                     abort_flag, err, 2u))) {
+                    ok = false;
+                    break;
+                }
                 if (!__all_sync(FULL_MASK, mbar_wait(full_bar(s), ph, abort_flag, err, 2u))) {
                     ok = false;
                     break;
                 }
+                if (i > 0) {
+                    if (!__all_sync(FULL_MASK, mbar_wait(baton(u ^ 1), bph, abort_flag, err, 2u))) {
+                        ok = false;
+                        break;
+                    }
+                    bph ^= 1u;
+                }
                 fence_after();
                 const uint64_t bd0 = smem_desc(b_tile(s));
                 const uint32_t acc0 = kb > k0 ? 1u : 0u;
+                if (elect_one()) {
 #pragma unroll
-                for (int p = 0; p < NP; ++p) {
-                    const uint32_t d = dbase + static_cast<uint32_t>(G128 ? 0 : p * C::ACC_STRIDE);
-                    // one MMA per 32 bytes of K (16 fp16 or 32 fp8 columns):
-                    // box kk / 4, and +32 bytes inside a swizzled box is +2
-                    // in the descriptor's address field
+                    for (int p = 0; p < NP; ++p) {
+                        const uint32_t d = dbase + static_cast<uint32_t>(G128 ? 0 : p * C::ACC_STRIDE);
+                        // one MMA per 32 bytes of K (16 fp16 or 32 fp8 columns):
+                        // box kk / 4, and +32 bytes inside a swizzled box is +2
+                        // in the descriptor's address field
 #pragma unroll
-                    for (int kk = 0; kk < WPS * C::COLS_PER_WORD / 8; ++kk) {
-                        const uint64_t bd = bd0 + ((kk >> 2) * C::SUB_BYTES >> 4) + 2u * (kk & 3);
-                        const uint32_t acc = (kk > 0 || (G128 && p > 0)) ? 1u : acc0;
-                        if (F8) umma_f8_ta_elect(d, tmem_base + a_col(s, p) + 8u * kk, bd, idesc, acc);
-                        else umma_f16_ta_elect(d, tmem_base + a_col(s, p) + 8u * kk, bd, idesc, acc);
+                        for (int kk = 0; kk < WPS * C::COLS_PER_WORD / 8; ++kk) {
+                            const uint64_t bd = bd0 + ((kk >> 2) * C::SUB_BYTES >> 4) + 2u * (kk & 3);
+                            const uint32_t acc = (kk > 0 || (G128 && p > 0)) ? 1u : acc0;
+                            if (F8) umma_f8_ta(d, tmem_base + a_col(s, p) + 8u * kk, bd, idesc, acc);
+                            else umma_f16_ta(d, tmem_base + a_col(s, p) + 8u * kk, bd, idesc, acc);
+                        }
                     }
+                    fence_before();
+                    mbar_arrive(baton(u));
+                    umma_commit(empty_bar(s));
                 }
-                umma_commit_elect(empty_bar(s));
+                __syncwarp();
             }
-            if (ok) umma_commit_elect(acc_full(b));
+            if (ok) {
+                if (elect_one()) umma_commit(acc_full(b));
+                __syncwarp();
+            }
         }
-        umma_commit_elect(fin_bar);   // every MMA issued above has completed once this arrives
+        if (elect_one()) umma_commit(fin_bar);   // every MMA issued above has completed once both arrive
+        __syncwarp();
     } else if (warp < 8) {
         // ---------------------------------------------------------- expansion
         // Thread = one row of the tile (its tensor-memory lane), all paths,
         // the stages i with i % 2 == grp. The plane words of a stage (SW / 32
-        // per path) are loaded PR of the group's stages ahead.
+        // per path) come from the TMA ring in shared memory (PTMA) or are
+        // loaded PR of the group's stages ahead into registers.
         const int q = warp & 3, grp = warp >> 2;
         const int r = 32 * q + lane;
         const uint32_t lane_q = static_cast<uint32_t>(32 * q) << 16;
@@ -253,8 +337,8 @@ gemm_dec_kernel(const __grid_constant__ CUtensorMap xmap, DecArgs a) {
         // (tile, stage-in-tile) of the next stage to load, stepping by 2
         int64_t lt = (lo + grp) / S;
         int lkb = static_cast<int>(lo + grp - lt * S);
-        WV ring[PR][NP][NV];
-        uint32_t nring[PR][NP];
+        WV ring[C::PTMA ? 1 : PR][NP][NV];
+        uint32_t nring[C::PTMA ? 1 : PR][NP];
         auto load_stage = [&](WV (&dst)[NP][NV], uint32_t (&ndst)[NP]) {
             const int64_t row64 = lt * BM + r;
             const uint32_t row = static_cast<uint32_t>(row64 < M ? row64 : M - 1);   // rows past M read a real row
@@ -308,51 +392,84 @@ gemm_dec_kernel(const __grid_constant__ CUtensorMap xmap, DecArgs a) {
                 return j == 0 ? u.x : j == 1 ? u.y : j == 2 ? u.z : u.w;
             }
         };
+        // expand the words of stage slot s into tensor memory and hand the slot to the MMA
+        auto expand_stage = [&](const WV (&cur)[NP][NV], const uint32_t (&ng)[NP], int s) {
 #pragma unroll
-        for (int d = 0; d < PR; ++d)
-            if (grp + 2 * d < n) load_stage(ring[d], nring[d]);
+            for (int p = 0; p < NP; ++p) {
+                if constexpr (F8) {
+#pragma unroll
+                    for (int wi = 0; wi < WPS; wi += 2)
+                        expand_store8(word(cur[p], wi), word(cur[p], wi + 1), a_col(s, p) + 8u * wi);
+                } else {
+#pragma unroll
+                    for (int wi = 0; wi < WPS; ++wi) expand_store(word(cur[p], wi), ng[p], a_col(s, p) + 16u * wi);
+                }
+            }
+            tmem_store_wait();
+            fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(full_bar(s));
+        };
         int s = grp % STAGES;
         uint32_t ph = static_cast<uint32_t>(grp / STAGES) & 1u;
-        bool go = true;
-        for (int64_t i0 = grp; i0 < n && go; i0 += 2 * PR) {
+        if constexpr (C::PTMA) {
+            const unsigned char* prow = dsm + (planes_s - raw) + static_cast<uint32_t>(r) * (WPS * 4);
+            uint32_t ng[NP];
 #pragma unroll
-            for (int d = 0; d < PR; ++d) {
-                const int64_t i = i0 + 2 * d;
-                if (i < n && go) {
-                    WV cur[NP][NV];
-                    uint32_t ng[NP];
+            for (int p = 0; p < NP; ++p) ng[p] = 0xBC00BC00u;   // -1.0 in both halves
+            for (int64_t i = grp; i < n; i += 2) {
+                const int ps = static_cast<int>(i % C::PS);
+                if (!__all_sync(FULL_MASK, mbar_wait(pfull(ps), static_cast<uint32_t>(i / C::PS) & 1u, abort_flag,
+                                                     err, 4u)))
+                    break;
+                WV cur[NP][NV];
 #pragma unroll
-                    for (int p = 0; p < NP; ++p) {
+                for (int p = 0; p < NP; ++p)
 #pragma unroll
-                        for (int v = 0; v < NV; ++v) cur[p][v] = ring[d][p][v];
-                        ng[p] = nring[d][p];
-                    }
-                    if (i + 2 * PR < n) load_stage(ring[d], nring[d]);
-                    // warp-uniform: the tensor-memory stores below are .sync.aligned
-                    if (!__all_sync(FULL_MASK, mbar_wait(empty_bar(s), ph ^ 1u, abort_flag, err, 4u))) {
-                        go = false;
-                    } else {
+                    for (int v = 0; v < NV; ++v)
+                        cur[p][v] = *reinterpret_cast<const WV*>(prow + ps * C::P_STAGE_BYTES + p * C::P_PATH_BYTES +
+                                                                 v * sizeof(WV));
+                __syncwarp();
+                if (lane == 0) mbar_arrive(pempty(ps));   // the words are in registers: the slot may refill
+                // warp-uniform: the tensor-memory stores are .sync.aligned
+                if (!__all_sync(FULL_MASK, mbar_wait(empty_bar(s), ph ^ 1u, abort_flag, err, 4u))) break;
+                expand_stage(cur, ng, s);
+                s += 2;
+                if (s >= STAGES) {
+                    s -= STAGES;
+                    ph ^= 1u;
+                }
+            }
+        } else {
+#pragma unroll
+            for (int d = 0; d < PR; ++d)
+                if (grp + 2 * d < n) load_stage(ring[d], nring[d]);
+            bool go = true;
+            for (int64_t i0 = grp; i0 < n && go; i0 += 2 * PR) {
+#pragma unroll
+                for (int d = 0; d < PR; ++d) {
+                    const int64_t i = i0 + 2 * d;
+                    if (i < n && go) {
+                        WV cur[NP][NV];
+                        uint32_t ng[NP];
 #pragma unroll
                         for (int p = 0; p < NP; ++p) {
-                            if constexpr (F8) {
 #pragma unroll
-                                for (int wi = 0; wi < WPS; wi += 2)
-                                    expand_store8(word(cur[p], wi), word(cur[p], wi + 1), a_col(s, p) + 8u * wi);
-                            } else {
-#pragma unroll
-                                for (int wi = 0; wi < WPS; ++wi)
-                                    expand_store(word(cur[p], wi), ng[p], a_col(s, p) + 16u * wi);
-                            }
+                            for (int v = 0; v < NV; ++v) cur[p][v] = ring[d][p][v];
+                            ng[p] = nring[d][p];
                         }
-                        tmem_store_wait();
-                        fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(full_bar(s));
-                    }
-                    s += 2;
-                    if (s >= STAGES) {
-                        s -= STAGES;
-                        ph ^= 1u;
+                        if (i + 2 * PR < n) load_stage(ring[d], nring[d]);
+                        // warp-uniform: the tensor-memory stores are .sync.aligned
+                        if (!__all_sync(FULL_MASK, mbar_wait(empty_bar(s), ph ^ 1u, abort_flag, err, 4u))) {
+                            go = false;
+                        } else {
+                            expand_stage(cur, ng, s);
+                        }
+                        s += 2;
+                        if (s >= STAGES) {
+                            s -= STAGES;
+                            ph ^= 1u;
+                        }
                     }
                 }
             }
@@ -559,16 +676,45 @@ __global__ void split_x_f8_kernel(const __half* __restrict__ X, int64_t ldx, int
     }
 }
 
+// Plane words as a 4-D uint32 tensor {word, row, slice, path}: in the sliced
+// order 16 words per 512-column slice (rows 64 bytes apart, slices M rows
+// apart); in the row order all K/32 words of a row and one slice. A box is
+// the stage's `words` words of 128 rows of one path.
+cudaError_t make_plane_map(CUtensorMap* map, const uint32_t* planes, int64_t M, int64_t K, int n_paths, bool sliced,
+                           int words) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return cudaErrorNotSupported;
+    const int64_t W32 = K / 32, SL = (K + 511) / 512;
+    const cuuint64_t wpr = static_cast<cuuint64_t>(sliced ? 16 : W32);   // words per row and slice
+    const cuuint64_t dims[4] = {wpr, static_cast<cuuint64_t>(M), static_cast<cuuint64_t>(sliced ? SL : 1),
+                                static_cast<cuuint64_t>(n_paths)};
+    const cuuint64_t row_b = wpr * 4, slice_b = row_b * static_cast<cuuint64_t>(M);
+    const cuuint64_t strides[3] = {row_b, slice_b, slice_b * dims[2]};
+    const cuuint32_t box[4] = {static_cast<cuuint32_t>(words), static_cast<cuuint32_t>(tc::BM), 1u, 1u};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    if (enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, const_cast<uint32_t*>(planes), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    return cudaSuccess;
+}
+
 template <int NP, int BN, bool G128, bool F8>
 cudaError_t launch_dec(const DecArgs& a, const void* Xp, int grid, cudaStream_t s) {
     using C = DecCfg<NP, BN, G128, F8>;
-    CUtensorMap map;
+    CUtensorMap map, pmap;
     cudaError_t e = F8 ? make_x8_map(&map, Xp, a.K, a.T, 4, BN) : make_x_map(&map, Xp, a.K, a.T, a.K, BN);
     if (e != cudaSuccess) return e;
+    if constexpr (C::PTMA) {
+        e = make_plane_map(&pmap, a.planes, a.M, a.K, NP, a.sliced, C::WPS);
+        if (e != cudaSuccess) return e;
+    } else {
+        pmap = map;   // unused
+    }
     auto kern = gemm_dec_kernel<NP, BN, G128, F8>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    kern<<<grid, THREADS, C::SMEM_BYTES, s>>>(map, a);
+    kern<<<grid, THREADS, C::SMEM_BYTES, s>>>(map, pmap, a);
     return cudaGetLastError();
 }
 
