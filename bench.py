@@ -293,7 +293,7 @@ def time_decode_shapes(torch, rb, synth, device, hbm_peak, tf_peak, wl_name, bat
         for T in batches:
             X = synth.device_activations(wl, 0, sp.name, T, device)
             Y = torch.empty((T, sp.M), dtype=torch.float16, device=device)
-            wsv = torch.empty(max(16, rb.gemv_workspace_bytes(sp.M, sp.K, n_paths, group, T)), dtype=torch.uint8,
+            wsv = torch.zeros(max(16, rb.gemv_workspace_bytes(sp.M, sp.K, n_paths, group, T)), dtype=torch.uint8,
                               device=device)
             wsg = torch.empty(max(16, rb.gemm_workspace_bytes(sp.M, sp.K, n_paths, group, T)), dtype=torch.uint8,
                               device=device)

@@ -130,9 +130,13 @@ RB_API rb_status rb_pack(const void* W, rb_dtype w_dtype, int64_t ldw, rb_layout
  * y         device, out, T rows of M values of type y_dtype, pitch ldy >= M.
  * T         tokens, 1..64.
  * workspace device scratch of at least rb_gemv_workspace_bytes(L, T) bytes,
- *           16-byte aligned; its first bytes are cleared by the call (a
- *           memset on `stream`) and it must not be shared by calls that may
- *           overlap on the GPU. May be NULL when that size is 0.
+ *           16-byte aligned, ZEROED ONCE before its first use (cudaMemset);
+ *           every call leaves its arrival counters at zero again, so no
+ *           clearing is needed between calls (the kernel clears the error
+ *           word itself; no memset is enqueued). A workspace zeroed once
+ *           serves any later shape that fits it. It must not be shared by
+ *           calls that may overlap on the GPU. May be NULL when that size is
+ *           0. A counter found non-zero is flagged (rb_gemv_check).
  * Errors: as rb_pack; RB_ERR_WORKSPACE if the workspace is too small. A
  *         kernel-side failure is recorded in the workspace; rb_gemv_check()
  *         reads it back.
@@ -174,7 +178,8 @@ typedef struct {
  * n           1..2047.  n_paths, group, order (an rb_order), alpha_dtype,
  *             y_dtype: shared by all.
  * T           tokens, 1..64.
- * workspace   device scratch of rb_gemv_grouped_workspace_bytes(...) bytes.
+ * workspace   device scratch of rb_gemv_grouped_workspace_bytes(...) bytes,
+ *             zeroed once before its first use, as for rb_gemv.
  */
 RB_API rb_status rb_gemv_grouped(const rb_gemv_desc* descs_host, const rb_gemv_desc* descs_dev,
                           int32_t n, int32_t n_paths, int32_t group, int32_t order,
@@ -207,8 +212,10 @@ RB_API size_t rb_gemv_grouped_workspace_bytes(const rb_gemv_desc* descs_host, in
  *           16-byte aligned, owned by the caller: a 256-byte header (word 1
  *           is the call's device error word) and, for T <= 64, arrival
  *           counters, fp32 partial sums and a column-permuted copy of X.
- *           The call clears what must start at zero (a memset on `stream`);
- *           calls that may overlap on the GPU need separate workspaces.
+ *           Nothing needs to be zero beforehand: for T <= 64 the call's
+ *           operand pre-pass clears the error word and the counters, the
+ *           prefill kernel clears the error word (no memset is enqueued).
+ *           Calls that may overlap on the GPU need separate workspaces.
  * Errors: validation as rb_gemv (RB_ERR_WORKSPACE if the workspace is too
  *         small); RB_ERR_CUDA if the tensor-map encoder or a launch fails. A
  *         kernel whose bounded pipeline waits ran out records a code in the
@@ -303,8 +310,8 @@ RB_API size_t rb_dual_gemv_workspace_bytes(rb_layout L, int32_t T);
  * - The first call on a device looks up the array's device address
  *   (cudaGetSymbolAddress) with that device current; make that first call
  *   before any stream capture.
- * - Every call on a device shares the array, and a call clears the part that
- *   must start at zero (a memset on `stream`). Calls whose work may overlap
+ * - Every call on a device shares the array (zero-initialised storage; each
+ *   call leaves its counters at zero again). Calls whose work may overlap
  *   on the GPU -- on different streams of one device -- race on the array and
  *   must be ordered by the caller.
  * - Nothing here calls cudaMalloc, cudaFree or any allocating routine.

@@ -133,8 +133,11 @@ def gemv(planes: torch.Tensor, alpha: torch.Tensor, x: torch.Tensor, group: int 
          workspace: Optional[torch.Tensor] = None, check_device: bool = False) -> torch.Tensor:
     """y[t] = sum_k alpha_k (.) (B_k x[t]) for T <= 64 tokens (CUDA-core table kernel).
 
-    With check_device=True the call waits for the stream and raises if the
-    kernel recorded a failure in its workspace (rb_gemv_check).
+    A caller-given workspace must have been zeroed once before its first use
+    (torch.zeros); each call leaves it ready for the next. Without one, a
+    zeroed workspace is allocated for the call. With check_device=True the
+    call waits for the stream and raises if the kernel recorded a failure in
+    its workspace (rb_gemv_check).
     """
     lib = _lib.load()
     x = _x2d(x)
@@ -147,7 +150,7 @@ def gemv(planes: torch.Tensor, alpha: torch.Tensor, x: torch.Tensor, group: int 
     L = layout(M, K, N, group, order)
     need = lib.rb_gemv_workspace_bytes(L, T)
     if workspace is None or workspace.numel() * workspace.element_size() < need:
-        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+        workspace = torch.zeros(max(need, 16), dtype=torch.uint8, device=dev)
     with torch.cuda.device(dev):
         check(lib.rb_gemv(_p(planes), _p(alpha), _DT[alpha.dtype], L, _p(x), x.stride(0), T,
                           _p(y), _DT[y.dtype], y.stride(0), _p(workspace),
@@ -199,7 +202,7 @@ class GroupedGemv:
         self.alpha_dtype, self.y_dtype = _DT[adt], _DT[ydt]
         self.order = _ORDERS[order]
         need = lib.rb_gemv_grouped_workspace_bytes(self.host, n, n_paths, T)
-        self.workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+        self.workspace = torch.zeros(max(need, 16), dtype=torch.uint8, device=dev)
         self.n = n
 
     def run(self) -> None:

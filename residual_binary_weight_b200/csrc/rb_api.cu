@@ -70,7 +70,7 @@ static bool valid_dtype(rb_dtype d) { return d == RB_F16 || d == RB_F32; }
 
 static size_t gv_ws_bytes(const GvPlan& pl) {
     if (pl.counters == 0 && pl.partials == 0) return GV_HEADER_BYTES;
-    return GV_HEADER_BYTES + ((pl.counters + 3) & ~size_t(3)) * 4 + pl.partials * 4;
+    return GV_HEADER_BYTES + GV_CTR_ZONE_BYTES + pl.partials * 4;
 }
 
 }  // namespace rb
@@ -160,9 +160,6 @@ rb_status rb_gemv(const uint32_t* planes, const void* alpha, rb_dtype alpha_dtyp
     if (!workspace || ws_bytes < need || !aligned16(workspace))
         return fail(RB_ERR_WORKSPACE, "workspace needs %zu bytes (16-byte aligned), got %zu", need, ws_bytes);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const size_t clear = GV_HEADER_BYTES + ((pl.counters + 3) & ~size_t(3)) * 4;
-    cudaError_t e = cudaMemsetAsync(workspace, 0, clear, s);
-    if (e != cudaSuccess) return cuda_fail(e, "rb_gemv workspace clear");
     GvArgs a{};
     a.one = GvJob{planes, alpha, x, y, L.M, L.K};
     a.jobs = nullptr;
@@ -181,7 +178,7 @@ rb_status rb_gemv(const uint32_t* planes, const void* alpha, rb_dtype alpha_dtyp
     a.expect_units = static_cast<uint32_t>(pl.units);
     a.expect_ctrs = static_cast<uint32_t>(pl.counters);
     a.expect_parts = static_cast<uint32_t>(pl.partials);
-    e = launch_gemv(a, pl, s);
+    const cudaError_t e = launch_gemv(a, pl, s);
     if (e != cudaSuccess) return cuda_fail(e, "rb_gemv launch");
     return RB_OK;
 }
@@ -236,9 +233,6 @@ rb_status rb_gemv_grouped(const rb_gemv_desc* descs_host, const rb_gemv_desc* de
     if (!workspace || ws_bytes < need || !aligned16(workspace))
         return fail(RB_ERR_WORKSPACE, "workspace needs %zu bytes (16-byte aligned), got %zu", need, ws_bytes);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const size_t clear = GV_HEADER_BYTES + ((pl.counters + 3) & ~size_t(3)) * 4;
-    cudaError_t e = cudaMemsetAsync(workspace, 0, clear, s);
-    if (e != cudaSuccess) return cuda_fail(e, "rb_gemv_grouped workspace clear");
     GvArgs a{};
     a.one = GvJob{};
     a.jobs = reinterpret_cast<const GvJob*>(descs_dev);
@@ -257,7 +251,7 @@ rb_status rb_gemv_grouped(const rb_gemv_desc* descs_host, const rb_gemv_desc* de
     a.expect_units = static_cast<uint32_t>(pl.units);
     a.expect_ctrs = static_cast<uint32_t>(pl.counters);
     a.expect_parts = static_cast<uint32_t>(pl.partials);
-    e = launch_gemv(a, pl, s);
+    const cudaError_t e = launch_gemv(a, pl, s);
     if (e != cudaSuccess) return cuda_fail(e, "rb_gemv_grouped launch");
     return RB_OK;
 }
@@ -338,17 +332,17 @@ rb_status rb_gemm(const uint32_t* planes, const void* alpha, rb_dtype alpha_dtyp
     if (reinterpret_cast<uintptr_t>(Y) & (dtype_size(y_dtype) - 1)) return fail(RB_ERR_ALIGNMENT, "Y misaligned");
     const bool dec = T <= GEMM_DEC_MAX_T;
     GemmDecPlan pl{};
-    size_t need = GEMM_HEADER_BYTES, clear = GEMM_HEADER_BYTES;
+    size_t need = GEMM_HEADER_BYTES;
     if (dec) {
         pl = gemm_dec_plan(L.M, L.K, L.n_paths, L.group, T, device_sm_count());
         need += pl.counters_bytes + pl.partials_bytes + pl.xp_bytes;
-        clear += pl.counters_bytes;
     }
     if (!workspace || ws_bytes < need || !aligned16(workspace))
         return fail(RB_ERR_WORKSPACE, "workspace needs %zu bytes (16-byte aligned), got %zu", need, ws_bytes);
+    // no memset: the decode path's operand pre-pass clears the error word
+    // and the arrival counters, the prefill kernel clears the error word
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = cudaMemsetAsync(workspace, 0, clear, s);
-    if (e != cudaSuccess) return cuda_fail(e, "rb_gemm workspace clear");
+    cudaError_t e;
     if (dec)
         e = launch_gemm_dec(planes, alpha, alpha_dtype == RB_F16, L.M, L.K, L.n_paths, L.group, L.order == RB_SLICED,
                             X, ldx, T, Y, y_dtype == RB_F16, ldy, workspace, pl, s);
@@ -382,9 +376,7 @@ rb_status rb_gemm_reconstruct(const uint32_t* planes, const void* alpha, rb_dtyp
         return fail(RB_ERR_WORKSPACE, "workspace needs %zu bytes (16-byte aligned), got %zu",
                     (size_t)GEMM_HEADER_BYTES, ws_bytes);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = cudaMemsetAsync(workspace, 0, GEMM_HEADER_BYTES, s);
-    if (e != cudaSuccess) return cuda_fail(e, "rb_gemm_reconstruct workspace clear");
-    e = launch_gemm_prefill(planes, alpha, alpha_dtype == RB_F16, L.M, L.K, 2, 0, L.order == RB_SLICED, X, ldx, T, Y,
+    const cudaError_t e = launch_gemm_prefill(planes, alpha, alpha_dtype == RB_F16, L.M, L.K, 2, 0, L.order == RB_SLICED, X, ldx, T, Y,
                             y_dtype == RB_F16, ldy, static_cast<uint32_t*>(workspace) + 1, true, s);
     if (e == cudaErrorNotSupported) return fail(RB_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
     if (e != cudaSuccess) return cuda_fail(e, "rb_gemm_reconstruct launch");
@@ -428,11 +420,13 @@ rb_status rb_gemv_check(const void* workspace, void* stream) {
     rb_status st = read_flags(header, stream, "rb_gemv_check", &flag);
     if (st != RB_OK) return st;
     if (flag)
-        return fail(RB_ERR_DEVICE, "matvec kernel flag 0x%x (%s%s%s)", flag,
+        return fail(RB_ERR_DEVICE, "matvec kernel flag 0x%x (%s%s%s%s)", flag,
                     (flag & GV_ERR_SMEM_LAYOUT) ? "shared-memory window not where the tables need it; " : "",
                     (flag & GV_ERR_BAD_JOB) ? "device descriptors differ from the host copy the launch was "
                                               "planned on; " : "",
-                    (flag & GV_ERR_TOO_MANY_JOBS) ? "more descriptors than a launch takes" : "");
+                    (flag & GV_ERR_TOO_MANY_JOBS) ? "more descriptors than a launch takes; " : "",
+                    (flag & GV_ERR_COUNTER) ? "an arrival counter was not zero (workspace not zeroed before its "
+                                              "first use)" : "");
     return RB_OK;
 }
 

@@ -155,7 +155,9 @@ DualPlan dual_plan(int64_t M, int64_t K, int N, int T, bool scaled_x) {
     d.gv = gemv_plan_grouped(jobs, N, 1, 0, T);
     delete[] jobs;
     auto a256 = [](size_t b) { return (b + 255) & ~size_t(255); };
-    const size_t gv_ws = GV_HEADER_BYTES + ((d.gv.counters + 3) & ~size_t(3)) * 4 + d.gv.partials * 4;
+    const size_t gv_ws = (d.gv.counters == 0 && d.gv.partials == 0)
+                             ? GV_HEADER_BYTES
+                             : GV_HEADER_BYTES + GV_CTR_ZONE_BYTES + d.gv.partials * 4;
     d.gv_bytes = a256(gv_ws);
     d.desc_bytes = a256(static_cast<size_t>(N) * sizeof(GvJob));
     d.xk_bytes = scaled_x ? a256(static_cast<size_t>(N) * T * K * 2) : a256(static_cast<size_t>(T) * K * 2);
@@ -171,7 +173,9 @@ cudaError_t launch_dual_gemv(const uint32_t* planes, bool sliced, int64_t M, int
     GvJob* descs = reinterpret_cast<GvJob*>(ws + d.gv_bytes);
     __half* xk = reinterpret_cast<__half*>(ws + d.gv_bytes + d.desc_bytes);
     float* yk = reinterpret_cast<float*>(ws + d.gv_bytes + d.desc_bytes + d.xk_bytes);
-    const size_t clear = GV_HEADER_BYTES + ((d.gv.counters + 3) & ~size_t(3)) * 4;
+    // this workspace carries no zeroed-once contract: clear header and counters
+    const size_t zone = GV_HEADER_BYTES + GV_CTR_ZONE_BYTES;
+    const size_t clear = d.gv_bytes < zone ? d.gv_bytes : zone;
     cudaError_t e = cudaMemsetAsync(workspace, 0, clear, s);
     if (e != cudaSuccess) return e;
     // the grouped descriptors take dense [T][K] activations: per path x_k with

@@ -163,6 +163,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, GemmArgs a) {
     // tensor-memory column of stage s, operand tile p of the A operand (ATM)
     auto a_col = [&](int s, int p) { return static_cast<uint32_t>(C::A_BASE + (s * NA + p) * (BK / 2)); };
 
+    // the call's error word is cleared here rather than by a memset before
+    // the launch: flags are raised only by waits that ran out, seconds after
+    // the first CTA started
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *a.err = 0u;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int row_tile = blockIdx.x, tok_tile = blockIdx.y;
     const int64_t M = a.M, K = a.K;

@@ -602,10 +602,19 @@ gemm_dec_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant_
 // X' = X with the columns of every 32-column block reordered so that
 // position 2k holds column k and position 2k + 1 column k + 16 (the operand
 // order the expansion above produces). One thread per (token, block).
+// The pre-pass also clears the call's error word and the arrival counters
+// of the main kernel (it runs before it on the same stream).
+__device__ __forceinline__ void clear_call_state(uint32_t* err, uint32_t* counters, int64_t n_ctr, int64_t idx) {
+    if (idx == 0) *err = 0u;
+    const int64_t step = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t i = idx; i < n_ctr; i += step) counters[i] = 0u;
+}
+
 __global__ void permute_x_kernel(const __half* __restrict__ X, int64_t ldx, int T, int64_t K,
-                                 __half* __restrict__ Xp) {
+                                 __half* __restrict__ Xp, uint32_t* err, uint32_t* counters, int64_t n_ctr) {
     const int64_t blocks = K >> 5;
     const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    clear_call_state(err, counters, n_ctr, idx);
     if (idx >= blocks * T) return;
     const int64_t t = idx / blocks, bl = idx - t * blocks;
     const uint4* src = reinterpret_cast<const uint4*>(X + t * ldx + 32 * bl);
@@ -637,9 +646,10 @@ __global__ void permute_x_kernel(const __half* __restrict__ X, int64_t ldx, int 
 // inside every 32-column block byte 4r + b holds column 8b + r (the order
 // the fp8 expansion produces). One thread per (token, block).
 __global__ void split_x_f8_kernel(const __half* __restrict__ X, int64_t ldx, int T, int64_t K,
-                                  uint8_t* __restrict__ Xq) {
+                                  uint8_t* __restrict__ Xq, uint32_t* err, uint32_t* counters, int64_t n_ctr) {
     const int64_t blocks = K >> 5;
     const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    clear_call_state(err, counters, n_ctr, idx);
     if (idx >= blocks * T) return;
     const int64_t t = idx / blocks, bl = idx - t * blocks;
     const uint4* src = reinterpret_cast<const uint4*>(X + t * ldx + 32 * bl);
@@ -773,15 +783,16 @@ cudaError_t launch_gemm_dec(const uint32_t* planes, const void* alpha, bool alph
     float* partials = reinterpret_cast<float*>(ws + GEMM_HEADER_BYTES + pl.counters_bytes);
     __half* Xp = reinterpret_cast<__half*>(ws + GEMM_HEADER_BYTES + pl.counters_bytes + pl.partials_bytes);
     const int64_t nthr = (K >> 5) * T;
+    uint32_t* err = reinterpret_cast<uint32_t*>(ws) + 1;
     if (pl.f8)
         split_x_f8_kernel<<<static_cast<unsigned>((nthr + 127) / 128), 128, 0, s>>>(
-            static_cast<const __half*>(X), ldx, T, K, reinterpret_cast<uint8_t*>(Xp));
+            static_cast<const __half*>(X), ldx, T, K, reinterpret_cast<uint8_t*>(Xp), err, counters, pl.tiles);
     else
         permute_x_kernel<<<static_cast<unsigned>((nthr + 255) / 256), 256, 0, s>>>(
-            static_cast<const __half*>(X), ldx, T, K, Xp);
+            static_cast<const __half*>(X), ldx, T, K, Xp, err, counters, pl.tiles);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    DecArgs a{reinterpret_cast<uint32_t*>(ws) + 1, counters, partials, planes, alpha, Y, M, K, ldy, pl.tiles,
+    DecArgs a{err, counters, partials, planes, alpha, Y, M, K, ldy, pl.tiles,
               pl.total, T, sliced, alpha_f16, y_f16};
     const bool g128 = group == 128;
     switch (n_paths) {

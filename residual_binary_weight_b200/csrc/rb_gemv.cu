@@ -337,6 +337,11 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_lut_kernel(GvArgs p, uint32_t
     extern __shared__ __align__(16) unsigned char dsm[];
     LowSmem& lo = *reinterpret_cast<LowSmem*>(dsm);
 
+    // The call's error word is cleared here, not by a memset before the
+    // launch: every condition below is detected by every CTA, CTA 0
+    // included, after this store, so a flag another CTA raised before it is
+    // raised again.
+    if (blockIdx.x == 0 && threadIdx.x == 0) hdr[1] = 0u;
     const uint32_t s0 = smem_addr(dsm);
     if (s0 + sizeof(LowSmem) > TBL0 || s0 + SMEM_BYTES < TBL0 + 2 * 0x10000u) {
         if (threadIdx.x == 0) atomicOr(hdr + 1, GV_ERR_SMEM_LAYOUT);
@@ -658,8 +663,13 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_lut_kernel(GvArgs p, uint32_t
             __threadfence();
             cta_sync();
             if (tid == 0) {
-                const uint32_t prev = atomicAdd(ctrs + lo.ctr_prefix[ue.j] + ue.rb * T + ue.t, 1u);
+                uint32_t* ctr = ctrs + lo.ctr_prefix[ue.j] + ue.rb * T + ue.t;
+                const uint32_t prev = atomicAdd(ctr, 1u);
                 lo.last = (prev == nch - 1) ? 1u : 0u;
+                // the last arrival puts the counter back to zero, so the
+                // workspace needs no clearing between calls
+                if (prev == nch - 1) *ctr = 0u;
+                if (prev >= nch) atomicOr(hdr + 1, GV_ERR_COUNTER);
             }
             cta_sync();
             if (lo.last) {
@@ -687,7 +697,7 @@ cudaError_t launch_one(const GvArgs& a, const GvPlan& plan, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     uint32_t* hdr = static_cast<uint32_t*>(a.workspace);
     uint32_t* ctrs = reinterpret_cast<uint32_t*>(static_cast<char*>(a.workspace) + GV_HEADER_BYTES);
-    float* parts = reinterpret_cast<float*>(ctrs + ((plan.counters + 3) & ~size_t(3)));
+    float* parts = reinterpret_cast<float*>(ctrs + GV_MAX_COUNTERS);
     const int sms = device_sm_count();
     size_t grid = plan.units;
     if (grid > static_cast<size_t>(sms)) grid = sms;
@@ -748,7 +758,9 @@ GvPlan gemv_plan_single(int64_t M, int64_t K, int n_paths, int group, int T, int
     const int64_t sms = num_sms > 0 ? num_sms : 1;
     int64_t best_nch = 1;
     double best = -1.0;
-    for (int64_t nch = 1; nch <= S; ++nch) {
+    // a split needs nrb * T arrival counters, at most GV_MAX_COUNTERS
+    const int64_t max_nch = nrb * T <= static_cast<int64_t>(GV_MAX_COUNTERS) ? S : 1;
+    for (int64_t nch = 1; nch <= max_nch; ++nch) {
         const int64_t units = nrb * nch * T;
         const int64_t per_cta = (units + sms - 1) / sms;
         const int64_t slices = (S + nch - 1) / nch;
@@ -771,9 +783,12 @@ GvPlan gemv_plan_grouped(const GvJob* jobs, int n, int n_paths, int group, int T
     // arrival counter, the last CTA's reduction), which costs more than the
     // load imbalance of longer units (7B stack: 8 -> 408 us, 12 -> 402 us;
     // 4 or 6, which split the 4096-wide matrices too: 519 and 506 us)
-    const int chunk = 12;
-    GvPlan pl{R, chunk, 0, 0, 0};
-    for (int i = 0; i < n; ++i) count_job(jobs[i].M, jobs[i].K, R, chunk, T, pl);
+    GvPlan pl{R, 12, 0, 0, 0};
+    for (int i = 0; i < n; ++i) count_job(jobs[i].M, jobs[i].K, R, pl.chunk_slices, T, pl);
+    if (pl.counters > GV_MAX_COUNTERS) {   // more splits than the counter zone holds: split nothing
+        pl = GvPlan{R, 1 << 20, 0, 0, 0};
+        for (int i = 0; i < n; ++i) count_job(jobs[i].M, jobs[i].K, R, pl.chunk_slices, T, pl);
+    }
     return pl;
 }
 

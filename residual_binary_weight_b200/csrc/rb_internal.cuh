@@ -63,9 +63,18 @@ struct GvArgs {
 // arrival counter per (job, row block, token) of every K-split job, then the
 // fp32 partial sums of the split jobs.
 constexpr size_t GV_HEADER_BYTES = 256;
+// Arrival counters of K-split units live in a zone of fixed size right after
+// the header, the fp32 partial sums after it: a workspace zeroed once keeps
+// zero counters whatever plans later calls use (every call leaves its
+// counters at zero, and no plan writes partial sums into the zone). A plan
+// with more counters than the zone holds does not split K.
+constexpr size_t GV_CTR_ZONE_BYTES = 65536;
+constexpr size_t GV_MAX_COUNTERS = GV_CTR_ZONE_BYTES / 4;
 // GV_ERR_BAD_JOB: the device descriptors do not give the plan the host sized
 // the workspace for (they differ from the host copy)
-enum : uint32_t { GV_ERR_SMEM_LAYOUT = 1u, GV_ERR_BAD_JOB = 2u, GV_ERR_TOO_MANY_JOBS = 4u };
+// GV_ERR_COUNTER: an arrival counter held more than its K chunks (the
+// workspace was not zeroed before its first use).
+enum : uint32_t { GV_ERR_SMEM_LAYOUT = 1u, GV_ERR_BAD_JOB = 2u, GV_ERR_TOO_MANY_JOBS = 4u, GV_ERR_COUNTER = 8u };
 
 struct GvPlan {
     int rows_per_cta;       // R

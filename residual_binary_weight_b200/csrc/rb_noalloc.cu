@@ -69,9 +69,9 @@ extern "C" rb_status rb_gemv_noalloc(const uint32_t* planes, const void* alpha, 
         rb::set_error_message(msg);
         return RB_ERR_CUDA;
     }
-    // rb_gemv validates the arguments, clears the counters in the scratch with
-    // a memset on `stream` and launches; an invalid layout (need == 0) is
-    // reported by it as well
+    // rb_gemv validates the arguments and launches (the static scratch starts
+    // at zero and every call leaves its counters at zero); an invalid layout
+    // (need == 0) is reported by it as well
     return rb_gemv(planes, alpha, alpha_dtype, L, x, ldx, T, y, y_dtype, ldy, scratch, kNoallocScratchBytes,
                    stream);
 }

@@ -318,3 +318,41 @@ def test_qbb_full_size_single_and_grouped(T):
     for (_, _, _, yg), (toks, y_ref, den) in zip(items, refs):
         nbad, worst = oracle.compare_outputs(yg[torch.from_numpy(toks).cuda()].float().cpu().numpy(), y_ref, den)
         assert nbad == 0, (T, worst)
+
+
+def test_workspace_reused_across_shapes_without_clearing():
+    """A workspace zeroed once serves later calls of other shapes: every call
+    that splits K leaves its arrival counters at zero again."""
+    rng = np.random.default_rng(41)
+    ws = torch.zeros(1 << 20, dtype=torch.uint8, device="cuda")
+    R = 512   # rows per CTA for two paths
+    for M, K, T in [(700, 8192, 3), (300, 6656, 1), (1100, 8192, 2), (700, 8192, 3)]:
+        assert rb.gemv_workspace_bytes(M, K, 2, 0, T) > 256, "the case must split K"
+        W = (rng.standard_normal((M, K)) * 0.02).astype(np.float16)
+        x = rng.standard_normal((T, K)).astype(np.float16)
+        ref_p, ref_a, _ = oracle.pack(W, 2, 0)
+        y = rb.gemv(to_dev_planes(ref_p), torch.from_numpy(ref_a.astype(np.float32)).cuda(),
+                    torch.from_numpy(x).cuda(), workspace=ws, check_device=True)
+        y_ref, den = oracle.matvec(ref_p, ref_a.astype(np.float32).astype(np.float64), x.astype(np.float64))
+        nbad, worst = oracle.compare_outputs(y.float().cpu().numpy(), y_ref, den)
+        assert nbad == 0, (M, K, T, worst)
+        n_ctr = -(-M // R) * T
+        assert int(ws[256:256 + 4 * n_ctr].view(torch.int32).abs().sum()) == 0, "counters left non-zero"
+
+
+def test_a_counter_left_non_zero_is_reported():
+    """A workspace that was not zeroed (here: one counter set on the host)
+    is reported by rb_gemv_check instead of passing silently."""
+    rng = np.random.default_rng(42)
+    M, K, T = 700, 8192, 1
+    W = (rng.standard_normal((M, K)) * 0.02).astype(np.float16)
+    ref_p, ref_a, _ = oracle.pack(W, 2, 0)
+    planes, alpha = to_dev_planes(ref_p), torch.from_numpy(ref_a.astype(np.float32)).cuda()
+    x = torch.from_numpy(rng.standard_normal((T, K)).astype(np.float16)).cuda()
+    ws = torch.zeros(rb.gemv_workspace_bytes(M, K, 2, 0, T), dtype=torch.uint8, device="cuda")
+    ws[256:260].view(torch.int32)[0] = 1000
+    rb.gemv(planes, alpha, x, workspace=ws)
+    with pytest.raises(rb.RbError, match="not zero"):
+        rb.gemv(planes, alpha, x, workspace=ws, check_device=True)
+    ws.zero_()
+    rb.gemv(planes, alpha, x, workspace=ws, check_device=True)
