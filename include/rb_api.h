@@ -148,6 +148,35 @@ RB_API rb_status rb_gemv(const uint32_t* planes, const void* alpha, rb_dtype alp
 
 RB_API size_t rb_gemv_workspace_bytes(rb_layout L, int32_t T);
 
+/*
+ * rb_gemv_swiglu -- h_t = silu(G x_t) (.) (U x_t) for the gated MLP block of
+ * the Llama models whose decode speed RaBiT section 5 reports (the pages do
+ * not print the block; silu(z) = z / (1 + e^-z) is that architecture's gate),
+ * with G and U both residual-binary matrices of layout L:
+ *     G x = sum_k alpha^G_k (.) (B^G_k x),   U x = sum_k alpha^U_k (.) (B^U_k x).
+ * One launch of the rb_gemv kernel: each unit evaluates the rows of both
+ * matrices and its epilogue applies the gate, so G x and U x never reach
+ * memory. The down projection that consumes h is a plain rb_gemv.
+ *
+ * planes    device, 2 * rb_planes_words(L) words: G's L.n_paths planes, then
+ *           U's (two rb_pack outputs stored back to back), in L.order.
+ * alpha     device, 2 * rb_scales_count(L) scales of type alpha_dtype: G's,
+ *           then U's.
+ * L         M, K, group, order of both matrices; n_paths = paths of each
+ *           (1..4).
+ * x, T      as rb_gemv.
+ * h         device, out, T rows of M values of type h_dtype, pitch ldh >= M:
+ *           silu(g) * u computed in fp32 from the fp32 sums g, u, then
+ *           rounded to h_dtype.
+ * workspace as rb_gemv, of rb_gemv_swiglu_workspace_bytes(L, T) bytes
+ *           (zeroed once before its first use).
+ * Errors: as rb_gemv; RB_ERR_UNSUPPORTED for more than 4 paths per matrix.
+ */
+RB_API rb_status rb_gemv_swiglu(const uint32_t* planes, const void* alpha, rb_dtype alpha_dtype, rb_layout L,
+                                const void* x, int64_t ldx, int32_t T, void* h, rb_dtype h_dtype, int64_t ldh,
+                                void* workspace, size_t ws_bytes, void* stream);
+RB_API size_t rb_gemv_swiglu_workspace_bytes(rb_layout L, int32_t T);
+
 /* One matrix of a grouped matvec; x is [T][K] and y is [T][M], both dense. */
 typedef struct {
     const uint32_t* planes;  /* device, rb_planes_words words in the call's order */

@@ -183,6 +183,30 @@ def dense_matvec(W: np.ndarray, x: np.ndarray):
     return x @ W.T, np.abs(x) @ np.abs(W).T
 
 
+def silu_gate(g: np.ndarray, u: np.ndarray) -> np.ndarray:
+    """h = silu(g) u = g u / (1 + e^-g) in fp64: the gate of the gated MLP
+    block of the Llama models whose decode RaBiT section 5 times (the pages
+    do not print the block; this is that architecture's SiLU gate)."""
+    g = np.asarray(g, dtype=np.float64)
+    with np.errstate(over="ignore"):
+        return g / (1.0 + np.exp(-g)) * np.asarray(u, dtype=np.float64)
+
+
+def swiglu_matvec(planes: np.ndarray, alpha: np.ndarray, x: np.ndarray):
+    """The gated pair evaluated from its planes: planes [2N, M, K/32] and
+    alpha [2N, M, K/G] hold the gate G's N paths, then the up projection
+    U's. g = G x and u = U x are the pinned matvec of each half; h =
+    silu_gate(g, u). Returns (h, g, u, Dg, Du), fp64 [T, M]; Dg, Du are the
+    matvec tolerance scales of g and u."""
+    n2 = planes.shape[0]
+    if n2 % 2:
+        raise ValueError("expected the gate's and the up projection's paths")
+    n = n2 // 2
+    g, dg = matvec(planes[:n], alpha[:n], x)
+    u, du = matvec(planes[n:], alpha[n:], x)
+    return silu_gate(g, u), g, u, dg, du
+
+
 def alpha_to_f16(alpha: np.ndarray) -> np.ndarray:
     """Round fp64 scales to the nearest fp16 (ties to even): the stored fp16 copy."""
     return np.asarray(alpha, dtype=np.float64).astype(np.float16)

@@ -18,13 +18,17 @@ from .api import (  # noqa: F401
     gemm,
     gemm_workspace_bytes,
     gemv,
+    gemv_swiglu,
+    gemv_swiglu_workspace_bytes,
     gemv_workspace_bytes,
     layout,
+    mlp_gemv,
     pack,
     pack_fixed,
     planes_words,
     scales_count,
 )
 
-__all__ = ["pack", "pack_fixed", "gemv", "dual_gemv", "gemm", "GroupedGemv", "layout", "planes_words", "scales_count",
-           "gemv_workspace_bytes", "gemm_workspace_bytes", "RbError", "load"]
+__all__ = ["pack", "pack_fixed", "gemv", "gemv_swiglu", "mlp_gemv", "dual_gemv", "gemm", "GroupedGemv", "layout",
+           "planes_words", "scales_count", "gemv_workspace_bytes", "gemv_swiglu_workspace_bytes",
+           "gemm_workspace_bytes", "RbError", "load"]

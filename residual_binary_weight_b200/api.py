@@ -160,6 +160,65 @@ def gemv(planes: torch.Tensor, alpha: torch.Tensor, x: torch.Tensor, group: int 
     return y
 
 
+def gemv_swiglu_workspace_bytes(M: int, K: int, n_paths: int, group: int, T: int) -> int:
+    return _lib.load().rb_gemv_swiglu_workspace_bytes(layout(M, K, n_paths, group), T)
+
+
+def gemv_swiglu(planes: torch.Tensor, alpha: torch.Tensor, x: torch.Tensor, group: int = 0,
+                h: Optional[torch.Tensor] = None, h_dtype: torch.dtype = torch.float16,
+                workspace: Optional[torch.Tensor] = None, check_device: bool = False) -> torch.Tensor:
+    """h[t] = silu(G x[t]) * (U x[t]) in one launch (rb_gemv_swiglu).
+
+    planes / alpha hold the gate's N paths followed by the up projection's N
+    paths (e.g. torch.cat of two pack() outputs along dim 0). The workspace
+    contract is gemv()'s (zeroed once before its first use).
+    """
+    lib = _lib.load()
+    x = _x2d(x)
+    dev = _require_cuda(planes, alpha, x, h, workspace)
+    K = x.shape[1]
+    N2, M, order = _planes_geometry(planes, K)
+    if N2 % 2:
+        raise ValueError("planes must hold the gate's and the up projection's paths (an even count)")
+    T = x.shape[0]
+    if h is None:
+        h = torch.empty((T, M), dtype=h_dtype, device=dev)
+    L = layout(M, K, N2 // 2, group, order)
+    need = lib.rb_gemv_swiglu_workspace_bytes(L, T)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.zeros(max(need, 16), dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        check(lib.rb_gemv_swiglu(_p(planes), _p(alpha), _DT[alpha.dtype], L, _p(x), x.stride(0), T,
+                                 _p(h), _DT[h.dtype], h.stride(0), _p(workspace),
+                                 workspace.numel() * workspace.element_size(), _stream(dev)))
+        if check_device:
+            check(lib.rb_gemv_check(_p(workspace), _stream(dev)))
+    return h
+
+
+def mlp_gemv(gu_planes: torch.Tensor, gu_alpha: torch.Tensor, d_planes: torch.Tensor, d_alpha: torch.Tensor,
+             x: torch.Tensor, group: int = 0, y: Optional[torch.Tensor] = None,
+             workspace: Optional[torch.Tensor] = None, check_device: bool = False):
+    """The gated MLP block for decode tokens: y = D (silu(G x) * (U x)).
+
+    Two launches on the current stream: rb_gemv_swiglu (gate and up, gated
+    in the epilogue, h in fp16) and rb_gemv for the down projection D.
+    Returns (y, h). One workspace (zeroed once) serves both launches.
+    """
+    x = _x2d(x)
+    K = x.shape[1]
+    _, M, order = _planes_geometry(gu_planes, K)
+    Nd, Md, _ = _planes_geometry(d_planes, M)
+    T = x.shape[0]
+    need = max(gemv_swiglu_workspace_bytes(M, K, gu_planes.shape[0] // 2, group, T),
+               gemv_workspace_bytes(Md, M, Nd, group, T), 16)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.zeros(need, dtype=torch.uint8, device=x.device)
+    h = gemv_swiglu(gu_planes, gu_alpha, x, group=group, workspace=workspace, check_device=check_device)
+    y = gemv(d_planes, d_alpha, h, group=group, y=y, workspace=workspace, check_device=check_device)
+    return y, h
+
+
 class GroupedGemv:
     """One persistent launch over many (planes, alpha, x, y) matrices.
 

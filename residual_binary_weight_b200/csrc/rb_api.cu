@@ -141,13 +141,15 @@ static rb_status check_gemv_common(const void* alpha, rb_dtype alpha_dtype, rb_d
     return RB_OK;
 }
 
-rb_status rb_gemv(const uint32_t* planes, const void* alpha, rb_dtype alpha_dtype,
-                  rb_layout L, const void* x, int64_t ldx, int32_t T,
-                  void* y, rb_dtype y_dtype, int64_t ldy,
-                  void* workspace, size_t ws_bytes, void* stream) {
+// rb_gemv, and rb_gemv_swiglu with `gated` (the planes and scales then hold
+// 2 L.n_paths paths: the gate's, then the up projection's)
+static rb_status gemv_one(const uint32_t* planes, const void* alpha, rb_dtype alpha_dtype, rb_layout L,
+                          const void* x, int64_t ldx, int32_t T, void* y, rb_dtype y_dtype, int64_t ldy,
+                          void* workspace, size_t ws_bytes, void* stream, bool gated) {
     g_last_error.clear();
     rb_status st = check_layout(L);
     if (st != RB_OK) return st;
+    if (gated && L.n_paths > 4) return fail(RB_ERR_UNSUPPORTED, "rb_gemv_swiglu takes 1..4 paths per matrix");
     if (!planes || !alpha || !x || !y) return fail(RB_ERR_INVALID_ARG, "null planes, alpha, x or y");
     if ((st = check_gemv_common(alpha, alpha_dtype, y_dtype, T)) != RB_OK) return st;
     if (ldx < L.K || ldy < L.M) return fail(RB_ERR_INVALID_ARG, "ldx < K or ldy < M");
@@ -155,7 +157,8 @@ rb_status rb_gemv(const uint32_t* planes, const void* alpha, rb_dtype alpha_dtyp
         return fail(RB_ERR_ALIGNMENT, "planes, x and the row pitch of x must be 16-byte aligned");
     if (reinterpret_cast<uintptr_t>(y) & (dtype_size(y_dtype) - 1)) return fail(RB_ERR_ALIGNMENT, "y misaligned");
     const int sms = device_sm_count();
-    GvPlan pl = gemv_plan_single(L.M, L.K, L.n_paths, L.group, T, sms);
+    const int np = gated ? 2 * L.n_paths : L.n_paths;
+    GvPlan pl = gemv_plan_single(L.M, L.K, np, L.group, T, sms, gated);
     const size_t need = gv_ws_bytes(pl);
     if (!workspace || ws_bytes < need || !aligned16(workspace))
         return fail(RB_ERR_WORKSPACE, "workspace needs %zu bytes (16-byte aligned), got %zu", need, ws_bytes);
@@ -164,7 +167,8 @@ rb_status rb_gemv(const uint32_t* planes, const void* alpha, rb_dtype alpha_dtyp
     a.one = GvJob{planes, alpha, x, y, L.M, L.K};
     a.jobs = nullptr;
     a.n_jobs = 1;
-    a.n_paths = L.n_paths;
+    a.n_paths = np;
+    a.swiglu = gated ? 1 : 0;
     a.group = L.group;
     a.sliced = L.order == RB_SLICED;
     a.alpha_f16 = alpha_dtype == RB_F16;
@@ -179,8 +183,26 @@ rb_status rb_gemv(const uint32_t* planes, const void* alpha, rb_dtype alpha_dtyp
     a.expect_ctrs = static_cast<uint32_t>(pl.counters);
     a.expect_parts = static_cast<uint32_t>(pl.partials);
     const cudaError_t e = launch_gemv(a, pl, s);
-    if (e != cudaSuccess) return cuda_fail(e, "rb_gemv launch");
+    if (e != cudaSuccess) return cuda_fail(e, gated ? "rb_gemv_swiglu launch" : "rb_gemv launch");
     return RB_OK;
+}
+
+rb_status rb_gemv(const uint32_t* planes, const void* alpha, rb_dtype alpha_dtype, rb_layout L, const void* x,
+                  int64_t ldx, int32_t T, void* y, rb_dtype y_dtype, int64_t ldy, void* workspace, size_t ws_bytes,
+                  void* stream) {
+    return gemv_one(planes, alpha, alpha_dtype, L, x, ldx, T, y, y_dtype, ldy, workspace, ws_bytes, stream, false);
+}
+
+rb_status rb_gemv_swiglu(const uint32_t* planes, const void* alpha, rb_dtype alpha_dtype, rb_layout L,
+                         const void* x, int64_t ldx, int32_t T, void* h, rb_dtype h_dtype, int64_t ldh,
+                         void* workspace, size_t ws_bytes, void* stream) {
+    return gemv_one(planes, alpha, alpha_dtype, L, x, ldx, T, h, h_dtype, ldh, workspace, ws_bytes, stream, true);
+}
+
+size_t rb_gemv_swiglu_workspace_bytes(rb_layout L, int32_t T) {
+    if (check_layout(L) != RB_OK || L.n_paths > 4 || T < 1) return 0;
+    GvPlan pl = gemv_plan_single(L.M, L.K, 2 * L.n_paths, L.group, T, device_sm_count(), true);
+    return gv_ws_bytes(pl);
 }
 
 static rb_status check_descs(const rb_gemv_desc* d, int32_t n, int32_t n_paths, int32_t group, int32_t order,

@@ -211,6 +211,10 @@ __device__ __forceinline__ void build_table(const uint4* xs, uint32_t tbl) {
     for (int lo = 0; lo < 16; ++lo) sts(a0 + (lo << 8), q01[lo & 3] + p23[lo >> 2]);
 }
 
+// silu(g) * u = g u / (1 + e^-g) in fp32 (expf; for g -> -inf the quotient
+// tends to -0)
+__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
+
 // Reduce acc[0..J) over the 8 lanes of an item group (lane bits 0-2); J is
 // a power of two <= 8. Afterwards lane t of the group holds the sum of item
 // load j = t >> (3 - log2 J) in acc[0].
@@ -288,7 +292,7 @@ __device__ __forceinline__ void scan_jobs(const GvArgs& p, LowSmem& lo, int n_jo
             cu[e] = static_cast<uint32_t>(nrb * nch * T);
             if (nch > 1) {
                 cc[e] = static_cast<uint32_t>(nrb * T);
-                cq[e] = static_cast<uint32_t>(nch * T) * static_cast<uint32_t>(jM);
+                cq[e] = static_cast<uint32_t>(nch * T * (p.swiglu ? 2 : 1)) * static_cast<uint32_t>(jM);
             }
         }
     }
@@ -634,32 +638,43 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_lut_kernel(GvArgs p, uint32_t
         // whose path-k item is load k * HR + r / 4 of item group r % 4
         const UnitRec& ue = lo.units[k % UCAP];
         const int64_t M = ue.M;
-        float yv = 0.0f;
+        // yv: sum over the paths (with the SiLU gate: over the gate's paths,
+        // yv2 over the up projection's)
+        float yv = 0.0f, yv2 = 0.0f;
+        const bool gated = p.swiglu != 0;
         const int64_t my_row = static_cast<int64_t>(ue.rb) * C::R + warp * C::RW + lane;
         const bool row_ok = lane < C::RW && my_row < M;
         if (row_ok) {
 #pragma unroll
             for (int kk = 0; kk < NP; ++kk) {
                 const float tk = lo.tot[warp][4 * (kk * HR + (lane >> 2)) + (lane & 3)];
+                float& dst = (gated && kk >= NP / 2) ? yv2 : yv;
                 if (G128) {
-                    yv += tk;
+                    dst += tk;
                 } else {
                     const size_t ai = static_cast<size_t>(kk) * M + my_row;
                     const float a = p.alpha_f16 ? __half2float(static_cast<const __half*>(ue.alpha)[ai])
                                                 : static_cast<const float*>(ue.alpha)[ai];
-                    yv = fmaf(a, tk, yv);
+                    dst = fmaf(a, tk, dst);
                 }
             }
         }
+        auto store_y = [&](int64_t row, float v, float v2) {
+            if (gated) v = silu_mul(v, v2);
+            if (p.y_f16) static_cast<__half*>(ue.y)[row] = __float2half_rn(v);
+            else static_cast<float*>(ue.y)[row] = v;
+        };
         const uint32_t nch = ue.nch;
         if (nch == 1) {
-            if (row_ok) {
-                if (p.y_f16) static_cast<__half*>(ue.y)[my_row] = __float2half_rn(yv);
-                else static_cast<float*>(ue.y)[my_row] = yv;
-            }
+            if (row_ok) store_y(my_row, yv, yv2);
         } else {
-            float* part = parts + lo.part_prefix[ue.j] + (static_cast<size_t>(ue.t) * nch) * M;
-            if (row_ok) part[static_cast<size_t>(ue.ch) * M + my_row] = yv;
+            // partial sums [t][chunk][1 or 2][M]
+            const uint32_t W = gated ? 2u : 1u;
+            float* part = parts + lo.part_prefix[ue.j] + (static_cast<size_t>(ue.t) * nch * W) * M;
+            if (row_ok) {
+                part[static_cast<size_t>(ue.ch * W) * M + my_row] = yv;
+                if (gated) part[static_cast<size_t>(ue.ch * W + 1) * M + my_row] = yv2;
+            }
             __threadfence();
             cta_sync();
             if (tid == 0) {
@@ -678,10 +693,12 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_lut_kernel(GvArgs p, uint32_t
                 for (int i = tid; i < C::R; i += THREADS) {
                     const int64_t row = rbase + i;
                     if (row < M) {
-                        float sum = 0.0f;
-                        for (uint32_t c = 0; c < nch; ++c) sum += __ldcg(part + static_cast<size_t>(c) * M + row);
-                        if (p.y_f16) static_cast<__half*>(ue.y)[row] = __float2half_rn(sum);
-                        else static_cast<float*>(ue.y)[row] = sum;
+                        float sum = 0.0f, sum2 = 0.0f;
+                        for (uint32_t c = 0; c < nch; ++c) {
+                            sum += __ldcg(part + static_cast<size_t>(c * W) * M + row);
+                            if (gated) sum2 += __ldcg(part + static_cast<size_t>(c * W + 1) * M + row);
+                        }
+                        store_y(row, sum, sum2);
                     }
                 }
             }
@@ -737,18 +754,18 @@ int gemv_rows_per_cta(int n_paths, int /*group*/) {
     return WARPS * 4 * hr;
 }
 
-static void count_job(int64_t M, int64_t K, int R, int chunk, int T, GvPlan& pl) {
+static void count_job(int64_t M, int64_t K, int R, int chunk, int T, GvPlan& pl, int sums_per_row = 1) {
     const int64_t nrb = (M + R - 1) / R;
     const int64_t S = (K + SLICE_COLS - 1) / SLICE_COLS;
     const int64_t nch = (S + chunk - 1) / chunk;
     pl.units += static_cast<size_t>(nrb * nch * T);
     if (nch > 1) {
         pl.counters += static_cast<size_t>(nrb * T);
-        pl.partials += static_cast<size_t>(nch * T * M);
+        pl.partials += static_cast<size_t>(nch * T * M * sums_per_row);
     }
 }
 
-GvPlan gemv_plan_single(int64_t M, int64_t K, int n_paths, int group, int T, int num_sms) {
+GvPlan gemv_plan_single(int64_t M, int64_t K, int n_paths, int group, int T, int num_sms, bool swiglu) {
     const int R = gemv_rows_per_cta(n_paths, group);
     const int64_t S = (K + SLICE_COLS - 1) / SLICE_COLS;
     const int64_t nrb = (M + R - 1) / R;
@@ -772,7 +789,7 @@ GvPlan gemv_plan_single(int64_t M, int64_t K, int n_paths, int group, int T, int
     }
     const int chunk = static_cast<int>((S + best_nch - 1) / best_nch);
     GvPlan pl{R, chunk, 0, 0, 0};
-    count_job(M, K, R, chunk, T, pl);
+    count_job(M, K, R, chunk, T, pl, swiglu ? 2 : 1);
     return pl;
 }
 

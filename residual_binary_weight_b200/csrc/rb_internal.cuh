@@ -57,6 +57,11 @@ struct GvArgs {
     // the plan the host sized the workspace for; a launch whose device
     // descriptors give another plan flags GV_ERR_BAD_JOB and does nothing
     uint32_t expect_units, expect_ctrs, expect_parts;
+    // SiLU-gated pair: the job's paths are those of two matrices of the same
+    // shape, [0, n_paths/2) the gate G and [n_paths/2, n_paths) the up
+    // projection U, and the output is y = silu(G x) * (U x) (K-split
+    // units keep two partial sums per row)
+    int swiglu;
 };
 
 // Workspace layout: a 256-byte header (word 1: error flags), then one
@@ -84,7 +89,7 @@ struct GvPlan {
     size_t units;
 };
 int gemv_rows_per_cta(int n_paths, int group);
-GvPlan gemv_plan_single(int64_t M, int64_t K, int n_paths, int group, int T, int num_sms);
+GvPlan gemv_plan_single(int64_t M, int64_t K, int n_paths, int group, int T, int num_sms, bool swiglu = false);
 GvPlan gemv_plan_grouped(const GvJob* host_jobs, int n, int n_paths, int group, int T);
 cudaError_t launch_gemv(const GvArgs& a, const GvPlan& plan, cudaStream_t s);
 int gemv_max_jobs();

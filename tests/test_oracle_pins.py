@@ -574,3 +574,32 @@ def test_reconstruct_matches_the_paths_and_dense_matvec_is_blas():
         y2, den2 = oracle.matvec(planes, alpha, x)
         assert np.allclose(y, y2, rtol=0, atol=1e-12 * den2.max())
         assert np.all(den <= den2 * (1 + 1e-12))
+
+
+# ---------------------------------------------------------- SiLU-gated pair
+def test_silu_gate_closed_forms():
+    """silu(0) = 0; silu(ln 3) = (3/4) ln 3 (e^-ln3 = 1/3); the odd part
+    silu(g) - silu(-g) = g; silu(g) -> g as g -> +inf and -> 0 as g -> -inf."""
+    assert oracle.silu_gate(0.0, 5.0) == 0.0
+    assert abs(oracle.silu_gate(np.log(3.0), 1.0) - 0.75 * np.log(3.0)) < 1e-15
+    rng = np.random.default_rng(3)
+    g = rng.standard_normal(1000) * 4
+    u = rng.standard_normal(1000)
+    assert np.allclose(oracle.silu_gate(g, u) - oracle.silu_gate(-g, u), g * u, rtol=0, atol=1e-12)
+    assert abs(oracle.silu_gate(60.0, 2.0) - 120.0) < 1e-20 * 120 + 1e-13
+    assert 0.0 > oracle.silu_gate(-60.0, 1.0) > -60.0 * np.exp(-59.0)
+    assert oracle.silu_gate(-1000.0, 1.0) == 0.0   # e^1000 overflows; the quotient is -0
+
+
+def test_swiglu_matvec_takes_the_gate_from_the_first_half():
+    """Gate planes all +1 (alpha 1), up planes all -1 (alpha 2), x = 1 over
+    K = 64: g = 64, u = -128, h = silu(64) * -128 (the halves swapped would
+    give silu(-128) * 64, about 0)."""
+    K = 64
+    planes = np.zeros((2, 1, K // 32), dtype=np.uint32)
+    planes[0] = 0xFFFFFFFF
+    alpha = np.array([[[1.0]], [[2.0]]])
+    h, g, u, dg, du = oracle.swiglu_matvec(planes, alpha, np.ones((1, K)))
+    assert g[0, 0] == 64.0 and u[0, 0] == -128.0
+    assert abs(h[0, 0] - (-128.0 * 64.0 / (1.0 + np.exp(-64.0)))) < 1e-9
+    assert dg[0, 0] == 64.0 and du[0, 0] == 128.0
