@@ -318,6 +318,64 @@ def time_decode_shapes(torch, rb, synth, device, hbm_peak, tf_peak, wl_name, bat
     return out
 
 
+def time_mlp(torch, rb, synth, device, hbm_peak):
+    """The gated MLP block at decode, T = 1 and 4: rb_gemv_swiglu (gate and up
+    in one launch, silu(g) * u in its epilogue) then rb_gemv of the down
+    projection, against the unfused sequence (three rb_gemv launches and a
+    torch silu * mul between them). Bytes: the planes and scales of the three
+    matrices, x, h written and read, y. Packed copies are rotated so that
+    every call reads its planes from HBM."""
+    out = {}
+    for label, wl_name, gate, up, down in (("llama2_7b", "llama2_7b_decode", (0, "gate"), (0, "up"), (0, "down")),
+                                           ("llama3_70b", "llama3_70b_decode", (1, "up"), (0, "up"), (0, "down"))):
+        wl = synth.WORKLOADS[wl_name]
+        packed, shapes = {}, {}
+        for key, (layer, name) in (("g", gate), ("u", up), ("d", down)):
+            W = synth.device_weight(wl, layer, name, device)
+            shapes[key] = tuple(W.shape)
+            packed[key] = rb.pack(W, 2, 0, order="sliced")[:2]
+            del W
+        gu_p = torch.cat([packed["g"][0], packed["u"][0]])
+        gu_a = torch.cat([packed["g"][1], packed["u"][1]])
+        d_p, d_a = packed["d"]
+        (M, K), Md = shapes["g"], shapes["d"][0]
+        nbytes = (gu_p.numel() + d_p.numel()) * 4 + (gu_a.numel() + d_a.numel()) * 4
+        n = _copies_for(nbytes)
+        cp = [(gu_p, gu_a, d_p, d_a)] + [(gu_p.clone(), gu_a.clone(), d_p.clone(), d_a.clone()) for _ in range(n - 1)]
+        rows = {}
+        for T in (1, 4):
+            x = synth.device_activations(wl, 0, up[1], T, device)
+            h = torch.empty((T, M), dtype=torch.float16, device=device)
+            y = torch.empty((T, Md), dtype=torch.float16, device=device)
+            gg = torch.empty((T, M), dtype=torch.float16, device=device)
+            uu = torch.empty((T, M), dtype=torch.float16, device=device)
+            ws = torch.zeros(max(rb.gemv_swiglu_workspace_bytes(M, K, 2, 0, T),
+                                 rb.gemv_workspace_bytes(Md, M, 2, 0, T), 16),
+                             dtype=torch.uint8, device=device)
+
+            def fused(i):
+                c = cp[i % n]
+                rb.gemv_swiglu(c[0], c[1], x, h=h, workspace=ws)
+                rb.gemv(c[2], c[3], h, y=y, workspace=ws)
+
+            def unfused(i):
+                c = cp[i % n]
+                rb.gemv(c[0][:2], c[1][:2], x, y=gg, workspace=ws)
+                rb.gemv(c[0][2:], c[1][2:], x, y=uu, workspace=ws)
+                torch.mul(torch.nn.functional.silu(gg), uu, out=h)
+                rb.gemv(c[2], c[3], h, y=y, workspace=ws)
+
+            f = time_calls_us(torch, fused)
+            u = time_calls_us(torch, unfused)
+            rb.mlp_gemv(gu_p, gu_a, d_p, d_a, x, workspace=ws, check_device=True)
+            b = nbytes + T * K * 2 + 2 * T * M * 2 + T * Md * 2
+            rows[f"T{T}"] = {"fused": _stats(*f), "unfused": _stats(*u), "bytes": b,
+                             "GB/s": round(b / f[0] / 1e3, 1), "frac_of_hbm": round(b / f[0] / 1e3 / hbm_peak, 3)}
+        out[f"{label} {M}x{K} -> {Md}x{M}"] = rows
+        del cp, packed, gu_p, gu_a, d_p, d_a
+    return out
+
+
 def read_ceiling_gbs(torch, device):
     """Context: a plain streaming read of 4 GiB (torch.sum over fp32 words) --
     the HBM read rate a library reduction reaches on this GPU."""
@@ -510,6 +568,7 @@ def run_gpu(args):
                                                         "llama3_70b_decode", (1, 4, 16, 64), 2, 0)
         parts["qbb_g128_decode"] = time_decode_shapes(torch, rb, synth, device, hbm_peak, bf16_peak,
                                                       "qbb_g128", (1, 16), 4, 128)
+        parts["mlp_decode"] = time_mlp(torch, rb, synth, device, hbm_peak)
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu:
