@@ -261,11 +261,22 @@ def time_gemm(torch, rb, synth, device, peak_tf):
                             replays=10)
         rb.gemm(planes, alpha, X, Y=Y, workspace=ws, check_device=True, reconstruct=True)
         rec_tf = 2.0 * 2048 * sp.M * sp.K / rec[0] / 1e6
+        # the training forward: planes and scales derived from W in the same call
+        W = Wd   # the fp16 weight
+        wsf = torch.empty(rb.gemm_from_weight_workspace_bytes(sp.M, sp.K, 2, 0, 2048), dtype=torch.uint8,
+                          device=device)
+        fw = time_calls_us(torch, lambda i: rb.gemm_from_weight(W, X, Y=Y, workspace=wsf), calls=10, replays=10)
+        rb.gemm_from_weight(W, X, Y=Y, workspace=wsf, check_device=True)
+        del W
         out[name] = dict(_stats(us, p10, p90), shape=[sp.M, sp.K], T=2048, **{
             "TFLOP/s": round(tf, 1), "frac_of_bf16_peak": round(tf / peak_tf, 3) if peak_tf else None,
             "cublas_fp16_dense_us": round(cu, 1),
             "cublas_fp16_dense_TFLOP/s": round(2.0 * 2048 * sp.M * sp.K / cu / 1e6, 1),
             "flops_counted": "2 * paths * T * M * K (one +-1 contraction per path)",
+            "from_weight": dict(_stats(*fw), **{
+                "TFLOP/s": round(flops / fw[0] / 1e6, 1),
+                "frac_of_bf16_peak": round(flops / fw[0] / 1e6 / peak_tf, 3) if peak_tf else None,
+                "what": "rb_pack of the fp16 weight into the workspace, then rb_gemm (training forward)"}),
             "reconstruct_once": dict(_stats(*rec), **{
                 "TFLOP/s": round(rec_tf, 1), "frac_of_bf16_peak": round(rec_tf / peak_tf, 3) if peak_tf else None,
                 "flops_counted": "2 * T * M * K (one contraction with the fp16 operand sum_k alpha_k B_k)"})})

@@ -272,6 +272,30 @@ RB_API rb_status rb_gemm_reconstruct(const uint32_t* planes, const void* alpha, 
                                      const void* X, int64_t ldx, int32_t T, void* Y, rb_dtype y_dtype, int64_t ldy,
                                      void* workspace, size_t ws_bytes, void* stream);
 
+/*
+ * rb_gemm_from_weight -- the training forward of a residual-binary layer:
+ * the planes and scales are derived afresh from the shared full-precision
+ * weight W and contracted with X in one call, as every training step
+ * re-derives every path from W_FP (RaBiT section 4.2 and appendix G):
+ *     rb_pack(W) into the workspace, then rb_gemm(planes, scales, X).
+ * The planes and scales live only in the call's workspace (with one scale
+ * per 128 columns the fp16 copy is contracted, as rb_gemm requires). The
+ * result equals rb_pack followed by rb_gemm bit for bit.
+ *
+ * W, w_dtype, ldw  as rb_pack.   X, ldx, T, Y, y_dtype, ldy  as rb_gemm.
+ * L         1..4 paths.
+ * workspace device scratch of rb_gemm_from_weight_workspace_bytes(L, T)
+ *           bytes, 16-byte aligned: the rb_gemm workspace, then the planes
+ *           and scales, each on a 256-byte boundary. Nothing needs to be
+ *           zero beforehand.
+ * Errors: everything rb_pack or rb_gemm would refuse, before either is
+ *         enqueued; rb_gemm_check(workspace) reads the device error word.
+ */
+RB_API rb_status rb_gemm_from_weight(const void* W, rb_dtype w_dtype, int64_t ldw, rb_layout L, const void* X,
+                                     int64_t ldx, int32_t T, void* Y, rb_dtype y_dtype, int64_t ldy, void* workspace,
+                                     size_t ws_bytes, void* stream);
+RB_API size_t rb_gemm_from_weight_workspace_bytes(rb_layout L, int32_t T);
+
 /* Workspace bytes rb_gemm needs for layout L and T tokens on the current
  * device (0 for an invalid layout or T < 1). */
 RB_API size_t rb_gemm_workspace_bytes(rb_layout L, int32_t T);

@@ -16,6 +16,8 @@ from .api import (  # noqa: F401
     GroupedGemv,
     dual_gemv,
     gemm,
+    gemm_from_weight,
+    gemm_from_weight_workspace_bytes,
     gemm_workspace_bytes,
     gemv,
     gemv_swiglu,
@@ -29,6 +31,7 @@ from .api import (  # noqa: F401
     scales_count,
 )
 
-__all__ = ["pack", "pack_fixed", "gemv", "gemv_swiglu", "mlp_gemv", "dual_gemv", "gemm", "GroupedGemv", "layout",
-           "planes_words", "scales_count", "gemv_workspace_bytes", "gemv_swiglu_workspace_bytes",
-           "gemm_workspace_bytes", "RbError", "load"]
+__all__ = ["pack", "pack_fixed", "gemv", "gemv_swiglu", "mlp_gemv", "dual_gemv", "gemm", "gemm_from_weight",
+           "GroupedGemv", "layout", "planes_words", "scales_count", "gemv_workspace_bytes",
+           "gemv_swiglu_workspace_bytes", "gemm_workspace_bytes", "gemm_from_weight_workspace_bytes", "RbError",
+           "load"]

@@ -25,7 +25,8 @@ EXPORTED = ("rb_planes_words", "rb_scales_count", "rb_status_string", "rb_last_e
             "rb_gemv_grouped_workspace_bytes", "rb_gemv_check", "rb_gemv_noalloc",
             "rb_gemm", "rb_gemm_workspace_bytes", "rb_gemm_check",
             "rb_pack_fixed", "rb_dual_gemv", "rb_dual_gemv_workspace_bytes", "rb_gemm_reconstruct",
-            "rb_gemv_swiglu", "rb_gemv_swiglu_workspace_bytes")
+            "rb_gemv_swiglu", "rb_gemv_swiglu_workspace_bytes", "rb_gemm_from_weight",
+            "rb_gemm_from_weight_workspace_bytes")
 
 
 class RbError(RuntimeError):
@@ -79,6 +80,10 @@ def load() -> ctypes.CDLL:
         lib.rb_gemv_swiglu.restype = st
         lib.rb_gemv_swiglu_workspace_bytes.argtypes = [Layout, i32]
         lib.rb_gemv_swiglu_workspace_bytes.restype = sz
+        lib.rb_gemm_from_weight.argtypes = [vp, st, i64, Layout, vp, i64, i32, vp, st, i64, vp, sz, vp]
+        lib.rb_gemm_from_weight.restype = st
+        lib.rb_gemm_from_weight_workspace_bytes.argtypes = [Layout, i32]
+        lib.rb_gemm_from_weight_workspace_bytes.restype = sz
         lib.rb_gemv_grouped.argtypes = [vp, vp, i32, i32, i32, i32, st, st, i32, vp, sz, vp]
         lib.rb_gemv_grouped.restype = st
         lib.rb_gemv_grouped_workspace_bytes.argtypes = [vp, i32, i32, i32]

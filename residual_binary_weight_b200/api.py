@@ -313,6 +313,40 @@ def gemm(planes: torch.Tensor, alpha: torch.Tensor, X: torch.Tensor, group: int 
     return Y
 
 
+def gemm_from_weight_workspace_bytes(M: int, K: int, n_paths: int, group: int, T: int, order: str = "sliced") -> int:
+    return _lib.load().rb_gemm_from_weight_workspace_bytes(layout(M, K, n_paths, group, order), T)
+
+
+def gemm_from_weight(W: torch.Tensor, X: torch.Tensor, n_paths: int = 2, group: int = 0, order: str = "sliced",
+                     Y: Optional[torch.Tensor] = None, y_dtype: torch.dtype = torch.float16,
+                     workspace: Optional[torch.Tensor] = None, check_device: bool = False) -> torch.Tensor:
+    """Training forward: Y[t] = sum_k alpha_k (.) (B_k X[t]) with the planes
+    and scales derived afresh from the full-precision weight W (M x K) in the
+    same call (rb_gemm_from_weight: pack into the workspace, then rb_gemm)."""
+    lib = _lib.load()
+    X = _x2d(X)
+    dev = _require_cuda(W, X, Y, workspace)
+    if W.dim() != 2 or W.stride(1) != 1 or W.dtype not in _DT:
+        raise ValueError("W must be a 2-D fp16/fp32 tensor with unit column stride")
+    M, K = W.shape
+    if X.shape[1] != K:
+        raise ValueError("X must have K columns")
+    T = X.shape[0]
+    if Y is None:
+        Y = torch.empty((T, M), dtype=y_dtype, device=dev)
+    L = layout(M, K, n_paths, group, order)
+    need = lib.rb_gemm_from_weight_workspace_bytes(L, T)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        check(lib.rb_gemm_from_weight(_p(W), _DT[W.dtype], W.stride(0), L, _p(X), X.stride(0), T, _p(Y),
+                                      _DT[Y.dtype], Y.stride(0), _p(workspace),
+                                      workspace.numel() * workspace.element_size(), _stream(dev)))
+        if check_device:
+            check(lib.rb_gemm_check(_p(workspace), _stream(dev)))
+    return Y
+
+
 def pack_fixed(W: torch.Tensor, h: torch.Tensor, g: Optional[torch.Tensor] = None, order: str = "rows",
                planes: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Sign planes of the dual-scale block for given scales: h fp32 [N, M]

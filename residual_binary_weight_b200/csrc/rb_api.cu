@@ -326,6 +326,59 @@ rb_status rb_dual_gemv(const uint32_t* planes, rb_layout L, const float* h, cons
     return RB_OK;
 }
 
+// rb_gemm_from_weight workspace: the rb_gemm workspace, then the planes, the
+// fp32 scales and (one scale per 128 columns) their fp16 copy, each
+// starting on a 256-byte boundary
+struct FromWeightLayout {
+    size_t gemm, planes, alpha, alpha16, total;
+};
+static FromWeightLayout from_weight_layout(rb_layout L, int32_t T) {
+    auto a256 = [](size_t b) { return (b + 255) & ~size_t(255); };
+    FromWeightLayout f{};
+    f.gemm = a256(rb_gemm_workspace_bytes(L, T));
+    f.planes = a256(rb_planes_words(L) * 4);
+    f.alpha = a256(rb_scales_count(L) * 4);
+    f.alpha16 = L.group ? a256(rb_scales_count(L) * 2) : 0;
+    f.total = (f.gemm && f.planes) ? f.gemm + f.planes + f.alpha + f.alpha16 : 0;
+    return f;
+}
+
+size_t rb_gemm_from_weight_workspace_bytes(rb_layout L, int32_t T) {
+    if (check_layout(L) != RB_OK || T < 1 || L.n_paths > 4) return 0;
+    return from_weight_layout(L, T).total;
+}
+
+rb_status rb_gemm_from_weight(const void* W, rb_dtype w_dtype, int64_t ldw, rb_layout L, const void* X, int64_t ldx,
+                              int32_t T, void* Y, rb_dtype y_dtype, int64_t ldy, void* workspace, size_t ws_bytes,
+                              void* stream) {
+    g_last_error.clear();
+    rb_status st = check_layout(L);
+    if (st != RB_OK) return st;
+    // everything rb_pack and rb_gemm would refuse is refused here, before
+    // either is enqueued
+    if (!W || !X || !Y) return fail(RB_ERR_INVALID_ARG, "null W, X or Y");
+    if (!valid_dtype(w_dtype) || !valid_dtype(y_dtype)) return fail(RB_ERR_INVALID_ARG, "bad dtype");
+    if (L.n_paths > 4) return fail(RB_ERR_UNSUPPORTED, "rb_gemm supports 1..4 paths");
+    if (ldw < L.K) return fail(RB_ERR_INVALID_ARG, "ldw=%lld < K=%lld", (long long)ldw, (long long)L.K);
+    if (!aligned16(W) || (ldw * dtype_size(w_dtype)) % 16 != 0)
+        return fail(RB_ERR_ALIGNMENT, "W and its row pitch must be 16-byte aligned");
+    if (L.group == 0 && L.K > 65536) return fail(RB_ERR_UNSUPPORTED, "one scale per row supports K <= 65536");
+    if (T < 1 || T > (1 << 22)) return fail(RB_ERR_UNSUPPORTED, "T=%d outside 1..2^22", T);
+    if (ldx < L.K || ldy < L.M) return fail(RB_ERR_INVALID_ARG, "ldx < K or ldy < M");
+    if (!aligned16(X) || (ldx * 2) % 16 != 0) return fail(RB_ERR_ALIGNMENT, "X and its row pitch must be 16-byte aligned");
+    if (reinterpret_cast<uintptr_t>(Y) & (dtype_size(y_dtype) - 1)) return fail(RB_ERR_ALIGNMENT, "Y misaligned");
+    const FromWeightLayout f = from_weight_layout(L, T);
+    if (!workspace || ws_bytes < f.total || !aligned16(workspace))
+        return fail(RB_ERR_WORKSPACE, "workspace needs %zu bytes (16-byte aligned), got %zu", f.total, ws_bytes);
+    char* ws = static_cast<char*>(workspace);
+    uint32_t* planes = reinterpret_cast<uint32_t*>(ws + f.gemm);
+    float* alpha = reinterpret_cast<float*>(ws + f.gemm + f.planes);
+    void* alpha16 = L.group ? ws + f.gemm + f.planes + f.alpha : nullptr;
+    if ((st = rb_pack(W, w_dtype, ldw, L, planes, alpha, alpha16, stream)) != RB_OK) return st;
+    return rb_gemm(planes, L.group ? alpha16 : alpha, L.group ? RB_F16 : RB_F32, L, X, ldx, T, Y, y_dtype, ldy,
+                   workspace, f.gemm, stream);
+}
+
 size_t rb_gemm_workspace_bytes(rb_layout L, int32_t T) {
     if (check_layout(L) != RB_OK || T < 1) return 0;
     if (T > GEMM_DEC_MAX_T) return GEMM_HEADER_BYTES;

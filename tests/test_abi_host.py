@@ -248,3 +248,26 @@ def test_dual_block_rejects_bad_arguments_before_launch():
     assert call(g=p(FAKE + 2)) == "RB_ERR_ALIGNMENT"
     assert call(x=p(FAKE + 2)) == "RB_ERR_ALIGNMENT"
     assert call(wsb=need - 1) == "RB_ERR_WORKSPACE"
+
+
+def test_gemm_from_weight_rejections():
+    """Refused before anything is enqueued (no GPU needed)."""
+    lib = _lib.load()
+    p = ctypes.c_void_p
+    L = Layout(256, 1024, 2, 0, 1, 0)
+    need = lib.rb_gemm_from_weight_workspace_bytes(L, 300)
+    assert need >= 256 + 2 * 256 * 1024 // 8 + 2 * 256 * 4
+    args = dict(W=p(FAKE), wd=1, ldw=1024, X=p(FAKE), ldx=1024, T=300, Y=p(FAKE), yd=1, ldy=256)
+
+    def call(L=L, ws=need, **kw):
+        a = dict(args, **kw)
+        return _status(lib.rb_gemm_from_weight(a["W"], a["wd"], a["ldw"], L, a["X"], a["ldx"], a["T"], a["Y"],
+                                               a["yd"], a["ldy"], p(FAKE), ws, None))
+    assert call(W=None) == "RB_ERR_INVALID_ARG"
+    assert call(L=Layout(256, 1024, 5, 0, 1, 0)) == "RB_ERR_UNSUPPORTED"
+    assert call(ldw=1000) == "RB_ERR_INVALID_ARG"
+    assert call(W=p(FAKE + 8)) == "RB_ERR_ALIGNMENT"
+    assert call(T=0) == "RB_ERR_UNSUPPORTED"
+    assert call(ldy=100) == "RB_ERR_INVALID_ARG"
+    assert call(ws=need - 16) == "RB_ERR_WORKSPACE"
+    assert lib.rb_gemm_from_weight_workspace_bytes(Layout(256, 1000, 2, 0, 1, 0), 300) == 0
