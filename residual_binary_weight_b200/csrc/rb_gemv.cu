@@ -332,7 +332,9 @@ __device__ __forceinline__ void scan_jobs(const GvArgs& p, LowSmem& lo, int n_jo
     cta_sync();
 }
 
-template <int NP, bool G128, bool A16, bool SLICED>
+// GATE: the SiLU-gated pair (GvArgs::swiglu), a separate instantiation so
+// that the plain kernel's epilogue carries none of it
+template <int NP, bool G128, bool A16, bool SLICED, bool GATE = false>
 __global__ void __launch_bounds__(THREADS, 1) gemv_lut_kernel(GvArgs p, uint32_t* __restrict__ hdr,
                                                               uint32_t* __restrict__ ctrs,
                                                               float* __restrict__ parts) {
@@ -641,7 +643,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_lut_kernel(GvArgs p, uint32_t
         // yv: sum over the paths (with the SiLU gate: over the gate's paths,
         // yv2 over the up projection's)
         float yv = 0.0f, yv2 = 0.0f;
-        const bool gated = p.swiglu != 0;
+        constexpr bool gated = GATE;
         const int64_t my_row = static_cast<int64_t>(ue.rb) * C::R + warp * C::RW + lane;
         const bool row_ok = lane < C::RW && my_row < M;
         if (row_ok) {
@@ -707,9 +709,9 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_lut_kernel(GvArgs p, uint32_t
     }
 }
 
-template <int NP, bool G128, bool A16, bool SLICED>
+template <int NP, bool G128, bool A16, bool SLICED, bool GATE = false>
 cudaError_t launch_one(const GvArgs& a, const GvPlan& plan, cudaStream_t s) {
-    auto kern = gemv_lut_kernel<NP, G128, A16, SLICED>;
+    auto kern = gemv_lut_kernel<NP, G128, A16, SLICED, GATE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
     uint32_t* hdr = static_cast<uint32_t*>(a.workspace);
@@ -725,6 +727,15 @@ cudaError_t launch_one(const GvArgs& a, const GvPlan& plan, cudaStream_t s) {
 
 template <int NP, bool SLICED>
 cudaError_t launch_np(const GvArgs& a, const GvPlan& plan, cudaStream_t s) {
+    if (a.swiglu) {
+        if constexpr (NP % 2 == 0) {
+            if (a.group == 0) return launch_one<NP, false, false, SLICED, true>(a, plan, s);
+            return a.alpha_f16 ? launch_one<NP, true, true, SLICED, true>(a, plan, s)
+                               : launch_one<NP, true, false, SLICED, true>(a, plan, s);
+        } else {
+            return cudaErrorInvalidValue;   // a gated pair has an even number of paths
+        }
+    }
     if (a.group == 0) return launch_one<NP, false, false, SLICED>(a, plan, s);   // scale dtype read at run time
     return a.alpha_f16 ? launch_one<NP, true, true, SLICED>(a, plan, s) : launch_one<NP, true, false, SLICED>(a, plan, s);
 }
