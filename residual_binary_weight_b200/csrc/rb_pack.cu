@@ -43,6 +43,45 @@ __device__ __forceinline__ float abs_sum8(const float* v) {
            ((fabsf(v[4]) + fabsf(v[5])) + (fabsf(v[6]) + fabsf(v[7])));
 }
 
+// Pairs of fp32 values in one 64-bit register, added with one add.f32x2.
+__device__ __forceinline__ uint64_t pack_f2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void unpack_f2(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t add_f2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+// 32 weights as fp32 with -0.0 turned into +0.0 (sign(0) = +1): fp16 values
+// are widened and added to +0.0 in one mixed-precision add.
+__device__ __forceinline__ void load32_nz(const __half* p, float (&v)[32]) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint4 u = __ldcs(reinterpret_cast<const uint4*>(p) + i);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const unsigned short h = static_cast<unsigned short>(w[j >> 1] >> (16 * (j & 1)));
+            asm("add.rn.f32.f16 %0, %1, %2;" : "=f"(v[8 * i + j]) : "h"(h), "f"(0.0f));
+        }
+    }
+}
+__device__ __forceinline__ void load32_nz(const float* p, float (&v)[32]) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float t[8];
+        load8(p + 8 * i, t);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[8 * i + e] = __fadd_rn(t[e], 0.0f);
+    }
+}
+
 __device__ __forceinline__ double warp_sum(double v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(FULL_MASK, v, o);
@@ -163,22 +202,25 @@ pack_words_kernel(const WT* __restrict__ W, int64_t ldw, int M, int K, int N, bo
     const double inv_k = 1.0 / static_cast<double>(K);
     float r[32];
     if (active) {
-        load32(W + static_cast<int64_t>(row) * ldw + 32 * tr, r);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) r[e] = __fadd_rn(r[e], 0.0f);   // -0.0 -> +0.0 (sign(0) = +1)
+        load32_nz(W + static_cast<int64_t>(row) * ldw + 32 * tr, r);   // -0.0 -> +0.0 (sign(0) = +1)
     } else {
 #pragma unroll
         for (int e = 0; e < 32; ++e) r[e] = 0.0f;
     }
     for (int k = 0; k < N; ++k) {
-        float t[16];
+        // balanced tree: |r| of neighbours, then pairs of partial sums in
+        // f32x2 registers (lane e with lane e + 8), then the two lanes
+        uint64_t t2[8];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) t[e] = fabsf(r[2 * e]) + fabsf(r[2 * e + 1]);
+        for (int e = 0; e < 8; ++e)
+            t2[e] = pack_f2(fabsf(r[2 * e]) + fabsf(r[2 * e + 1]), fabsf(r[2 * e + 16]) + fabsf(r[2 * e + 17]));
 #pragma unroll
-        for (int w = 8; w >= 1; w >>= 1)
+        for (int w = 4; w >= 1; w >>= 1)
 #pragma unroll
-            for (int e = 0; e < w; ++e) t[e] = t[2 * e] + t[2 * e + 1];
-        double sum = static_cast<double>(t[0]);
+            for (int e = 0; e < w; ++e) t2[e] = add_f2(t2[e], t2[e + w]);
+        float tlo, thi;
+        unpack_f2(t2[0], tlo, thi);
+        double sum = static_cast<double>(tlo + thi);
         if (tpr <= 32) {
             for (int o = 1; o < tpr; o <<= 1) sum += __shfl_xor_sync(FULL_MASK, sum, o);
         } else {
@@ -211,8 +253,11 @@ pack_words_kernel(const WT* __restrict__ W, int64_t ldw, int M, int K, int N, bo
         if (active && k + 1 < N) {
             const uint32_t neg_a = __float_as_uint(-a);
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-                r[e] = __fadd_rn(r[e], __uint_as_float((__float_as_uint(r[e]) & 0x80000000u) ^ neg_a));
+            for (int e = 0; e < 16; ++e) {
+                const float q0 = __uint_as_float((__float_as_uint(r[2 * e]) & 0x80000000u) ^ neg_a);
+                const float q1 = __uint_as_float((__float_as_uint(r[2 * e + 1]) & 0x80000000u) ^ neg_a);
+                unpack_f2(add_f2(pack_f2(r[2 * e], r[2 * e + 1]), pack_f2(q0, q1)), r[2 * e], r[2 * e + 1]);
+            }
         }
         if (active) {
             const size_t wo = sliced ? ((static_cast<size_t>(k) * S + (tr >> 4)) * M + row) * 16 + (tr & 15)
@@ -225,7 +270,7 @@ pack_words_kernel(const WT* __restrict__ W, int64_t ldw, int M, int K, int N, bo
 // One scale per (path, row, 128 columns): lanes 4g..4g+3 of a warp own group g
 // (eight groups per warp per step); lane (4g + q) holds columns 32q..32q+31.
 template <typename WT>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(128)
 pack_g128_kernel(const WT* __restrict__ W, int64_t ldw, int M, int K, int N, bool sliced,
                  uint32_t* __restrict__ planes, float* __restrict__ alpha,
                  __half* __restrict__ alpha16) {
@@ -244,9 +289,7 @@ pack_g128_kernel(const WT* __restrict__ W, int64_t ldw, int M, int K, int N, boo
         const int wi = gi * 4 + (lane & 3);
         float r[32];
         if (valid) {
-            load32(W + row * ldw + 32 * wi, r);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) r[e] = __fadd_rn(r[e], 0.0f);   // -0.0 -> +0.0 (sign(0) = +1)
+            load32_nz(W + row * ldw + 32 * wi, r);   // -0.0 -> +0.0 (sign(0) = +1)
         } else {
 #pragma unroll
             for (int e = 0; e < 32; ++e) r[e] = 0.0f;
@@ -267,8 +310,11 @@ pack_g128_kernel(const WT* __restrict__ W, int64_t ldw, int M, int K, int N, boo
             if (k + 1 < N) {
                 const uint32_t neg_a = __float_as_uint(-a);
 #pragma unroll
-                for (int e = 0; e < 32; ++e)
-                    r[e] = __fadd_rn(r[e], __uint_as_float((__float_as_uint(r[e]) & 0x80000000u) ^ neg_a));
+                for (int e = 0; e < 16; ++e) {
+                    const float q0 = __uint_as_float((__float_as_uint(r[2 * e]) & 0x80000000u) ^ neg_a);
+                    const float q1 = __uint_as_float((__float_as_uint(r[2 * e + 1]) & 0x80000000u) ^ neg_a);
+                    unpack_f2(add_f2(pack_f2(r[2 * e], r[2 * e + 1]), pack_f2(q0, q1)), r[2 * e], r[2 * e + 1]);
+                }
             }
             if (valid) {
                 const int64_t wo = sliced ? ((k * S + (wi >> 4)) * M + row) * 16 + (wi & 15)
@@ -301,7 +347,10 @@ cudaError_t launch_words(const PackArgs& a, cudaStream_t s) {
     } else {
         tpr = (words + 31) & ~31;
     }
-    const int rows_per_cta = tpr >= 512 ? 1 : 512 / tpr;   // 512-thread CTAs: two per SM
+    // 128-thread CTAs (one row for K >= 4096): many small CTAs per SM hide the
+    // load latency of one behind the arithmetic of others (512-thread CTAs
+    // were 15 % slower on 11008 x 4096)
+    const int rows_per_cta = tpr >= 128 ? 1 : 128 / tpr;
     const int64_t blocks = (a.M + rows_per_cta - 1) / rows_per_cta;
     pack_words_kernel<WT><<<static_cast<unsigned>(blocks), rows_per_cta * tpr, 0, s>>>(
         static_cast<const WT*>(a.W), a.ldw, static_cast<int>(a.M), static_cast<int>(a.K), a.n_paths, a.sliced, tpr,
@@ -331,11 +380,11 @@ template <typename WT>
 cudaError_t launch_g128(const PackArgs& a, cudaStream_t s) {
     const int64_t groups = a.M * (a.K >> 7);
     const int64_t warps_needed = (groups + 7) / 8;
-    int64_t blocks = (warps_needed + 7) / 8;
-    const int64_t cap = static_cast<int64_t>(device_sm_count()) * 8;
-    if (blocks > cap) blocks = cap;
+    // 128-thread CTAs, one group of 8 per warp: many small CTAs per SM hide
+    // load latency (a grid capped at 8 CTAs of 256 per SM was 2 % slower)
+    int64_t blocks = (warps_needed + 3) / 4;
     if (blocks < 1) blocks = 1;
-    pack_g128_kernel<WT><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+    pack_g128_kernel<WT><<<static_cast<unsigned>(blocks), 128, 0, s>>>(
         static_cast<const WT*>(a.W), a.ldw, static_cast<int>(a.M), static_cast<int>(a.K),
         a.n_paths, a.sliced, a.planes, a.alpha, a.alpha16);
     return cudaGetLastError();
