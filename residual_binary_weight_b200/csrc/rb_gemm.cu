@@ -211,7 +211,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, GemmArgs a) {
         // ---------------------------------------------------------- MMA issuer
         // the whole warp runs the loop (warp-uniform operands); one elected
         // lane issues each MMA
-        constexpr uint32_t idesc = instr_desc(BN);
+        // The last token tile of a block may be narrower than BN: its MMAs
+        // compute only the columns that hold tokens, rounded up to 16 (the
+        // TMA box still fills BN rows, zeros past T; the epilogue stores
+        // tokens < T only). With 240-wide tiles over 2048 tokens the ninth
+        // tile holds 128 tokens, and those CTAs run last.
+        const int t_left = a.T - tok_tile * BN;
+        const uint32_t idesc = instr_desc(t_left >= BN ? BN : ((t_left + 15) & ~15));
         bool ok = true;
         for (int kb = 0; kb < nk && ok; ++kb) {
             const int s = kb % STAGES;
