@@ -224,9 +224,9 @@ class GroupedGemv:
 
     The descriptor table is uploaded once at construction; call ``run()`` for
     every step (the x tensors are read and the y tensors written in place).
-    A y tensor may also be a pinned host tensor: the kernel then writes its
-    rows straight into host memory over the bus, so the result needs no
-    separate device-to-host copy.
+    An x or y tensor may also be a pinned host tensor: the kernel then reads
+    x from, or writes y to, host memory over the bus (zero-copy), so a step
+    needs no separate host-to-device or device-to-host copy.
     """
 
     def __init__(self, items: Sequence[tuple], n_paths: int, group: int = 0, T: int = 1):
@@ -238,7 +238,9 @@ class GroupedGemv:
         adt = ydt = order = None
         dev = None
         for i, (planes, alpha, x, y) in enumerate(self.items):
-            dev = _require_cuda(planes, alpha, x, None if (not y.is_cuda and y.is_pinned()) else y)
+            host_x = not x.is_cuda and x.is_pinned()
+            host_y = not y.is_cuda and y.is_pinned()
+            dev = _require_cuda(planes, alpha, None if host_x else x, None if host_y else y)
             K = x.shape[-1]
             N, M, o = _planes_geometry(planes, K)
             order = o if order is None else order
@@ -253,8 +255,9 @@ class GroupedGemv:
             ydt = y.dtype if ydt is None else ydt
             if alpha.dtype != adt or y.dtype != ydt:
                 raise ValueError("all items must share the scale and output dtypes")
+            x_ptr = x.data_ptr() if x.is_cuda else _mapped_host_ptr(x)
             y_ptr = y.data_ptr() if y.is_cuda else _mapped_host_ptr(y)
-            self.host[i] = GemvDesc(planes.data_ptr(), alpha.data_ptr(), x.data_ptr(), y_ptr, M, K)
+            self.host[i] = GemvDesc(planes.data_ptr(), alpha.data_ptr(), x_ptr, y_ptr, M, K)
         self.device = dev
         raw = bytes(self.host)
         self.dev_descs = torch.frombuffer(bytearray(raw), dtype=torch.uint8).to(dev)

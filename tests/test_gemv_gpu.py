@@ -181,6 +181,26 @@ def test_grouped_output_in_pinned_host_memory():
         assert nbad == 0, worst
 
 
+@pytest.mark.parametrize("T", [1, 2])
+def test_grouped_input_and_output_in_pinned_host_memory(T):
+    """x and y given as pinned host tensors (zero-copy): the launch reads x and
+    writes y over the bus, and y equals the device run's and the oracle's."""
+    items, refs = _grouped_case("llama2_7b_decode", 1, 16, T, 2, 0, False, "sliced")
+    host_items = [(p, a, x.cpu().pin_memory(), torch.empty(y.shape, dtype=y.dtype, pin_memory=True).fill_(float("nan")))
+                  for p, a, x, y in items]
+    g = rb.GroupedGemv(host_items, n_paths=2, group=0, T=T)
+    g.run()
+    torch.cuda.synchronize()
+    g.check_device_flag()
+    gd = rb.GroupedGemv(items, n_paths=2, group=0, T=T)
+    gd.run()
+    torch.cuda.synchronize()
+    for (_, _, _, yh), (_, _, _, yd), (y_ref, den) in zip(host_items, items, refs):
+        assert torch.equal(yh, yd.cpu())
+        nbad, worst = oracle.compare_outputs(yh.float().numpy().reshape(y_ref.shape), y_ref, den)
+        assert nbad == 0, worst
+
+
 @pytest.mark.parametrize("order", ORDERS)
 def test_grouped_many_units_per_cta(order):
     """The largest grouped launch (2047 descriptors) of small matrices at
