@@ -29,18 +29,18 @@
 // into the workspace, and the last of its CTAs to finish adds the parts in
 // CTA order (deterministic) and stores Y.
 //
-// Roles (16 warps):
-//   warps 0-7   expansion: warp w writes rows 32 (w % 4) .. + 31 (its tensor
-//               memory lane quarter) of every path, for the stages i of the
-//               CTA's range with i % 2 == w / 4;
-//   warps 8-11  epilogue: tcgen05.ld of the accumulators, per-row scales,
+// Roles (NG = 3 expansion groups where the plane words come by TMA, else 2):
+//   warps 0 .. 4 NG - 1   expansion: warp w writes rows 32 (w % 4) .. + 31
+//               (its tensor-memory lane quarter) of every path, for the
+//               stages i of the CTA's range with i % NG == w / 4;
+//   next 4 warps  epilogue: tcgen05.ld of the accumulators, per-row scales,
 //               store or partial sums;
-//   warp 12     TMA loads of the permuted X tiles;
-//   warps 13-14 MMA issue, alternate stages (warp 13 allocates tensor memory);
-//   warp 15     TMA loads of the plane words (per-row scales, >= 4 words per
+//   next warp   TMA loads of the permuted X tiles;
+//   next 2      MMA issue, alternate stages (the first allocates tensor memory);
+//   last warp   TMA loads of the plane words (per-row scales, >= 4 words per
 //               row and stage) into an 8-stage shared-memory ring, so that
 //               the expansion warps issue no global loads.
-// Warps 12-15 run their loops converged (warp-uniform operands) and issue
+// The TMA, MMA and plane warps run their loops converged (warp-uniform operands) and issue
 // through one elected lane. mbarriers: full[s] (TMA bytes + the 4 warps of
 // the stage's group), empty[s] (MMAs of stage s done), acc_full[b] /
 // acc_empty[b] (accumulator buffer b filled / read), pfull[k] / pempty[k]
@@ -58,11 +58,12 @@ namespace {
 
 using namespace tc;
 
-constexpr int THREADS = 512;
-constexpr int EPI_WARP0 = 8;
-constexpr int TMA_WARP = 12;
-constexpr int MMA_WARP = 13;   // and MMA_WARP + 1
-constexpr int PL_WARP = 15;
+// Warp roles for NG expansion groups of 4 warps: [0, 4 NG) expansion, then 4
+// epilogue warps, the X TMA warp, two MMA warps and the plane-word TMA warp.
+__host__ __device__ constexpr int epi_warp0(int ng) { return 4 * ng; }
+__host__ __device__ constexpr int tma_warp(int ng) { return 4 * ng + 4; }
+__host__ __device__ constexpr int mma_warp(int ng) { return 4 * ng + 5; }   // and the next one
+__host__ __device__ constexpr int pl_warp(int ng) { return 4 * ng + 7; }
 
 struct DecArgs {
     uint32_t* err;          // the call's device error word
@@ -100,6 +101,14 @@ struct DecCfg {
     static constexpr int ACC_COLS = ACC_BUF * NACC * ACC_STRIDE;
     static constexpr int STAGES_FIT = (512 - ACC_COLS) / A_STAGE_COLS;
     static constexpr int STAGES = STAGES_FIT < 8 ? STAGES_FIT : 8;
+    // Expansion groups: three where the plane words come by TMA (no register
+    // ring, so 640 threads fit), else two. A group waits on slot s for the
+    // MMAs of stage i - STAGES; its previous stage (i - NG) waited for those
+    // of i - NG - STAGES, and MMAs complete in issue order, so with
+    // NG <= STAGES the barrier is never two phases behind the waiter (which
+    // would let a parity wait pass early).
+    static constexpr int NG = (!G128 && SW / 32 >= 4) ? 3 : 2;
+    static constexpr int THREADS = 32 * (4 * NG + 8);
     static constexpr uint32_t SUB_BYTES = NMMA * 128;      // one 128-byte-wide box of NMMA rows
     static constexpr uint32_t B_TILE_BYTES = SUB * SUB_BYTES;
     // plane words through TMA into a shared-memory ring (per-row scales, at
@@ -112,6 +121,7 @@ struct DecCfg {
     // at least 120 KB, so that two CTAs never share an SM's tensor memory
     static constexpr uint32_t SMEM_BYTES = SMEM_USED < 120u * 1024u ? 120u * 1024u : SMEM_USED;
     static_assert(STAGES >= 2, "operand stages do not fit beside the accumulators");
+    static_assert(NG <= STAGES, "an expansion group could run two phases ahead of a stage slot");
     static_assert(F8 ? (BN == 4 || BN == 8 || BN == 16) : (BN == 16 || BN == 32 || BN == 64), "token tile");
     static_assert(!F8 || (!G128 && NP <= 2), "fp8 operands: per-row scales, 1-2 paths");
     static_assert(SUB_BYTES % 1024 == 0, "X box must keep the 1024-byte swizzle alignment");
@@ -122,10 +132,11 @@ __device__ __forceinline__ int64_t range_lo(int64_t c, int64_t total, int64_t G)
 __device__ __forceinline__ int64_t cta_of(int64_t g, int64_t total, int64_t G) { return ((g + 1) * G - 1) / total; }
 
 template <int NP, int BN, bool G128, bool F8>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(DecCfg<NP, BN, G128, F8>::THREADS, 1)
 gemm_dec_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap pmap, DecArgs a) {
     using C = DecCfg<NP, BN, G128, F8>;
-    constexpr int STAGES = C::STAGES, ACC_BUF = C::ACC_BUF, SW = C::SW, WPS = C::WPS;
+    constexpr int STAGES = C::STAGES, ACC_BUF = C::ACC_BUF, SW = C::SW, WPS = C::WPS, NG = C::NG;
+    constexpr int EPI_WARP0 = epi_warp0(NG), TMA_WARP = tma_warp(NG), MMA_WARP = mma_warp(NG), PL_WARP = pl_warp(NG);
     extern __shared__ __align__(1024) unsigned char dsm[];
     const uint32_t raw = smem_addr(dsm);
     const uint32_t tiles_s = (raw + 1023u) & ~1023u;
@@ -317,10 +328,10 @@ gemm_dec_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant_
         }
         if (elect_one()) umma_commit(fin_bar);   // every MMA issued above has completed once both arrive
         __syncwarp();
-    } else if (warp < 8) {
+    } else if (warp < 4 * NG) {
         // ---------------------------------------------------------- expansion
         // Thread = one row of the tile (its tensor-memory lane), all paths,
-        // the stages i with i % 2 == grp. The plane words of a stage (SW / 32
+        // the stages i with i % NG == grp. The plane words of a stage (SW / 32
         // per path) come from the TMA ring in shared memory (PTMA) or are
         // loaded PR of the group's stages ahead into registers.
         const int q = warp & 3, grp = warp >> 2;
@@ -335,7 +346,7 @@ gemm_dec_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant_
         constexpr int PR = F8 ? 2 : NP <= 2 ? 4 : 2;   // stages of this group loaded ahead
         const int64_t n = hi - lo;
         // (tile, stage-in-tile) of the next stage to load, stepping by 2
-        int64_t lt = (lo + grp) / S;
+        int64_t lt = (lo + grp) / S;   // (tile, stage) of the next register-ring load
         int lkb = static_cast<int>(lo + grp - lt * S);
         WV ring[C::PTMA ? 1 : PR][NP][NV];
         uint32_t nring[C::PTMA ? 1 : PR][NP];
@@ -357,7 +368,7 @@ gemm_dec_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant_
                     ndst[p] = 0xBC00BC00u;   // -1.0 in both halves
                 }
             }
-            lkb += 2;
+            lkb += NG;
             while (lkb >= S) {
                 lkb -= static_cast<int>(S);
                 ++lt;
@@ -417,7 +428,7 @@ gemm_dec_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant_
             uint32_t ng[NP];
 #pragma unroll
             for (int p = 0; p < NP; ++p) ng[p] = 0xBC00BC00u;   // -1.0 in both halves
-            for (int64_t i = grp; i < n; i += 2) {
+            for (int64_t i = grp; i < n; i += NG) {
                 const int ps = static_cast<int>(i % C::PS);
                 if (!__all_sync(FULL_MASK, mbar_wait(pfull(ps), static_cast<uint32_t>(i / C::PS) & 1u, abort_flag,
                                                      err, 4u)))
@@ -434,8 +445,8 @@ gemm_dec_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant_
                 // warp-uniform: the tensor-memory stores are .sync.aligned
                 if (!__all_sync(FULL_MASK, mbar_wait(empty_bar(s), ph ^ 1u, abort_flag, err, 4u))) break;
                 expand_stage(cur, ng, s);
-                s += 2;
-                if (s >= STAGES) {
+                s += NG;
+                while (s >= STAGES) {
                     s -= STAGES;
                     ph ^= 1u;
                 }
@@ -443,12 +454,12 @@ gemm_dec_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant_
         } else {
 #pragma unroll
             for (int d = 0; d < PR; ++d)
-                if (grp + 2 * d < n) load_stage(ring[d], nring[d]);
+                if (grp + NG * d < n) load_stage(ring[d], nring[d]);
             bool go = true;
-            for (int64_t i0 = grp; i0 < n && go; i0 += 2 * PR) {
+            for (int64_t i0 = grp; i0 < n && go; i0 += NG * PR) {
 #pragma unroll
                 for (int d = 0; d < PR; ++d) {
-                    const int64_t i = i0 + 2 * d;
+                    const int64_t i = i0 + NG * d;
                     if (i < n && go) {
                         WV cur[NP][NV];
                         uint32_t ng[NP];
@@ -458,15 +469,15 @@ gemm_dec_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant_
                             for (int v = 0; v < NV; ++v) cur[p][v] = ring[d][p][v];
                             ng[p] = nring[d][p];
                         }
-                        if (i + 2 * PR < n) load_stage(ring[d], nring[d]);
+                        if (i + NG * PR < n) load_stage(ring[d], nring[d]);
                         // warp-uniform: the tensor-memory stores are .sync.aligned
                         if (!__all_sync(FULL_MASK, mbar_wait(empty_bar(s), ph ^ 1u, abort_flag, err, 4u))) {
                             go = false;
                         } else {
                             expand_stage(cur, ng, s);
                         }
-                        s += 2;
-                        if (s >= STAGES) {
+                        s += NG;
+                        while (s >= STAGES) {
                             s -= STAGES;
                             ph ^= 1u;
                         }
@@ -724,7 +735,7 @@ cudaError_t launch_dec(const DecArgs& a, const void* Xp, int grid, cudaStream_t 
     auto kern = gemm_dec_kernel<NP, BN, G128, F8>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    kern<<<grid, THREADS, C::SMEM_BYTES, s>>>(map, pmap, a);
+    kern<<<grid, C::THREADS, C::SMEM_BYTES, s>>>(map, pmap, a);
     return cudaGetLastError();
 }
 
