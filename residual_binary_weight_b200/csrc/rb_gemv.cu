@@ -343,6 +343,12 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_lut_kernel(GvArgs p, uint32_t
     extern __shared__ __align__(16) unsigned char dsm[];
     LowSmem& lo = *reinterpret_cast<LowSmem*>(dsm);
 
+    // Programmatic dependent launch: the next kernel of the stream may be
+    // launched now (its CTAs start as this grid's CTAs leave their SMs and
+    // wait below until this grid has finished), and this grid waits here for
+    // the one before it: nothing above touches global memory.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     // The call's error word is cleared here, not by a memset before the
     // launch: every condition below is detected by every CTA, CTA 0
     // included, after this store, so a flag another CTA raised before it is
@@ -721,8 +727,20 @@ cudaError_t launch_one(const GvArgs& a, const GvPlan& plan, cudaStream_t s) {
     size_t grid = plan.units;
     if (grid > static_cast<size_t>(sms)) grid = sms;
     if (grid < 1) grid = 1;
-    kern<<<static_cast<unsigned>(grid), THREADS, SMEM_BYTES, s>>>(a, hdr, ctrs, parts);
-    return cudaGetLastError();
+    // launched as a programmatic dependent of the stream's previous kernel
+    // (the kernel waits for it with griddepcontrol.wait before any global
+    // access), so the launch overlaps that kernel's tail
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, a, hdr, ctrs, parts);
 }
 
 template <int NP, bool SLICED>
