@@ -52,6 +52,7 @@
 #include <cuda_fp8.h>
 
 #include <type_traits>
+#include <utility>
 
 namespace rb {
 namespace {
@@ -188,6 +189,10 @@ gemm_dec_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant_
     __syncthreads();
     fence_after();
     const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(dsm + (tmem_slot - raw));
+    // programmatic dependent launch: the barriers and tensor memory above are
+    // set up while the operand pre-pass may still run; wait for it (and
+    // everything before it) here, before the first global access
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     if (warp == TMA_WARP) {
         // ------------------------------------------------------------ X tiles
@@ -616,6 +621,11 @@ gemm_dec_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant_
 // The pre-pass also clears the call's error word and the arrival counters
 // of the main kernel (it runs before it on the same stream).
 __device__ __forceinline__ void clear_call_state(uint32_t* err, uint32_t* counters, int64_t n_ctr, int64_t idx) {
+    // programmatic dependent launch: let the main kernel launch and set up;
+    // wait for the previous kernel of the stream (which may still read this
+    // workspace) before the first global access
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     if (idx == 0) *err = 0u;
     const int64_t step = static_cast<int64_t>(gridDim.x) * blockDim.x;
     for (int64_t i = idx; i < n_ctr; i += step) counters[i] = 0u;
@@ -720,6 +730,23 @@ cudaError_t make_plane_map(CUtensorMap* map, const uint32_t* planes, int64_t M, 
     return cudaSuccess;
 }
 
+// Launch as a programmatic dependent of the stream's previous kernel (the
+// kernels wait for it with griddepcontrol.wait before any global access).
+template <typename... P, typename... A>
+cudaError_t launch_pdl(void (*kern)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, A&&... args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<A>(args)...);
+}
+
 template <int NP, int BN, bool G128, bool F8>
 cudaError_t launch_dec(const DecArgs& a, const void* Xp, int grid, cudaStream_t s) {
     using C = DecCfg<NP, BN, G128, F8>;
@@ -735,8 +762,7 @@ cudaError_t launch_dec(const DecArgs& a, const void* Xp, int grid, cudaStream_t 
     auto kern = gemm_dec_kernel<NP, BN, G128, F8>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    kern<<<grid, C::THREADS, C::SMEM_BYTES, s>>>(map, pmap, a);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, s, map, pmap, a);
 }
 
 template <int NP, bool G128>
@@ -795,13 +821,14 @@ cudaError_t launch_gemm_dec(const uint32_t* planes, const void* alpha, bool alph
     __half* Xp = reinterpret_cast<__half*>(ws + GEMM_HEADER_BYTES + pl.counters_bytes + pl.partials_bytes);
     const int64_t nthr = (K >> 5) * T;
     uint32_t* err = reinterpret_cast<uint32_t*>(ws) + 1;
+    cudaError_t e;
     if (pl.f8)
-        split_x_f8_kernel<<<static_cast<unsigned>((nthr + 127) / 128), 128, 0, s>>>(
-            static_cast<const __half*>(X), ldx, T, K, reinterpret_cast<uint8_t*>(Xp), err, counters, pl.tiles);
+        e = launch_pdl(split_x_f8_kernel, dim3(static_cast<unsigned>((nthr + 127) / 128)), dim3(128), 0, s,
+                       static_cast<const __half*>(X), ldx, T, K, reinterpret_cast<uint8_t*>(Xp), err, counters,
+                       static_cast<int64_t>(pl.tiles));
     else
-        permute_x_kernel<<<static_cast<unsigned>((nthr + 255) / 256), 256, 0, s>>>(
-            static_cast<const __half*>(X), ldx, T, K, Xp, err, counters, pl.tiles);
-    cudaError_t e = cudaGetLastError();
+        e = launch_pdl(permute_x_kernel, dim3(static_cast<unsigned>((nthr + 255) / 256)), dim3(256), 0, s,
+                       static_cast<const __half*>(X), ldx, T, K, Xp, err, counters, static_cast<int64_t>(pl.tiles));
     if (e != cudaSuccess) return e;
     DecArgs a{err, counters, partials, planes, alpha, Y, M, K, ldy, pl.tiles,
               pl.total, T, sliced, alpha_f16, y_f16};
