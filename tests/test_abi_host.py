@@ -271,3 +271,39 @@ def test_gemm_from_weight_rejections():
     assert call(ldy=100) == "RB_ERR_INVALID_ARG"
     assert call(ws=need - 16) == "RB_ERR_WORKSPACE"
     assert lib.rb_gemm_from_weight_workspace_bytes(Layout(256, 1000, 2, 0, 1, 0), 300) == 0
+
+
+def test_matvec_workspace_layout_and_counter_zone():
+    """A K-split plan needs the 256-byte header, the fixed 64 KB counter zone
+    and its fp32 partial sums; a plan that would need more counters than the
+    zone holds does not split (header only); the SiLU-gated pair keeps two
+    partial sums per row."""
+    lib = _lib.load()
+    L = Layout(512, 8192, 2, 0, 1, 0)
+    b = lib.rb_gemv_workspace_bytes(L, 1)
+    assert b > 256 + 65536 and (b - 256 - 65536) % (4 * 512) == 0   # partials: nch x T x M fp32
+    nch = (b - 256 - 65536) // (4 * 512)
+    assert nch >= 2
+    # 257 row blocks of 512 rows x 64 tokens = 16448 counters > 16384: no split
+    assert lib.rb_gemv_workspace_bytes(Layout(512 * 257, 8192, 2, 0, 1, 0), 64) == 256
+    g = lib.rb_gemv_swiglu_workspace_bytes(Layout(512, 8192, 1, 0, 1, 0), 1)
+    assert g > 256 + 65536 and (g - 256 - 65536) % (2 * 4 * 512) == 0   # two sums per row and chunk
+    assert lib.rb_gemv_swiglu_workspace_bytes(Layout(512, 8192, 5, 0, 1, 0), 1) == 0   # > 4 paths per matrix
+
+
+def test_swiglu_rejections():
+    lib = _lib.load()
+    p = ctypes.c_void_p
+    L = Layout(256, 1024, 2, 0, 1, 0)
+    ws = lib.rb_gemv_swiglu_workspace_bytes(L, 1)
+
+    def call(L=L, **kw):
+        a = dict(planes=p(FAKE), alpha=p(FAKE), x=p(FAKE), T=1, h=p(FAKE), ldh=256)
+        a.update(kw)
+        return _status(lib.rb_gemv_swiglu(a["planes"], a["alpha"], 0, L, a["x"], 1024, a["T"], a["h"], 1, a["ldh"],
+                                          p(FAKE), max(ws, 256), None))
+    assert call(planes=None) == "RB_ERR_INVALID_ARG"
+    assert call(L=Layout(256, 1024, 5, 0, 1, 0)) == "RB_ERR_UNSUPPORTED"
+    assert call(T=65) == "RB_ERR_UNSUPPORTED"
+    assert call(ldh=100) == "RB_ERR_INVALID_ARG"
+    assert call(h=p(FAKE + 1)) == "RB_ERR_ALIGNMENT"
