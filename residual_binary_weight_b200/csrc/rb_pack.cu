@@ -182,12 +182,14 @@ __device__ __forceinline__ void load32(const WT* p, float (&v)[32]) {
 // CTA packs rows_per_cta rows; |R| is summed in fp32 over the 32 values of
 // a word (balanced tree), then in fp64 over the words of the row (warp
 // shuffles, then the row's warps through shared memory, in a fixed order).
-template <typename WT>
+// NPC: the path count as a compile-time constant (1..4), 0 to read N
+template <typename WT, int NPC>
 __global__ void __launch_bounds__(1024)
-pack_words_kernel(const WT* __restrict__ W, int64_t ldw, int M, int K, int N, bool sliced, int tpr,
+pack_words_kernel(const WT* __restrict__ W, int64_t ldw, int M, int K, int N_rt, bool sliced, int tpr,
                   int rows_per_cta, uint32_t* __restrict__ planes, float* __restrict__ alpha,
                   __half* __restrict__ alpha16) {
     __shared__ double red[2][32];
+    const int N = NPC > 0 ? NPC : N_rt;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int rl = tid / tpr, tr = tid - rl * tpr;
     const int row = blockIdx.x * rows_per_cta + rl;
@@ -352,7 +354,12 @@ cudaError_t launch_words(const PackArgs& a, cudaStream_t s) {
     // were 15 % slower on 11008 x 4096)
     const int rows_per_cta = tpr >= 128 ? 1 : 128 / tpr;
     const int64_t blocks = (a.M + rows_per_cta - 1) / rows_per_cta;
-    pack_words_kernel<WT><<<static_cast<unsigned>(blocks), rows_per_cta * tpr, 0, s>>>(
+    auto kern = a.n_paths == 1   ? pack_words_kernel<WT, 1>
+                : a.n_paths == 2 ? pack_words_kernel<WT, 2>
+                : a.n_paths == 3 ? pack_words_kernel<WT, 3>
+                : a.n_paths == 4 ? pack_words_kernel<WT, 4>
+                                 : pack_words_kernel<WT, 0>;
+    kern<<<static_cast<unsigned>(blocks), rows_per_cta * tpr, 0, s>>>(
         static_cast<const WT*>(a.W), a.ldw, static_cast<int>(a.M), static_cast<int>(a.K), a.n_paths, a.sliced, tpr,
         rows_per_cta, a.planes, a.alpha, a.alpha16);
     return cudaGetLastError();
