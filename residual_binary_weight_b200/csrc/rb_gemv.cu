@@ -332,6 +332,39 @@ __device__ __forceinline__ void scan_jobs(const GvArgs& p, LowSmem& lo, int n_jo
     cta_sync();
 }
 
+// A single matrix (descriptor in the kernel parameters, sliced planes):
+// bring the first two slices of this CTA's first unit into L2 with bulk
+// prefetches, so that their HBM reads overlap the end of the previous kernel
+// in the stream. A prefetch to L2 only moves lines into the point of
+// coherence and hands no data to the thread, so it may run before the
+// dependent-launch wait even if an earlier kernel still writes the planes.
+// The unit follows the numbering of decode_rec: (row block, chunk, token),
+// token fastest; units of token t > 0 read the planes of token 0's unit and
+// skip it.
+template <int R, int NP>
+__device__ __forceinline__ void prefetch_first_unit(const GvArgs& p) {
+    const int64_t M = p.one.M, K = p.one.K;
+    const uint32_t S = static_cast<uint32_t>(slices_of(K));
+    const uint32_t nch = (S + static_cast<uint32_t>(p.chunk_slices) - 1) / static_cast<uint32_t>(p.chunk_slices);
+    const uint64_t nrb = static_cast<uint64_t>((M + R - 1) / R);
+    const uint64_t u = blockIdx.x, T = static_cast<uint64_t>(p.T);
+    if (u >= nrb * nch * T || u % T != 0) return;
+    const uint64_t q = u / T;
+    const uint32_t ch = static_cast<uint32_t>(q % nch);
+    const uint64_t rb = q / nch;
+    const uint32_t s_begin = (ch * S) / nch, s_end = ((ch + 1) * S) / nch;
+    const uint32_t ns = min(2u, s_end - s_begin);
+    const uint64_t row0 = rb * R;
+    const uint32_t bytes = static_cast<uint32_t>(min(static_cast<uint64_t>(R), static_cast<uint64_t>(M) - row0)) * 64u;
+    const uint32_t i = threadIdx.x;
+    if (i < NP * ns) {
+        // sliced layout: path k, slice s, row m at ((k S + s) M + m) * 64 bytes
+        const uint64_t k = i / ns, s = s_begin + i % ns;
+        const char* a = reinterpret_cast<const char*>(p.one.planes) + ((k * S + s) * static_cast<uint64_t>(M) + row0) * 64u;
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a), "r"(bytes) : "memory");
+    }
+}
+
 // GATE: the SiLU-gated pair (GvArgs::swiglu), a separate instantiation so
 // that the plain kernel's epilogue carries none of it
 template <int NP, bool G128, bool A16, bool SLICED, bool GATE = false>
@@ -345,17 +378,31 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_lut_kernel(GvArgs p, uint32_t
 
     // Programmatic dependent launch: the next kernel of the stream may be
     // launched now (its CTAs start as this grid's CTAs leave their SMs and
-    // wait below until this grid has finished), and this grid waits here for
-    // the one before it: nothing above touches global memory.
+    // wait in join() until this grid has finished). join() waits for the
+    // kernel before this one. Everything before it reads only the kernel
+    // parameters and shared memory: the grouped descriptors are device
+    // memory, so a grouped call joins first; a single matrix scans its plan,
+    // decodes its first units and prefetches its first planes to L2 (a
+    // prefetch hands no data to the CTA) while the previous kernel ends.
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    // The call's error word is cleared here, not by a memset before the
-    // launch: every condition below is detected by every CTA, CTA 0
-    // included, after this store, so a flag another CTA raised before it is
-    // raised again.
-    if (blockIdx.x == 0 && threadIdx.x == 0) hdr[1] = 0u;
+    const bool single = p.jobs == nullptr;
+    if (SLICED && single) prefetch_first_unit<C::R, NP>(p);
+    // The call's error word is cleared in join(), not by a memset before
+    // the launch: every condition below is detected by every CTA, CTA 0
+    // included, after CTA 0's join, so a flag another CTA raised before the
+    // clear is raised again. Every global access and every return follows a
+    // join() (a second griddepcontrol.wait returns at once).
+    bool joined = false;
+    auto join = [&]() {
+        if (joined) return;
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        if (blockIdx.x == 0 && threadIdx.x == 0) hdr[1] = 0u;
+        joined = true;
+    };
+    if (!single) join();
     const uint32_t s0 = smem_addr(dsm);
     if (s0 + sizeof(LowSmem) > TBL0 || s0 + SMEM_BYTES < TBL0 + 2 * 0x10000u) {
+        join();
         if (threadIdx.x == 0) atomicOr(hdr + 1, GV_ERR_SMEM_LAYOUT);
         return;
     }
@@ -365,6 +412,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_lut_kernel(GvArgs p, uint32_t
     const int T = p.T;
     const int n_jobs = p.jobs ? p.n_jobs : 1;
     if (n_jobs > MAX_JOBS) {
+        join();
         if (tid == 0) atomicOr(hdr + 1, GV_ERR_TOO_MANY_JOBS);
         return;
     }
@@ -375,6 +423,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_lut_kernel(GvArgs p, uint32_t
     // counters and partial sums past the workspace)
     if (total_units != p.expect_units || lo.ctr_prefix[n_jobs] != p.expect_ctrs ||
         lo.part_prefix[n_jobs] != p.expect_parts) {
+        join();
         if (tid == 0) atomicOr(hdr + 1, GV_ERR_BAD_JOB);
         return;   // uniform: every thread read the same shared values
     }
@@ -398,7 +447,10 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_lut_kernel(GvArgs p, uint32_t
     // into the ring of unit records ahead of use
     const uint32_t G = gridDim.x, bid = blockIdx.x;
     const uint32_t n_my = total_units > bid ? (total_units - bid + G - 1) / G : 0u;
-    if (n_my == 0) return;   // uniform over the CTA
+    if (n_my == 0) {   // uniform over the CTA
+        join();
+        return;
+    }
     uint32_t decoded = 0;
     auto decode_upto = [&](uint32_t to) {
         for (uint32_t k = decoded + tid; k < to; k += THREADS)
@@ -407,6 +459,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_lut_kernel(GvArgs p, uint32_t
         cta_sync();
     };
     decode_upto(min(n_my, static_cast<uint32_t>(UCAP)));
+    join();
 
     // The step `d` steps after (unit k, slice s) in this CTA's sequence of
     // (unit, slice) steps; false past the last unit. Needs units up to k + d
