@@ -376,3 +376,37 @@ def test_a_counter_left_non_zero_is_reported():
         rb.gemv(planes, alpha, x, workspace=ws, check_device=True)
     ws.zero_()
     rb.gemv(planes, alpha, x, workspace=ws, check_device=True)
+
+
+@pytest.mark.parametrize("M,K,group", [(8192, 4096, 0), (700, 8192, 0), (1000, 4096, 128)])
+def test_planes_rewritten_by_pack_right_before_the_matvec(M, K, group):
+    """A single-matrix matvec is a dependent launch that starts while the
+    previous kernel of its stream runs, and brings its first planes into L2
+    before it waits for that kernel. An rb_pack that rewrites those very
+    planes just before it, with no synchronisation in between, must still be
+    seen: with two weights packed in turn into the same buffers, every
+    result equals the same call made after a device synchronise (the kernel
+    is deterministic, so bit for bit)."""
+    g = torch.Generator(device="cuda").manual_seed(M + K + group)
+    a16 = group == 128
+    Ws = [(torch.randn(M, K, device="cuda", generator=g) * 0.02).half() for _ in range(2)]
+    x = torch.randn(1, K, device="cuda", generator=g).half()
+    planes, alpha, al16 = rb.pack(Ws[0], 2, group, alpha_f16=a16, order="sliced")
+    sc = al16 if a16 else alpha
+    ws = torch.zeros(max(16, rb.gemv_workspace_bytes(M, K, 2, group, 1)), dtype=torch.uint8, device="cuda")
+    n = 6
+    ys = [torch.empty(1, M, dtype=torch.float16, device="cuda") for _ in range(n)]
+    torch.cuda.synchronize()
+    for i in range(n):   # pack, then matvec at once: adjacent kernels of one stream
+        rb.pack(Ws[i % 2], 2, group, alpha_f16=a16, order="sliced", planes=planes, alpha=alpha, alpha16=al16)
+        rb.gemv(planes, sc, x, group=group, y=ys[i], workspace=ws)
+    torch.cuda.synchronize()
+    ref = []
+    for w in range(2):
+        rb.pack(Ws[w], 2, group, alpha_f16=a16, order="sliced", planes=planes, alpha=alpha, alpha16=al16)
+        torch.cuda.synchronize()
+        ref.append(rb.gemv(planes, sc, x, group=group, workspace=ws, check_device=True))
+        torch.cuda.synchronize()
+    assert not torch.equal(ref[0], ref[1])
+    for i in range(n):
+        assert torch.equal(ys[i], ref[i % 2]), i
