@@ -231,7 +231,17 @@ pack_words_kernel(const WT* __restrict__ W, int64_t ldw, int M, int K, int N_rt,
             if (lane == 0) red[k & 1][warp] = sum;
             __syncthreads();
             sum = 0.0;
-            for (int w = 0; w < wpr; ++w) sum += red[k & 1][rl * wpr + w];
+            if (wpr > 8) {
+                // long rows: the row's partials as a shuffle tree (five
+                // levels instead of wpr dependent adds); a + b == b + a, so
+                // every lane ends with the same sum
+                double v = lane < wpr ? red[k & 1][rl * wpr + lane] : 0.0;
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(FULL_MASK, v, o);
+                sum = v;
+            } else {
+                for (int w = 0; w < wpr; ++w) sum += red[k & 1][rl * wpr + w];
+            }
         }
         // every lane of a row holds the same sum; one lane per warp divides
         float a = 0.0f;
