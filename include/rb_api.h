@@ -23,7 +23,12 @@
  *   the caller owns every buffer. Calls never allocate device memory.
  * - Every call that takes `stream` (a cudaStream_t, NULL for the legacy
  *   default stream) only enqueues work and returns; results are ready when the
- *   stream reaches that point.
+ *   stream reaches that point. Stream order holds for the inputs: a call sees
+ *   everything earlier work on the stream wrote. (The matvec and decode
+ *   kernels are programmatic dependent launches that start while the
+ *   previous kernel ends; before they wait for it they only set up, and a
+ *   single-matrix matvec prefetches its first planes into L2, which reads
+ *   no stale data.)
  * - Arguments are validated on the host before anything is enqueued; a call
  *   that returns an error has enqueued nothing, except where stated.
  * - Plane words: bit j of word w of a row holds column 32*w + j (least
